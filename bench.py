@@ -1,0 +1,474 @@
+"""Benchmark of the block-scaled FP8 hot path on B200.
+
+One step = one pass of the fine-grained FP8 GEMM workload: quantize the
+activations A [4096, 7168] (bf16 -> E4M3, fp32 scale per 1x128 tile),
+quantize the weights B [2048, 7168] (fp32 scale per 128x128 block), then
+C = A B^T with fp32 accumulation and bf16 output (120.3 GFLOP).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload ds_fp8_gemm|qat_forward|moe_grouped|moe_prequant|mxfp8_256x512]
+
+Prints one JSON line (rank 0).  `value` is whole-step throughput in TFLOP/s
+(GEMM flops of the step / step time, quantization included), with the
+inputs resident in HBM and L2 flushed (256 MiB write) before every step; the
+per-kernel times, the quantize GB/s and the roofline of the dominant kernel
+come from CUDA events on the launching stream.  With N > 1 (torchrun) every
+rank runs an independent replica (the path has no exchange step): the time
+is the max over ranks and `value` counts all ranks' work.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._nv:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "nvml" if self._nv else "unavailable"}
+
+
+# ------------------------------------------------------------------ workloads on the GPU
+
+class Step:
+    """A workload bound to device buffers; run() enqueues one step."""
+    name = ""
+    flops = 0.0
+    quant_bytes = 0.0
+    launches = 0
+    dominant = ""
+
+    def kernels(self):  # list of (label, callable)
+        raise NotImplementedError
+
+
+class DsFp8Gemm(Step):
+    name = "ds_fp8_gemm"
+    dominant = "gemm_fp8_f32scale"
+
+    def __init__(self, fpq, dev, m=4096, n=2048, k=7168):
+        self.f = fpq
+        self.m, self.n, self.k = m, n, k
+        wl = workloads.ds_fp8_gemm(m, n, k)
+        self.a_host, self.b_host = wl["a"].pin_memory(), wl["b"].pin_memory()
+        self.a, self.b = self.a_host.to(dev), self.b_host.to(dev)
+        f = fpq
+        self.qa = torch.empty((m, k), dtype=torch.uint8, device=dev)
+        self.sa = torch.empty((m, k // 128), dtype=torch.float32, device=dev)
+        self.qb = torch.empty((n, k), dtype=torch.uint8, device=dev)
+        self.sb = torch.empty(((n + 127) // 128, k // 128), dtype=torch.float32, device=dev)
+        self.c = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        self.c_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
+        self.flops = 2.0 * m * n * k
+        self.qa_bytes = m * k * (2 + 1) + m * (k // 128) * 4
+        self.qb_bytes = n * k * (2 + 1) + ((n + 127) // 128) * (k // 128) * 4
+        self.quant_bytes = self.qa_bytes + self.qb_bytes
+        self.launches = 3
+        self.config = {"workload": "ds_fp8_gemm: A bf16 4096x7168 N(0,1) -> E4M3 with fp32 scale per 1x128 tile; "
+                                   "B bf16 2048x7168 N(0,0.02) -> E4M3 with fp32 scale per 128x128 block; "
+                                   "C = A B^T fp32 accumulate, bf16 out",
+                       "m": m, "n": n, "k": k, "l2": "flushed before every step (256 MiB write)"}
+
+    def kernels(self):
+        f = self.f
+        return [
+            ("quant_fp8_1x128", lambda: f.fpq_quantize_block(f.FP8_1x128, self.a, 1, self.m, self.k, self.qa, self.sa)),
+            ("quant_fp8_128x128", lambda: f.fpq_quantize_block(f.FP8_128x128, self.b, 1, self.n, self.k, self.qb, self.sb)),
+            ("gemm_fp8_f32scale", lambda: f.fpq_scaled_gemm(f.FP8_1x128, self.qa, self.sa, f.FP8_128x128, self.qb,
+                                                            self.sb, self.m, self.n, self.k, self.c, f.OUT_BF16)),
+        ]
+
+    def kernel_work(self):
+        return {"quant_fp8_1x128": ("GB/s", self.qa_bytes), "quant_fp8_128x128": ("GB/s", self.qb_bytes),
+                "gemm_fp8_f32scale": ("TFLOP/s", self.flops)}
+
+    def e2e_step(self, stream):
+        """Host buffers in, host buffer out: the same step through the C ABI
+        with the copies inside the timed region."""
+        self.a.copy_(self.a_host, non_blocking=True)
+        self.b.copy_(self.b_host, non_blocking=True)
+        for _, fn in self.kernels():
+            fn()
+        self.c_host.copy_(self.c, non_blocking=True)
+        return self.a_host.numel() * 2 + self.b_host.numel() * 2, self.c.numel() * 2
+
+
+class MoeGrouped(Step):
+    name = "moe_grouped"
+    dominant = "gemm_grouped_mxfp8"
+
+    def __init__(self, fpq, dev):
+        self.f = fpq
+        wl = workloads.moe_grouped()
+        x_perm = wl["x"][wl["perm"]]
+        self.x = x_perm.to(dev)
+        self.offsets = wl["offsets"].to(dev)
+        self.w = wl["w"].to(dev)
+        self.wq, self.ws = fpq.quantize(self.w, fpq.MXFP8)      # weights are prequantized once (serving)
+        del self.w
+        self.total, self.k = self.x.shape
+        self.groups, self.n = self.wq.shape[0], self.wq.shape[1]
+        self.qx = torch.empty_like(self.x, dtype=torch.uint8)
+        self.sx = torch.empty((self.total, self.k // 32), dtype=torch.uint8, device=dev)
+        self.c = torch.empty((self.total, self.n), dtype=torch.bfloat16, device=dev)
+        self.flops = 2.0 * self.total * self.n * self.k
+        self.qx_bytes = self.total * self.k * 3 + self.total * self.k // 32
+        self.quant_bytes = self.qx_bytes
+        self.launches = 2
+        self.counts = np.diff(wl["offsets"].numpy()).tolist()
+        self.config = {"workload": "moe_grouped: X 16384x7168 N(0,1), top-8 of 64 experts (Zipf 1.1 Gumbel-top-8), "
+                                   "131072 permuted rows -> MXFP8; grouped GEMM with MXFP8 expert weights 64x2048x7168",
+                       "expert_rows_max": max(self.counts), "expert_rows_min": min(self.counts),
+                       "l2": "flushed before every step (256 MiB write)"}
+
+    def kernels(self):
+        f = self.f
+        return [
+            ("quant_mxfp8", lambda: f.fpq_quantize_block(f.MXFP8, self.x, 1, self.total, self.k, self.qx, self.sx)),
+            ("gemm_grouped_mxfp8", lambda: f.fpq_grouped_scaled_gemm(f.MXFP8, self.qx, self.sx, self.wq, self.ws,
+                                                                     self.offsets, self.groups, self.total, self.n,
+                                                                     self.k, self.c, f.OUT_BF16)),
+        ]
+
+    def kernel_work(self):
+        return {"quant_mxfp8": ("GB/s", self.qx_bytes), "gemm_grouped_mxfp8": ("TFLOP/s", self.flops)}
+
+
+class QatForward(Step):
+    name = "qat_forward"
+    dominant = "gemm_fp8_f32scale"
+
+    def __init__(self, fpq, dev):
+        self.f = fpq
+        wl = workloads.qat_forward()
+        self.w, self.la, self.lb, self.x = (wl[t].to(dev) for t in ("w", "lora_a", "lora_b", "x"))
+        self.aor = wl["alpha_over_r"]
+        self.n, self.k = self.w.shape
+        self.m = self.x.shape[0]
+        self.wq = torch.empty((self.n, self.k), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty((self.n // 128, self.k // 128), dtype=torch.float32, device=dev)
+        self.xq = torch.empty((self.m, self.k), dtype=torch.uint8, device=dev)
+        self.xs = torch.empty((self.m, self.k // 128), dtype=torch.float32, device=dev)
+        self.c = torch.empty((self.m, self.n), dtype=torch.bfloat16, device=dev)
+        self.flops = 2.0 * self.m * self.n * self.k
+        self.merge_bytes = self.n * self.k * 3 + (self.la.numel() + self.lb.numel()) * 2
+        self.xq_bytes = self.m * self.k * 3 + self.m * (self.k // 128) * 4
+        self.quant_bytes = self.merge_bytes + self.xq_bytes
+        self.launches = 3
+        self.config = {"workload": "qat_forward: merge W 2048x7168 + (32/16) B A (r=16) -> 128x128 FP8 fake-quant; "
+                                   "X 8192x7168 -> 1x128 FP8; C = X W_eff^T", "l2": "flushed before every step"}
+
+    def kernels(self):
+        f = self.f
+        return [
+            ("lora_merge_fq", lambda: f.fpq_lora_merge_fakequant(self.w, self.la, self.lb, self.n, self.k, 16, self.aor,
+                                                                 self.wq, self.ws)),
+            ("quant_fp8_1x128", lambda: f.fpq_quantize_block(f.FP8_1x128, self.x, 1, self.m, self.k, self.xq, self.xs)),
+            ("gemm_fp8_f32scale", lambda: f.fpq_scaled_gemm(f.FP8_1x128, self.xq, self.xs, f.FP8_128x128, self.wq,
+                                                            self.ws, self.m, self.n, self.k, self.c, f.OUT_BF16)),
+        ]
+
+    def kernel_work(self):
+        return {"lora_merge_fq": ("GB/s", self.merge_bytes), "quant_fp8_1x128": ("GB/s", self.xq_bytes),
+                "gemm_fp8_f32scale": ("TFLOP/s", self.flops)}
+
+
+STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": QatForward}
+
+
+# ------------------------------------------------------------------ traffic from committed ncu summaries
+
+def _source_hash(kernel: str) -> str | None:
+    src = {"gemm_fp8_f32scale": "gemm_fp8_f32scale.cu", "gemm_grouped_mxfp8": "gemm_mxfp8.cu",
+           "gemm_mxfp8": "gemm_mxfp8.cu", "quant_fp8_1x128": "quant_kernels.cu",
+           "quant_mxfp8": "quant_kernels.cu", "lora_merge_fq": "merge_kernel.cu"}.get(kernel)
+    if not src:
+        return None
+    with open(os.path.join(ROOT, "mxfp8_block_scaled_warp_b200", "csrc", src), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch recorded in profiles/<kernel>__<workload>.md
+    ('dram_bytes_per_launch: X' and 'source_sha256_16: H'); null when absent
+    or when the kernel's source has changed since the capture."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.md")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    if not b or not h or h.group(1) != _source_hash(kernel):
+        return None
+    return float(b.group(1))
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+
+def cpu_baseline(workload: str, budget_s: float = 12.0):
+    """Time the oracle (as it stands, single thread) on a bounded sample of
+    the workload and extrapolate to the whole step in TFLOP/s."""
+    import oracle
+    oracle.build()
+    if workload != "ds_fp8_gemm":
+        return None
+    m, n, k = 4096, 2048, 7168
+    wl = workloads.ds_fp8_gemm(m, n, k)
+    a, b = workloads.as_u16(wl["a"]), workloads.as_u16(wl["b"])
+    t0 = time.perf_counter()
+    rows_a = 64
+    qa, sa = oracle.quant_fp8_1x128(a[:rows_a])
+    t_qa = (time.perf_counter() - t0) / (rows_a * k)
+    t0 = time.perf_counter()
+    qb, sb = oracle.quant_fp8_128x128(b[:256])
+    t_qb = (time.perf_counter() - t0) / (256 * k)
+    # GEMM entries: calibrate, then fill the remaining budget
+    spent = (t_qa * rows_a + t_qb * 256) * k
+    probe = 64
+    rr = np.arange(probe) % rows_a
+    cc = np.arange(probe) % 256
+    t0 = time.perf_counter()
+    oracle.gemm_entries(0, qa, sa, 1, qb, sb, rr, cc)
+    per = (time.perf_counter() - t0) / probe
+    count = int(max(probe, min(200000, (budget_s - spent) / max(per, 1e-9))))
+    rng = np.random.default_rng(0)
+    rr, cc = rng.integers(0, rows_a, count), rng.integers(0, 256, count)
+    t0 = time.perf_counter()
+    oracle.gemm_entries(0, qa, sa, 1, qb, sb, rr, cc)
+    per = (time.perf_counter() - t0) / count
+    step_s = t_qa * m * k + t_qb * n * k + per * m * n
+    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"1x128 quantize of {rows_a} rows and 128x128 quantize of 256 rows of the 7168-wide "
+                      f"operands, {count} fp64 GEMM entries (K=7168); extrapolated to the full 4096x2048x7168 "
+                      f"step ({step_s:.1f} s per step on one core)"}
+
+
+# ------------------------------------------------------------------ main
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle timed as it stands."""
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline(args.workload, budget_s=1.0)
+    t_total = 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        r = cpu_baseline(args.workload, budget_s=3.0)
+        t_total += time.perf_counter() - t0
+        vals.append(r["value"])
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 2.0 * 4096 * 2048 * 7168 / (v * 1e12) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": r["sample"]},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+METRIC = "quantize GB/s vs HBM peak; block-scaled FP8 GEMM TFLOPS vs FP8 tensor peak"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fpq", choices=["fpq", "reference"])
+    ap.add_argument("--workload", default="ds_fp8_gemm", choices=sorted(STEPS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import mxfp8_block_scaled_warp_b200 as fpq
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    step = STEPS[args.workload](fpq, dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    kern = step.kernels()
+    names = [n for n, _ in kern]
+
+    def one_step(events=None):
+        for i, (_, fn) in enumerate(kern):
+            if events is not None:
+                events[i][0].record(stream)
+            fn()
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step()
+    torch.cuda.synchronize()
+    assert fpq.fpq_get_device_error() == 0
+
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in kern] for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            one_step(ev[s])
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    status = fpq.fpq_get_device_error()
+    if status != 0:
+        raise SystemExit(f"device error word {status} after the timed steps")
+
+    per_kernel = {n: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i, n in enumerate(names)}
+    step_ms = [ev[s][0][0].elapsed_time(ev[s][-1][1]) for s in range(args.steps)]
+    total_ms = sum(step_ms)
+    if pg:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * step.flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    peaks = _peaks()
+    fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
+    kernels_out = {}
+    for n in names:
+        unit, work = step.kernel_work()[n]
+        ms = statistics.mean(per_kernel[n])
+        ach = work / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+        pk = peaks["hbm_gbs"] if unit == "GB/s" else fp8_peak_burst
+        kernels_out[n] = {"ms": ms, "achieved": ach, "unit": unit, "frac_of_peak": ach / pk}
+    dom = kernels_out[step.dominant]
+    traffic = _traffic(step.dominant, step.name)
+    roofline = {"kernel": step.dominant, "bound": "tensor", "achieved": dom["achieved"], "peak": fp8_peak_burst,
+                "unit": "TFLOP/s", "frac": dom["achieved"] / fp8_peak_burst, "traffic": traffic,
+                "peak_note": f"fp8 = 2 x {peaks['source']} cuBLAS bf16 burst ({peaks['bf16_tflops']} TFLOP/s)"}
+    quant_ms = sum(statistics.mean(per_kernel[n]) for n in names if not n.startswith("gemm"))
+    quant_gbs = step.quant_bytes / (quant_ms * 1e-3) / 1e9
+
+    # end to end: host buffers through the public API, copies inside the timed region
+    e2e = None
+    if hasattr(step, "e2e_step"):
+        for _ in range(2):
+            step.e2e_step(stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(3, min(args.steps, 20))
+        e0.record(stream)
+        for _ in range(reps):
+            hb, db = step.e2e_step(stream)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / reps
+        if pg:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * step.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": hb,
+               "d2h_bytes_per_step": db, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(step.name)
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3xe4m3->f32 (bf16 in/out)", "data": "synthetic",
+            "config": step.config, "quantize_gbs": quant_gbs, "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"],
+            "kernels": kernels_out, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": step.launches * args.steps, "clocks": clk.summary(),
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp8_tflops": fp8_peak_burst, "source": peaks["source"]}}
+    if rank == 0:
+        print(json.dumps(line))
+    if pg:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

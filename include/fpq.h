@@ -1,0 +1,228 @@
+/*
+ * fpq.h -- C ABI of the B200 (sm_100a) library for fine-grained block-scaled
+ * low-precision quantization and the block-scaled matmul that consumes it.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All data pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or keeps them past the call; it enqueues kernels
+ *    on `stream` (a cudaStream_t passed as void*, NULL = the legacy default
+ *    stream) and returns without synchronizing.  The caller must keep every
+ *    buffer alive until the stream has passed the enqueued work.
+ *  - Tensors are dense and row-major; batched tensors are batch-major with
+ *    no padding ([batch][rows][cols]).  bf16 values are raw 16-bit patterns.
+ *  - Every pointer must be 16-byte aligned.
+ *  - Scales are DEQUANTIZATION MULTIPLIERS ("scale inverse"): an element's
+ *    value is approximately decode(code) * scale.
+ *  - Return values are synchronous status codes (fpq_status).  On any error
+ *    nothing is enqueued.  FPQ_ERR_CUDA carries the CUDA error text in
+ *    fpq_last_error_detail() (per thread).  Faults detected inside a kernel
+ *    (a bounded wait that ran out, a malformed group offset list) are written
+ *    to a device-side error word read by fpq_get_device_error().
+ *  - There is no CPU fallback: a missing or non-sm_100 device gives
+ *    FPQ_ERR_UNSUPPORTED.
+ *
+ * Numerics (all formats): round-to-nearest-even, E4M3 saturating to +-448,
+ * E2M1 saturating to +-6, IEEE fp32 arithmetic with gradual underflow.
+ * Element encodings are those of the OCP Microscaling (MX) v1.0 formats.
+ *
+ * Sources (web pages, cited by title and section):
+ *  [FP]  "fireworks-prequant 0.1.0" (PyPI): "Formats" (mxfp8 = 1x32 block
+ *        FP8 with E8M0 scales; nvfp4 = packed FP4 with FP8 block scales) and
+ *        "Quick start" (float8_e4m3fn weight + uint8 E8M0 weight_scale_inv;
+ *        only routed MoE expert projections are quantized).
+ *  [DS]  "FP8 в DeepSeek V3: как низкая точность ускоряет обучение и
+ *        инференс": "Как FP8 встроен в DeepSeek V3" (online
+ *        per-token-per-128-channel activation quantization), "Почему обычное
+ *        округление не подходит" (128x128 weight blocks, scale inverse for
+ *        dequantization), "Инференс с FP8" (activation quantization, weight
+ *        dequantization and FP8 matmul kernels).
+ *  [B5]  "DeepSeek-V3 Blog 5: Low-Precision Training -- The FP8 Revolution":
+ *        "The Solution: Block-Wise Quantization", "Hardware Optimization"
+ *        (FP8 products promoted to higher precision before accumulation).
+ *  [QAT] "DeepSeek R1 and V3 get quantization-aware fine-tuning on
+ *        Fireworks": "Synopsis"/"Interpretation" (LoRA merged into the base
+ *        weight, merged bf16 weight converted to block-wise FP8, forward
+ *        pass fake-quantizes merged weights and activations).
+ */
+#ifndef FPQ_H
+#define FPQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FPQ_API __attribute__((visibility("default")))
+#else
+#define FPQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t fpq_status;
+enum {
+    FPQ_OK = 0,
+    FPQ_ERR_INVALID_ARG = 1,     /* null pointer, bad shape, bad enum value     */
+    FPQ_ERR_ALIGNMENT = 2,       /* a pointer is not 16-byte aligned            */
+    FPQ_ERR_UNSUPPORTED = 3,     /* no sm_100 device, or format pair not built  */
+    FPQ_ERR_CUDA = 4,            /* a CUDA call failed (see detail string)      */
+    FPQ_ERR_DEVICE_TIMEOUT = 5,  /* device error word: a bounded wait ran out   */
+    FPQ_ERR_DEVICE_BAD_INPUT = 6,/* device error word: malformed device input   */
+    FPQ_ERR_WORKSPACE = 7        /* workspace missing or too small              */
+};
+
+/* Block formats (fpq_format). */
+typedef int32_t fpq_format;
+enum {
+    /* FP8-E4M3, one fp32 scale per 1x128 tile of a row (activations) [DS].
+     * codes uint8 [B,R,C]; scales fp32 [B,R,C/128]; C % 128 == 0.
+     * s = fp32(amax/448) (1.0 for an all-zero tile); q = E4M3(fp32(x / s)). */
+    FPQ_FP8_1x128 = 0,
+    /* FP8-E4M3, one fp32 scale per 128x128 block (weights) [DS].
+     * codes uint8 [B,R,C]; scales fp32 [B,ceil(R/128),C/128]; C % 128 == 0;
+     * the last block row may be short.  Same s and q rule as FPQ_FP8_1x128. */
+    FPQ_FP8_128x128 = 1,
+    /* MXFP8: FP8-E4M3, one E8M0 scale per 1x32 block of a row [FP].
+     * codes uint8 [B,R,C]; scales uint8 [B,R,C/32]; C % 32 == 0.
+     * e = clamp(ceil(log2(amax/448)), -127, 127), scale code e + 127,
+     * q = E4M3(x * 2^-e) (exact scaling; no element saturates). */
+    FPQ_MXFP8 = 2,
+    /* NVFP4: E2M1 packed two per byte (element 2i in the low nibble), one
+     * E4M3 scale per 1x16 block, one fp32 tensor scale g per batch item [FP].
+     * codes uint8 [B,R,C/2]; scales uint8 [B,R,C/16]; g fp32 [B]; C % 32 == 0.
+     * g = fp32(amax_T/2688) (1 for an all-zero tensor),
+     * s_b = E4M3(fp32(fp32(amax_b/6)/g)), S = fp32(dec(s_b)*g),
+     * q = E2M1(fp32(x/S)) (all zero when S == 0). */
+    FPQ_NVFP4 = 3
+};
+
+/* GEMM output element type. */
+enum { FPQ_OUT_BF16 = 0, FPQ_OUT_F32 = 1 };
+
+/* Version of this ABI: major * 10000 + minor * 100 + patch. */
+FPQ_API int32_t fpq_version(void);
+
+/* Static text for a status code. */
+FPQ_API const char* fpq_status_string(fpq_status status);
+
+/* Detail of the last failing call on this host thread ("" if none). */
+FPQ_API const char* fpq_last_error_detail(void);
+
+/* Bytes of device workspace fpq_quantize_block needs for `fmt` and `batch`
+ * (NVFP4: 4 bytes per batch item for the tensor amax; 0 otherwise). */
+FPQ_API size_t fpq_quantize_workspace_bytes(fpq_format fmt, int64_t batch);
+
+/*
+ * fpq_quantize_block -- block-wise quantization of bf16 to FP8/FP4 with
+ * per-block scales [B5 "The Solution: Block-Wise Quantization"; DS; FP].
+ *
+ *   x              bf16 [batch, rows, cols] (input, read only)
+ *   q              codes, layout of `fmt` (output)
+ *   scales         block scales, layout of `fmt` (output)
+ *   tensor_scale   NVFP4 only: fp32 g per batch item (output); NULL otherwise
+ *   workspace      NVFP4 only: >= fpq_quantize_workspace_bytes() bytes of
+ *                  device memory, contents overwritten; NULL otherwise
+ *
+ * Outputs are bit-identical for any stream, batch split and launch history.
+ * Errors: FPQ_ERR_INVALID_ARG (null pointer, batch/rows/cols < 1, cols not a
+ * multiple of the format's block), FPQ_ERR_ALIGNMENT, FPQ_ERR_WORKSPACE,
+ * FPQ_ERR_UNSUPPORTED, FPQ_ERR_CUDA.
+ */
+FPQ_API fpq_status fpq_quantize_block(fpq_format fmt, const void* x, int64_t batch, int64_t rows,
+                              int64_t cols, void* q, void* scales, float* tensor_scale,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fpq_dequantize -- out = bf16(fp32(decode(q) * scale)) per element, the
+ * "scale inverse" dequantization [DS "Почему обычное округление не подходит";
+ * "Практический смысл для инференс-инфраструктуры" (conversion to BF16)].
+ * For NVFP4 the scale is S = fp32(dec(s_b) * g).
+ *
+ *   q, scales, tensor_scale   as produced by fpq_quantize_block
+ *   out                       bf16 [batch, rows, cols] (output)
+ *
+ * Errors: as fpq_quantize_block.
+ */
+FPQ_API fpq_status fpq_dequantize(fpq_format fmt, const void* q, const void* scales,
+                          const float* tensor_scale, int64_t batch, int64_t rows,
+                          int64_t cols, void* out, void* stream);
+
+/*
+ * fpq_lora_merge_fakequant -- the weight side of the QAT forward [QAT]:
+ *   delta[n,k] = sum_{j<r} B[n,j] * A[j,k]   (fp32, fused multiply-adds,
+ *                                              j ascending, from zero)
+ *   W_eff[n,k] = bf16(fma(alpha_over_r, delta[n,k], W[n,k]))
+ * then W_eff is quantized with 128x128 blocks (FPQ_FP8_128x128 rules).
+ *
+ *   w        bf16 [n, k] base weight (out_features x in_features)
+ *   lora_a   bf16 [r, k]
+ *   lora_b   bf16 [n, r]
+ *   wq       uint8 e4m3 [n, k] (output)
+ *   ws       fp32 [ceil(n/128), k/128] (output)
+ *   w_fq     bf16 [n, k] fake-quantized weight dequant(wq, ws) (optional
+ *            output for an autograd caller; NULL skips it)
+ *
+ * Requires k % 128 == 0, 1 <= r <= 64.  Errors: as fpq_quantize_block.
+ */
+FPQ_API fpq_status fpq_lora_merge_fakequant(const void* w, const void* lora_a, const void* lora_b,
+                                    int64_t n, int64_t k, int32_t r, float alpha_over_r,
+                                    void* wq, float* ws, void* w_fq, void* stream);
+
+/*
+ * fpq_scaled_gemm -- C = A * B^T on block-quantized operands with fp32
+ * accumulation [B5 "Hardware Optimization"; DS "Инференс с FP8" (FP8
+ * matrix multiplication)]:
+ *   C[m,n] = sum_k decA[m,k] * decB[n,k],  dec = decode(code) * block scale.
+ *
+ *   aq, as   A [m, k] codes and scales in format fmt_a
+ *   bq, bs   B [n, k] codes and scales in format fmt_b (weights, K-major)
+ *   c        [m, n] bf16 (FPQ_OUT_BF16, round-to-nearest-even) or fp32
+ *
+ * Supported pairs: (FPQ_MXFP8, FPQ_MXFP8) -- the block-scaled tensor-core
+ * path; (FPQ_FP8_1x128, FPQ_FP8_128x128) -- per-128-K partial sums promoted
+ * to fp32 with the product of the two scales.  Others: FPQ_ERR_UNSUPPORTED.
+ * Requires k % 128 == 0, n % 16 == 0, m >= 1.
+ */
+FPQ_API fpq_status fpq_scaled_gemm(fpq_format fmt_a, const void* aq, const void* as,
+                           fpq_format fmt_b, const void* bq, const void* bs,
+                           int64_t m, int64_t n, int64_t k, void* c, int32_t c_dtype,
+                           void* stream);
+
+/*
+ * fpq_grouped_scaled_gemm -- per-expert product over a token-permuted
+ * activation matrix (MoE routed experts) [FP "Quick start": routed MoE
+ * expert projections; DS "Как FP8 связан с MoE-архитектурой DeepSeek V3"]:
+ *   for every expert g and row m in [off[g], off[g+1]):
+ *     C[m, :] = A[m, :] * B[g]^T
+ *
+ *   aq, as          A [total_m, k] codes/scales (fmt)
+ *   bq, bs          B [groups, n, k] codes/scales (fmt)
+ *   group_offsets   DEVICE int32 [groups + 1], off[0] = 0, non-decreasing,
+ *                   off[groups] = total_m (empty experts are legal);
+ *                   a violation is reported through the device error word
+ *                   (FPQ_ERR_DEVICE_BAD_INPUT) and C is left unspecified
+ *   c               [total_m, n] bf16 or fp32
+ *
+ * Supported: fmt = FPQ_MXFP8.  Requires k % 128 == 0, n % 16 == 0.
+ */
+FPQ_API fpq_status fpq_grouped_scaled_gemm(fpq_format fmt, const void* aq, const void* as,
+                                   const void* bq, const void* bs,
+                                   const int32_t* group_offsets, int32_t groups,
+                                   int64_t total_m, int64_t n, int64_t k, void* c,
+                                   int32_t c_dtype, void* stream);
+
+/*
+ * fpq_get_device_error -- synchronize `stream`, then read and clear the
+ * current device's error word.  *code receives FPQ_OK or the first
+ * FPQ_ERR_DEVICE_* raised by a kernel since the last read.  Returns
+ * FPQ_ERR_CUDA if the synchronization itself fails.
+ */
+FPQ_API fpq_status fpq_get_device_error(void* stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FPQ_H */

@@ -1,0 +1,220 @@
+"""Block-scaled FP8/FP4 quantization and block-scaled GEMM for B200 (sm_100a).
+
+A thin ctypes binding over ``libfpq.so`` (C ABI: ``include/fpq.h``).  Every
+step of the computation runs in the library's CUDA kernels; this module only
+checks and marshals torch tensors (device memory, streams) into the C calls.
+There is no CPU fallback: importing fails loudly when ``libfpq.so`` is missing
+(build it with ``python -m mxfp8_block_scaled_warp_b200.build``), and every
+call fails with FPQ_ERR_UNSUPPORTED on a device that is not sm_100.
+
+The ``fpq_*`` functions mirror the C entry points one to one (tensors in
+place of pointers, the current torch stream by default).  ``quantize``,
+``dequantize``, ``lora_merge_fakequant``, ``scaled_gemm`` and
+``grouped_scaled_gemm`` are conveniences that allocate the outputs with
+torch and call them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "FP8_1x128", "FP8_128x128", "MXFP8", "NVFP4", "OUT_BF16", "OUT_F32", "FpqError", "lib_path",
+    "fpq_version", "fpq_quantize_workspace_bytes", "fpq_quantize_block", "fpq_dequantize",
+    "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_grouped_scaled_gemm", "fpq_get_device_error",
+    "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "grouped_scaled_gemm",
+    "scale_shape", "code_shape",
+]
+
+FP8_1x128, FP8_128x128, MXFP8, NVFP4 = 0, 1, 2, 3
+OUT_BF16, OUT_F32 = 0, 1
+STATUS = {0: "FPQ_OK", 1: "FPQ_ERR_INVALID_ARG", 2: "FPQ_ERR_ALIGNMENT", 3: "FPQ_ERR_UNSUPPORTED",
+          4: "FPQ_ERR_CUDA", 5: "FPQ_ERR_DEVICE_TIMEOUT", 6: "FPQ_ERR_DEVICE_BAD_INPUT",
+          7: "FPQ_ERR_WORKSPACE"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libfpq.so")
+
+
+class FpqError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({detail})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(lib_path):
+        raise ImportError(f"{lib_path} is not built; run `python -m mxfp8_block_scaled_warp_b200.build`")
+    L = ctypes.CDLL(lib_path)
+    P, I64, I32, F, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "fpq_version": (I32, []),
+        "fpq_status_string": (ctypes.c_char_p, [I32]),
+        "fpq_last_error_detail": (ctypes.c_char_p, []),
+        "fpq_quantize_workspace_bytes": (SZ, [I32, I64]),
+        "fpq_quantize_block": (I32, [I32, P, I64, I64, I64, P, P, P, P, SZ, P]),
+        "fpq_dequantize": (I32, [I32, P, P, P, I64, I64, I64, P, P]),
+        "fpq_lora_merge_fakequant": (I32, [P, P, P, I64, I64, I32, F, P, P, P, P]),
+        "fpq_scaled_gemm": (I32, [I32, P, P, I32, P, P, I64, I64, I64, P, I32, P]),
+        "fpq_grouped_scaled_gemm": (I32, [I32, P, P, P, P, P, I32, I64, I64, I64, P, I32, P]),
+        "fpq_get_device_error": (I32, [P, ctypes.POINTER(I32)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype, fn.argtypes = res, args
+    return L
+
+
+_lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise FpqError(status, where, _lib.fpq_last_error_detail().decode(errors="replace"))
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the library must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+# ---------------------------------------------------------------- raw C entry points
+
+def fpq_version() -> int:
+    return _lib.fpq_version()
+
+
+def fpq_quantize_workspace_bytes(fmt: int, batch: int) -> int:
+    return _lib.fpq_quantize_workspace_bytes(fmt, batch)
+
+
+def fpq_quantize_block(fmt, x, batch, rows, cols, q, scales, tensor_scale=None, workspace=None, stream=None):
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.fpq_quantize_block(fmt, _ptr(x), batch, rows, cols, _ptr(q), _ptr(scales), _ptr(tensor_scale),
+                                   _ptr(workspace), wsb, _stream(stream)), "fpq_quantize_block")
+
+
+def fpq_dequantize(fmt, q, scales, tensor_scale, batch, rows, cols, out, stream=None):
+    _check(_lib.fpq_dequantize(fmt, _ptr(q), _ptr(scales), _ptr(tensor_scale), batch, rows, cols, _ptr(out),
+                               _stream(stream)), "fpq_dequantize")
+
+
+def fpq_lora_merge_fakequant(w, lora_a, lora_b, n, k, r, alpha_over_r, wq, ws, w_fq=None, stream=None):
+    _check(_lib.fpq_lora_merge_fakequant(_ptr(w), _ptr(lora_a), _ptr(lora_b), n, k, r, float(alpha_over_r),
+                                         _ptr(wq), _ptr(ws), _ptr(w_fq), _stream(stream)),
+           "fpq_lora_merge_fakequant")
+
+
+def fpq_scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, m, n, k, c, c_dtype, stream=None):
+    _check(_lib.fpq_scaled_gemm(fmt_a, _ptr(aq), _ptr(as_), fmt_b, _ptr(bq), _ptr(bs), m, n, k, _ptr(c), c_dtype,
+                                _stream(stream)), "fpq_scaled_gemm")
+
+
+def fpq_grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, groups, total_m, n, k, c, c_dtype, stream=None):
+    _check(_lib.fpq_grouped_scaled_gemm(fmt, _ptr(aq), _ptr(as_), _ptr(bq), _ptr(bs), _ptr(group_offsets), groups,
+                                        total_m, n, k, _ptr(c), c_dtype, _stream(stream)),
+           "fpq_grouped_scaled_gemm")
+
+
+def fpq_get_device_error(stream=None) -> int:
+    code = ctypes.c_int32(0)
+    _check(_lib.fpq_get_device_error(_stream(stream), ctypes.byref(code)), "fpq_get_device_error")
+    return code.value
+
+
+# ---------------------------------------------------------------- allocating conveniences
+
+def code_shape(fmt: int, shape) -> tuple:
+    *lead, cols = shape
+    return tuple(lead) + ((cols // 2,) if fmt == NVFP4 else (cols,))
+
+
+def scale_shape(fmt: int, shape) -> tuple:
+    *lead, rows, cols = shape
+    if fmt == FP8_1x128:
+        return tuple(lead) + (rows, cols // 128)
+    if fmt == FP8_128x128:
+        return tuple(lead) + ((rows + 127) // 128, cols // 128)
+    if fmt == MXFP8:
+        return tuple(lead) + (rows, cols // 32)
+    if fmt == NVFP4:
+        return tuple(lead) + (rows, cols // 16)
+    raise ValueError(f"unknown format {fmt}")
+
+
+def _scale_dtype(fmt):
+    return torch.float32 if fmt in (FP8_1x128, FP8_128x128) else torch.uint8
+
+
+def _brc(shape):
+    if len(shape) == 2:
+        return 1, shape[0], shape[1]
+    if len(shape) == 3:
+        return shape
+    raise ValueError("expected a 2-D or 3-D tensor")
+
+
+def quantize(x: torch.Tensor, fmt: int, stream=None):
+    """bf16 [(B,) R, C] -> (codes, scales[, tensor_scale]) in the layouts of include/fpq.h."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError("quantize expects bf16 input")
+    b, r, c = _brc(x.shape)
+    q = torch.empty(code_shape(fmt, x.shape), dtype=torch.uint8, device=x.device)
+    s = torch.empty(scale_shape(fmt, x.shape), dtype=_scale_dtype(fmt), device=x.device)
+    if fmt == NVFP4:
+        g = torch.empty((b,), dtype=torch.float32, device=x.device)
+        ws = torch.empty((max(1, fpq_quantize_workspace_bytes(fmt, b)) + 15) // 16 * 16, dtype=torch.uint8,
+                         device=x.device)
+        fpq_quantize_block(fmt, x, b, r, c, q, s, g, ws, stream)
+        return q, s, g
+    fpq_quantize_block(fmt, x, b, r, c, q, s, None, None, stream)
+    return q, s
+
+
+def dequantize(fmt: int, q: torch.Tensor, s: torch.Tensor, tensor_scale: torch.Tensor | None = None, stream=None):
+    shape = tuple(q.shape[:-1]) + ((q.shape[-1] * 2,) if fmt == NVFP4 else (q.shape[-1],))
+    b, r, c = _brc(shape)
+    out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
+    fpq_dequantize(fmt, q, s, tensor_scale, b, r, c, out, stream)
+    return out
+
+
+def lora_merge_fakequant(w, lora_a, lora_b, alpha_over_r: float, want_fq: bool = False, stream=None):
+    n, k = w.shape
+    r = lora_a.shape[0]
+    wq = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    ws = torch.empty(((n + 127) // 128, k // 128), dtype=torch.float32, device=w.device)
+    w_fq = torch.empty((n, k), dtype=torch.bfloat16, device=w.device) if want_fq else None
+    fpq_lora_merge_fakequant(w, lora_a, lora_b, n, k, r, alpha_over_r, wq, ws, w_fq, stream)
+    return (wq, ws, w_fq) if want_fq else (wq, ws)
+
+
+def scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, out_dtype=torch.bfloat16, stream=None):
+    m, k = aq.shape
+    n = bq.shape[0]
+    c = torch.empty((m, n), dtype=out_dtype, device=aq.device)
+    fpq_scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, m, n, k, c, OUT_F32 if out_dtype == torch.float32 else OUT_BF16,
+                    stream)
+    return c
+
+
+def grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, out_dtype=torch.bfloat16, stream=None):
+    total_m, k = aq.shape
+    groups, n, _ = bq.shape
+    c = torch.empty((total_m, n), dtype=out_dtype, device=aq.device)
+    fpq_grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, groups, total_m, n, k, c,
+                            OUT_F32 if out_dtype == torch.float32 else OUT_BF16, stream)
+    return c

@@ -1,0 +1,116 @@
+// common.cuh -- device helpers shared by the sm_100a kernels: element
+// conversions through the hardware cvt instructions, bf16 bit handling,
+// the device error word, vector memory access.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/fpq.h"
+
+namespace fpq {
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// ----------------------------------------------------------------- errors
+
+// Record the first device-side error; later ones are dropped.
+__device__ __forceinline__ void raise_device_error(uint32_t* err, uint32_t code) {
+    if (err) atomicCAS(err, 0u, code);
+}
+
+// ----------------------------------------------------------------- bf16
+
+// bf16 pattern -> fp32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// fp32 -> bf16 pattern, round to nearest even (hardware cvt, gradual underflow).
+__device__ __forceinline__ uint32_t f32_to_bf16(float f) {
+    uint16_t h;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(f));
+    return h;
+}
+// two fp32 -> packed bf16x2, `lo` in the low half
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ----------------------------------------------------------------- e4m3 / e2m1
+
+// two fp32 -> two E4M3 codes, round to nearest even, finite values saturate
+// to +-448; `lo` lands in bits 0..7.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// two fp32 -> two E2M1 codes in one byte, round to nearest even, saturating
+// to +-6; `lo` lands in bits 0..3.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// E4M3 code (low byte of `c`) -> fp32, exact (through the f16x2 converter).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)(c & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// two E4M3 codes (bits 0..15) -> two fp32, exact.
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t c2) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)(c2 & 0xFFFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return make_float2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))),
+                       __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+}
+
+// two E2M1 codes (bits 0..7, element 0 in bits 0..3) -> two fp32, exact.
+__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t c2) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.u8.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h2) : "r"(c2 & 0xFFu));
+    return make_float2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))),
+                       __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+}
+
+// ----------------------------------------------------------------- absmax
+
+// Largest magnitude pattern of the two bf16 halves of each word, as a packed
+// pair of 15-bit magnitudes (integer order = magnitude order for finite
+// values; NaN patterns order above infinity, so a NaN propagates).
+__device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7FFF7FFFu; }
+__device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) { return __vmaxu2(a, b); }
+__device__ __forceinline__ uint32_t hmax2(uint32_t a) { return max(a & 0xFFFFu, a >> 16); }
+
+// ----------------------------------------------------------------- memory
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void st_v2(void* p, uint2 v) {
+    asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+}  // namespace fpq

@@ -1,0 +1,334 @@
+// gemm_mxfp8.cu -- block-scaled MXFP8 GEMM on the 5th-generation tensor
+// cores: C = A * B^T with A [M, K], B [N, K] E4M3 codes and one E8M0 scale
+// per 32 K-elements of every row of A and of B, fp32 accumulation in TMEM,
+// bf16 (round-to-nearest-even) or fp32 output.  The same kernel serves the
+// grouped (per-expert) product, where row ranges of A select the expert
+// weight B[g].
+//
+// Per CTA one 128 x 256 output tile; the K loop runs over 128-wide K tiles
+// through a STAGES-deep shared-memory ring.  Warp roles:
+//   warp 0  TMA producer: A and B tiles (128-byte swizzle, no multicast)
+//   warp 1  scale-factor loader: gathers the row-major E8M0 scales of the
+//           tile's 128 A rows and 256 B rows into the 32x4x4 chunk layout the
+//           shared->TMEM copy expects (rows r, r+32, r+64, r+96 interleaved)
+//   warp 2  TMEM allocator and MMA issuer (one elected thread):
+//           tcgen05.cp of the scales, then 4 x tcgen05.mma kind::mxf8f6f4
+//           (K = 32 each, scale byte selected per MMA), tcgen05.commit
+//   warps 4-7 epilogue: tcgen05.ld of the accumulator, convert, store
+// Every wait on an mbarrier is bounded by wall time; on expiry the kernel
+// records FPQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace fpq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BK, B_TILE = BN * BK;
+constexpr int SFA_BYTES = 512, SFB_BYTES = 1024;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL0 = BN;            // scale columns follow the accumulator
+constexpr uint32_t SF_COLS_PER_STAGE = 16;  // 4 (A) + 8 (B), padded
+constexpr int NUM_THREADS = 256;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+
+struct __align__(1024) Smem {
+    uint8_t a[STAGES][A_TILE];
+    uint8_t b[STAGES][B_TILE];
+    uint8_t sfa[STAGES][SFA_BYTES];
+    uint8_t sfb[STAGES][SFB_BYTES];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tmem_full;
+    uint32_t tmem_base;
+    int32_t tile_valid;
+    int32_t group;
+    int32_t row_begin, row_end;   // A rows owned by this tile's group
+    int32_t m_tile, n_tile;
+};
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > kTimeoutNs) {
+            raise_device_error(err, FPQ_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t pick(const uint4& v, int j) {
+    return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+// Scales of one row for K tiles [4*kg, 4*kg + 4): 16 bytes (one word per K
+// tile, one byte per 32-wide sub-block).  Rows outside [0, nrows) and K tiles
+// past the end read as zero.
+__device__ __forceinline__ uint4 load_sf_group(const uint8_t* sf, int64_t row, int64_t nrows, int sf_pitch,
+                                               int kg, bool vec16) {
+    if (row < 0 || row >= nrows) return make_uint4(0, 0, 0, 0);
+    const uint8_t* p = sf + row * sf_pitch + kg * 16;
+    if (vec16) return *reinterpret_cast<const uint4*>(p);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        w[j] = (kg * 16 + 4 * j + 4 <= sf_pitch) ? *reinterpret_cast<const uint32_t*>(p + 4 * j) : 0u;
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// grouped: offsets != nullptr.  For the dense product groups = 1 and the
+// single group spans rows [0, M).
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
+                  const int32_t* __restrict__ offsets, int groups, int64_t M, int64_t N, int64_t K,
+                  void* __restrict__ C, int c_f32, uint32_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = (int)((N + BN - 1) / BN);
+    const int KT = (int)(K / BK);
+    const int sf_pitch = (int)(K / 32);
+
+    if (threadIdx.x == 0) {
+        // map this CTA to (group, m tile, n tile)
+        int valid = 0, g = 0, mt = 0, nt = 0;
+        int32_t rb = 0, re = (int32_t)M;
+        if (offsets == nullptr) {
+            const int t = blockIdx.x;
+            mt = t / n_tiles;
+            nt = t - mt * n_tiles;
+            valid = (int64_t)mt * BM < M;
+        } else {
+            bool ok = offsets[0] == 0 && offsets[groups] == (int32_t)M;
+            int t = blockIdx.x;
+            for (int e = 0; e < groups && ok; ++e) {
+                const int32_t b0 = offsets[e], b1 = offsets[e + 1];
+                if (b1 < b0) { ok = false; break; }
+                const int tiles_e = ((b1 - b0 + BM - 1) / BM) * n_tiles;
+                if (!valid && t < tiles_e) {
+                    valid = 1;
+                    g = e;
+                    mt = t / n_tiles;
+                    nt = t - mt * n_tiles;
+                    rb = b0;
+                    re = b1;
+                } else if (!valid) {
+                    t -= tiles_e;
+                }
+            }
+            if (!ok) {
+                if (blockIdx.x == 0) raise_device_error(err, FPQ_ERR_DEVICE_BAD_INPUT);
+                valid = 0;
+            }
+        }
+        sm.tile_valid = valid;
+        sm.group = g;
+        sm.m_tile = mt;
+        sm.n_tile = nt;
+        sm.row_begin = rb;
+        sm.row_end = re;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 2);     // TMA bytes + scale-factor warp
+            mbar_init(&sm.empty[s], 1);    // tcgen05.commit
+        }
+        mbar_init(&sm.tmem_full, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (!sm.tile_valid) return;
+
+    if (warp == 2) {
+        tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    const int64_t a_row0 = (int64_t)sm.row_begin + (int64_t)sm.m_tile * BM;   // first A row of the tile
+    const int64_t a_rows_end = sm.row_end;                                     // rows >= this are masked
+    const int64_t n0 = (int64_t)sm.n_tile * BN;
+    const int64_t b_row0 = (int64_t)sm.group * N + n0;                         // first row of B (flattened)
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
+                mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE);
+                tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)a_row0);
+                tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)b_row0);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- scale factors
+        const bool vec16 = (sf_pitch % 16) == 0;
+        const int KG = (KT + 3) / 4;
+        const int64_t b_rows_valid = (int64_t)sm.group * N + N;   // B rows of this group end here
+        uint4 ca[4], cb[8], na[4], nb[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            ca[i] = load_sf_group(sfa, a_row0 + lane + 32 * i, a_rows_end, sf_pitch, 0, vec16);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            cb[i] = load_sf_group(sfb, (b_row0 + lane + 32 * i < b_rows_valid) ? b_row0 + lane + 32 * i : -1,
+                                  b_rows_valid, sf_pitch, 0, vec16);
+        bool alive = true;
+        for (int kg = 0; kg < KG && alive; ++kg) {
+            if (kg + 1 < KG) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    na[i] = load_sf_group(sfa, a_row0 + lane + 32 * i, a_rows_end, sf_pitch, kg + 1, vec16);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    nb[i] = load_sf_group(sfb, (b_row0 + lane + 32 * i < b_rows_valid) ? b_row0 + lane + 32 * i : -1,
+                                          b_rows_valid, sf_pitch, kg + 1, vec16);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int kt = kg * 4 + j;
+                if (kt >= KT) break;
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) { alive = false; break; }
+                *reinterpret_cast<uint4*>(sm.sfa[s] + lane * 16) =
+                    make_uint4(pick(ca[0], j), pick(ca[1], j), pick(ca[2], j), pick(ca[3], j));
+                *reinterpret_cast<uint4*>(sm.sfb[s] + lane * 16) =
+                    make_uint4(pick(cb[0], j), pick(cb[1], j), pick(cb[2], j), pick(cb[3], j));
+                *reinterpret_cast<uint4*>(sm.sfb[s] + 512 + lane * 16) =
+                    make_uint4(pick(cb[4], j), pick(cb[5], j), pick(cb[6], j), pick(cb[7], j));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.full[s]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ca[i] = na[i];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cb[i] = nb[i];
+        }
+    } else if (warp == 2) {
+        // ---------------------------------------------------------- MMA issuer
+        if (elect_one()) {
+            bool ok = true;
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!wait_or_timeout(&sm.full[s], ph, err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sf_col = tmem + SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
+                tmem_cp_32x128b_warpx4(sf_col + 0, smem_desc(smem_u32(sm.sfa[s]), 0, 128, kLayoutNone));
+                tmem_cp_32x128b_warpx4(sf_col + 4, smem_desc(smem_u32(sm.sfb[s]), 0, 128, kLayoutNone));
+                tmem_cp_32x128b_warpx4(sf_col + 8, smem_desc(smem_u32(sm.sfb[s] + 512), 0, 128, kLayoutNone));
+                const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
+#pragma unroll
+                for (int k = 0; k < BK / 32; ++k) {
+                    const uint32_t idesc = idesc_mxf8f6f4(BM, BN, (uint32_t)k, (uint32_t)k);
+                    mma_mxf8f6f4(tmem, desc_kmajor_sw128(a_base + 32 * k), desc_kmajor_sw128(b_base + 32 * k), idesc,
+                                 (sf_col + 0) | ((uint32_t)k << 30), (sf_col + 4) | ((uint32_t)k << 30),
+                                 (kt > 0 || k > 0) ? 1u : 0u);
+                }
+                mma_commit(&sm.empty[s]);
+            }
+            if (ok) mma_commit(&sm.tmem_full);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;                       // TMEM lane quadrant of this warp
+        const int64_t row = a_row0 + 32 * q + lane;
+        const bool row_ok = row < a_rows_end;
+        if (wait_or_timeout(&sm.tmem_full, 0, err)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+                tmem_ld_wait();
+                const int64_t col0 = n0 + 32 * c;
+                if (!row_ok || col0 >= N) continue;
+                if (c_f32) {
+                    float* out = reinterpret_cast<float*>(C) + row * N + col0;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        if (col0 + 4 * v < N) st_v4(out + 4 * v, make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]));
+                } else {
+                    uint16_t* out = reinterpret_cast<uint16_t*>(C) + row * N + col0;
+                    uint32_t h[16];
+#pragma unroll
+                    for (int v = 0; v < 16; ++v) h[v] = f32x2_to_bf16x2(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        if (col0 + 8 * v < N) st_v4(out + 8 * v, make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]));
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+int smem_bytes() { return (int)sizeof(Smem) + 1024; }
+
+cudaError_t launch(const void* aq, const void* as, const void* bq, const void* bs, const int32_t* offsets,
+                   int groups, int64_t M, int64_t N, int64_t K, void* c, int c_f32, uint32_t* err,
+                   int64_t grid, cudaStream_t st) {
+    CUtensorMap ta, tb;
+    cudaError_t e = make_tmap_u8_2d(&ta, aq, (uint64_t)M, (uint64_t)K, (uint64_t)K, BM, BK);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_u8_2d(&tb, bq, (uint64_t)(groups * N), (uint64_t)K, (uint64_t)K, BN, BK);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemm_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+    if (e != cudaSuccess) return e;
+    if (grid < 1) return cudaSuccess;
+    gemm_mxfp8_kernel<<<(unsigned)grid, NUM_THREADS, smem_bytes(), st>>>(
+        ta, tb, (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs, int64_t m,
+                              int64_t n, int64_t k, void* c, int c_f32, uint32_t* err, int sms, cudaStream_t st) {
+    (void)sms;
+    const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
+    return launch(aq, as, bq, bs, nullptr, 1, m, n, k, c, c_f32, err, grid, st);
+}
+
+cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs,
+                                      const int32_t* offsets, int groups, int64_t total_m, int64_t n, int64_t k,
+                                      void* c, int c_f32, uint32_t* err, int sms, cudaStream_t st) {
+    (void)sms;
+    // Upper bound on the tile count without reading the device-side offsets:
+    // every group adds at most one partial row tile.
+    const int64_t grid = ((total_m + BM - 1) / BM + groups) * ((n + BN - 1) / BN);
+    return launch(aq, as, bq, bs, offsets, groups, total_m, n, k, c, c_f32, err, grid, st);
+}
+
+}  // namespace fpq

@@ -1,0 +1,37 @@
+// internal.h -- host-side launchers shared between the kernel translation
+// units and the C-ABI layer (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fpq {
+
+// Quantize `batch` dense row-major bf16 matrices [rows, cols] (fmt: fpq_format).
+cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows, int64_t cols,
+                            void* q, void* scales, float* tensor_scale, void* workspace,
+                            int sms, cudaStream_t st);
+
+cudaError_t launch_dequantize(int fmt, const void* q, const void* scales, const float* tensor_scale,
+                              int64_t batch, int64_t rows, int64_t cols, void* out, int sms,
+                              cudaStream_t st);
+
+cudaError_t launch_lora_merge_fakequant(const void* w, const void* a, const void* b, int64_t n,
+                                        int64_t k, int r, float alpha_over_r, void* wq, float* ws,
+                                        void* w_fq, cudaStream_t st);
+
+// Dense block-scaled GEMMs: C[m,n] = sum_k A[m,k] B[n,k].
+cudaError_t launch_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs,
+                              int64_t m, int64_t n, int64_t k, void* c, int c_f32,
+                              uint32_t* err, int sms, cudaStream_t st);
+
+cudaError_t launch_gemm_fp8_f32scale(const void* aq, const float* as, const void* bq,
+                                     const float* bs, int64_t m, int64_t n, int64_t k, void* c,
+                                     int c_f32, uint32_t* err, int sms, cudaStream_t st);
+
+cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void* bq,
+                                      const void* bs, const int32_t* offsets, int groups,
+                                      int64_t total_m, int64_t n, int64_t k, void* c, int c_f32,
+                                      uint32_t* err, int sms, cudaStream_t st);
+
+}  // namespace fpq

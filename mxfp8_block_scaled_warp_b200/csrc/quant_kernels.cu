@@ -1,0 +1,408 @@
+// quant_kernels.cu -- block quantize / dequantize kernels for sm_100a.
+//
+// Every kernel here streams HBM: 16-byte vector loads, several independent
+// loads in flight per thread (an unrolled grid-stride loop), absmax of a
+// block reduced with warp shuffles, packed hardware conversion to E4M3 or
+// E2M1, and 8/16-byte stores with the scales written alongside.
+//
+// Work unit: 16 consecutive bf16 elements of a row (32 bytes), held by one
+// lane as eight 32-bit words.  A block of the format is 2 units (MXFP8 1x32),
+// 8 units (1x128) or 1 unit (NVFP4 1x16); because every row length is a
+// multiple of the block, blocks never straddle rows and a flat unit index
+// addresses both the data and the row-major scale arrays.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace fpq {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;   // units in flight per thread
+
+struct Unit { uint32_t w[8]; };
+
+__device__ __forceinline__ Unit load_unit(const uint4* x, int64_t u) {
+    uint4 a = ld_stream(x + 2 * u), b = ld_stream(x + 2 * u + 1);
+    return Unit{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
+}
+
+__device__ __forceinline__ uint32_t unit_absmax(const Unit& v) {
+    uint32_t m = abs2(v.w[0]);
+#pragma unroll
+    for (int i = 1; i < 8; ++i) m = max2(m, abs2(v.w[i]));
+    return hmax2(m);
+}
+
+// Reduce a magnitude pattern over `width` adjacent lanes (power of two).
+template <int width>
+__device__ __forceinline__ uint32_t group_max(uint32_t m) {
+#pragma unroll
+    for (int o = 1; o < width; o <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    return m;
+}
+
+// MXFP8 block exponent from the block's largest magnitude pattern a (15 bits
+// of a bf16): e = ceil(log2(amax/448)) clamped to [-127, 127], computed from
+// the exponent and mantissa fields.  With amax = mu * 2^E, mu in [1, 2):
+// amax/448 = (mu/1.75) * 2^(E-8), so e = E - 8 when mu <= 1.75 and E - 7
+// when mu > 1.75 (mantissa field > 0x60).  Zero and subnormal amax clamp to
+// -127; infinity gives 127; NaN gives code 0xFF (returned as 128).
+__device__ __forceinline__ int mx_exponent(uint32_t a) {
+    if (a > 0x7F80u) return 128;
+    if (a == 0x7F80u) return 127;
+    uint32_t E = a >> 7;
+    if (E == 0) return -127;
+    int e = (int)E - 127 - 8 + ((a & 0x7Fu) > 0x60u ? 1 : 0);
+    return max(-127, min(127, e));
+}
+
+// 2^-e as fp32 for e in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float pow2_neg(int e) {
+    return (e == 127) ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(127 - e) << 23);
+}
+
+__device__ __forceinline__ uint4 scale_to_e4m3(const Unit& v, float mul) {
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = f32x2_to_e4m3x2(bf16_lo(v.w[i]) * mul, bf16_hi(v.w[i]) * mul);
+    return make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+}
+
+__device__ __forceinline__ uint4 divide_to_e4m3(const Unit& v, float s) {
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        c[i] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(v.w[i]), s), __fdiv_rn(bf16_hi(v.w[i]), s));
+    return make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+}
+
+// fp32 block scale s = fp32(amax / 448), 1 for an all-zero block.
+__device__ __forceinline__ float fp32_scale(uint32_t a) {
+    return a == 0 ? 1.0f : __fdiv_rn(__uint_as_float(a << 16), 448.0f);
+}
+
+// ----------------------------------------------------------------- MXFP8
+
+__global__ void __launch_bounds__(kThreads)
+quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* __restrict__ s,
+                   int64_t units) {
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units; base += stride) {
+        Unit v[kUnroll];
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            if (u < units) v[i] = load_unit(x, u);
+        }
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            // both lanes of a block are in range or out of range together
+            // (units is even), so the shuffle below is uniform per pair
+            uint32_t a = group_max<2>(u < units ? unit_absmax(v[i]) : 0u);
+            if (u >= units) continue;
+            int e = mx_exponent(a);
+            uint4 out;
+            if (e == 128) out = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+            else out = scale_to_e4m3(v[i], pow2_neg(e));
+            st_v4(q + u, out);
+            if ((u & 1) == 0) s[u >> 1] = (uint8_t)(e + 127);
+        }
+    }
+}
+
+// ----------------------------------------------------------------- FP8 1x128
+
+__global__ void __launch_bounds__(kThreads)
+quant_fp8_1x128_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
+                       float* __restrict__ s, int64_t units) {
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units; base += stride) {
+        Unit v[kUnroll];
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            if (u < units) v[i] = load_unit(x, u);
+        }
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            uint32_t a = group_max<8>(u < units ? unit_absmax(v[i]) : 0u);
+            if (u >= units) continue;
+            float sc = fp32_scale(a);
+            st_v4(q + u, divide_to_e4m3(v[i], sc));
+            if ((u & 7) == 0) s[u >> 3] = sc;
+        }
+    }
+}
+
+// ----------------------------------------------------------------- FP8 128x128
+
+// One CTA per 128x128 block: 256 threads x 8 chunks of 8 elements (16 B).
+// Chunk c of the block covers row c/16, columns 8*(c%16) .. +8.
+__global__ void __launch_bounds__(256)
+quant_fp8_128x128_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s,
+                         int64_t rows, int64_t cols) {
+    const int64_t bj = blockIdx.x, bi = blockIdx.y, b = blockIdx.z;
+    const int64_t nbr = (rows + 127) / 128, nbc = cols / 128;
+    const uint16_t* xb = x + (b * rows + bi * 128) * cols + bj * 128;
+    uint8_t* qb = q + (b * rows + bi * 128) * cols + bj * 128;
+    const int64_t rmax = min64(128, rows - bi * 128);
+    uint4 v[8];
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int c = threadIdx.x + 256 * i, r = c >> 4, c8 = (c & 15) * 8;
+        if (r < rmax) {
+            v[i] = ld_stream(xb + r * cols + c8);
+            m = max2(m, max2(max2(abs2(v[i].x), abs2(v[i].y)), max2(abs2(v[i].z), abs2(v[i].w))));
+        }
+    }
+    m = group_max<32>(hmax2(m));
+    __shared__ uint32_t red[8];
+    __shared__ float sc_sh;
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t a = red[0];
+        for (int w = 1; w < 8; ++w) a = max(a, red[w]);
+        float sc = fp32_scale(a);
+        sc_sh = sc;
+        s[(b * nbr + bi) * nbc + bj] = sc;
+    }
+    __syncthreads();
+    const float sc = sc_sh;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int c = threadIdx.x + 256 * i, r = c >> 4, c8 = (c & 15) * 8;
+        if (r < rmax) {
+            uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            uint32_t e[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                e[j] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[j]), sc), __fdiv_rn(bf16_hi(w[j]), sc));
+            st_v2(qb + r * cols + c8, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
+        }
+    }
+}
+
+// ----------------------------------------------------------------- NVFP4
+
+// Pass 1: per-matrix amax as a 15-bit magnitude pattern, atomicMax into
+// amax_bits[b] (zeroed by the launcher).  grid = (slices, matrices).
+__global__ void __launch_bounds__(kThreads)
+tensor_amax_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, uint32_t* __restrict__ amax_bits) {
+    const int64_t b = blockIdx.y;
+    const uint4* xb = x + 2 * b * units_per_matrix;
+    uint32_t m = 0;
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units_per_matrix; base += stride) {
+        Unit v[kUnroll];
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            if (u < units_per_matrix) v[i] = load_unit(xb, u);
+        }
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            if (u < units_per_matrix) m = max(m, unit_absmax(v[i]));
+        }
+    }
+    m = group_max<32>(m);
+    if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax_bits + b, m);
+}
+
+// Per-tensor scale g = fp32(amax_T / 2688), 1 for an all-zero tensor.
+__device__ __forceinline__ float nvfp4_tensor_scale(uint32_t a) {
+    return a == 0 ? 1.0f : __fdiv_rn(__uint_as_float(a << 16), 2688.0f);
+}
+
+// Pass 2: one lane per 16-element block.  grid = (slices, matrices).
+__global__ void __launch_bounds__(kThreads)
+quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, const uint32_t* __restrict__ amax_bits,
+                   uint2* __restrict__ q, uint8_t* __restrict__ s, float* __restrict__ g_out) {
+    const int64_t b = blockIdx.y;
+    const uint4* xb = x + 2 * b * units_per_matrix;
+    uint2* qb = q + b * units_per_matrix;
+    uint8_t* sb = s + b * units_per_matrix;
+    const float g = nvfp4_tensor_scale(amax_bits[b]);
+    if (blockIdx.x == 0 && threadIdx.x == 0) g_out[b] = g;
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units_per_matrix; base += stride) {
+        Unit v[kUnroll];
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            if (u < units_per_matrix) v[i] = load_unit(xb, u);
+        }
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            int64_t u = base + i * kThreads + threadIdx.x;
+            if (u >= units_per_matrix) continue;
+            const uint32_t a = unit_absmax(v[i]);
+            const float t = __fdiv_rn(__uint_as_float(a << 16), 6.0f);
+            const uint32_t code = f32x2_to_e4m3x2(__fdiv_rn(t, g), 0.0f) & 0xFFu;
+            const float S = e4m3_to_f32(code) * g;
+            uint32_t packed[2] = {0u, 0u};
+            if (S != 0.0f) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(bf16_lo(v[i].w[j]), S),
+                                                    __fdiv_rn(bf16_hi(v[i].w[j]), S));
+                    packed[j >> 2] |= byte << (8 * (j & 3));
+                }
+            }
+            st_v2(qb + u, make_uint2(packed[0], packed[1]));
+            sb[u] = (uint8_t)code;
+        }
+    }
+}
+
+// ----------------------------------------------------------------- dequantize
+
+__device__ __forceinline__ void store_bf16x16(uint4* out, int64_t u, const float (&f)[16]) {
+    uint32_t h[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] = f32x2_to_bf16x2(f[2 * j], f[2 * j + 1]);
+    st_v4(out + 2 * u, make_uint4(h[0], h[1], h[2], h[3]));
+    st_v4(out + 2 * u + 1, make_uint4(h[4], h[5], h[6], h[7]));
+}
+
+// fmt: 0 = 1x128 (fp32 scale per 8 units), 2 = MXFP8 (E8M0 per 2 units),
+// 1 = 128x128 (fp32 scale per 128x128 block).
+template <int kFmt>
+__global__ void __launch_bounds__(kThreads)
+dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales, uint4* __restrict__ out,
+                   int64_t units, int64_t rows, int64_t cols) {
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    const int64_t units_per_row = cols / 16;
+    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
+        uint4 c = ld_stream(q + u);
+        float sc;
+        if (kFmt == 2) {
+            uint32_t code = ((const uint8_t*)scales)[u >> 1];
+            sc = code == 0xFFu ? __uint_as_float(0x7FC00000u)
+               : code == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(code << 23);
+        } else if (kFmt == 0) {
+            sc = ((const float*)scales)[u >> 3];
+        } else {
+            int64_t row = u / units_per_row, colu = u - row * units_per_row;
+            int64_t b = row / rows, r = row - b * rows;
+            int64_t nbr = (rows + 127) / 128, nbc = cols / 128;
+            sc = ((const float*)scales)[(b * nbr + r / 128) * nbc + colu / 8];
+        }
+        uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        float f[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float2 lo = e4m3x2_to_f32x2(w[j] & 0xFFFFu), hi = e4m3x2_to_f32x2(w[j] >> 16);
+            f[4 * j + 0] = lo.x * sc; f[4 * j + 1] = lo.y * sc;
+            f[4 * j + 2] = hi.x * sc; f[4 * j + 3] = hi.y * sc;
+        }
+        store_bf16x16(out, u, f);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+dequant_nvfp4_kernel(const uint2* __restrict__ q, const uint8_t* __restrict__ s, const float* __restrict__ g,
+                     uint4* __restrict__ out, int64_t units, int64_t units_per_matrix) {
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
+        uint2 c = q[u];
+        const float S = e4m3_to_f32(s[u]) * g[u / units_per_matrix];
+        uint32_t w[2] = {c.x, c.y};
+        float f[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float2 e = e2m1x2_to_f32x2((w[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+            f[2 * j] = e.x * S;
+            f[2 * j + 1] = e.y * S;
+        }
+        store_bf16x16(out, u, f);
+    }
+}
+
+int grid_for(int64_t work_items, int per_cta, int sms) {
+    int64_t g = (work_items + per_cta - 1) / per_cta;
+    int64_t cap = (int64_t)sms * 8;
+    return (int)max64(1, min(g, cap));
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------- launchers
+
+cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows, int64_t cols,
+                            void* q, void* scales, float* tensor_scale, void* workspace,
+                            int sms, cudaStream_t st) {
+    const int64_t n = batch * rows * cols, units = n / 16;
+    switch (fmt) {
+    case FPQ_MXFP8:
+        quant_mxfp8_kernel<<<grid_for(units, kThreads * kUnroll, sms), kThreads, 0, st>>>(
+            (const uint4*)x, (uint4*)q, (uint8_t*)scales, units);
+        break;
+    case FPQ_FP8_1x128:
+        quant_fp8_1x128_kernel<<<grid_for(units, kThreads * kUnroll, sms), kThreads, 0, st>>>(
+            (const uint4*)x, (uint4*)q, (float*)scales, units);
+        break;
+    case FPQ_FP8_128x128: {
+        dim3 grid((unsigned)(cols / 128), (unsigned)((rows + 127) / 128), (unsigned)batch);
+        quant_fp8_128x128_kernel<<<grid, 256, 0, st>>>((const uint16_t*)x, (uint8_t*)q, (float*)scales, rows, cols);
+        break;
+    }
+    case FPQ_NVFP4: {
+        const int64_t upm = rows * cols / 16;
+        uint32_t* amax = (uint32_t*)workspace;
+        cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t) * batch, st);
+        if (e != cudaSuccess) return e;
+        // Matrices are processed in chunks small enough that the amax pass
+        // leaves the chunk resident in L2 for the quantize pass.
+        const int64_t chunk_bytes = 64ll << 20;
+        int64_t per_chunk = max64(1, chunk_bytes / max64(1, rows * cols * 2));
+        for (int64_t b0 = 0; b0 < batch; b0 += per_chunk) {
+            int64_t nb = min(per_chunk, batch - b0);
+            int slices = (int)max64(1, min64((sms * 8 + nb - 1) / nb,
+                                                           (upm + kThreads * kUnroll - 1) / (kThreads * kUnroll)));
+            dim3 grid((unsigned)slices, (unsigned)nb);
+            tensor_amax_kernel<<<grid, kThreads, 0, st>>>((const uint4*)x + 2 * b0 * upm, upm, amax + b0);
+            quant_nvfp4_kernel<<<grid, kThreads, 0, st>>>((const uint4*)x + 2 * b0 * upm, upm, amax + b0,
+                                                          (uint2*)q + b0 * upm, (uint8_t*)scales + b0 * upm,
+                                                          tensor_scale + b0);
+        }
+        break;
+    }
+    default:
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(int fmt, const void* q, const void* scales, const float* tensor_scale,
+                              int64_t batch, int64_t rows, int64_t cols, void* out, int sms, cudaStream_t st) {
+    const int64_t units = batch * rows * cols / 16;
+    const int grid = grid_for(units, kThreads, sms);
+    switch (fmt) {
+    case FPQ_MXFP8:
+        dequant_fp8_kernel<2><<<grid, kThreads, 0, st>>>((const uint4*)q, scales, (uint4*)out, units, rows, cols);
+        break;
+    case FPQ_FP8_1x128:
+        dequant_fp8_kernel<0><<<grid, kThreads, 0, st>>>((const uint4*)q, scales, (uint4*)out, units, rows, cols);
+        break;
+    case FPQ_FP8_128x128:
+        dequant_fp8_kernel<1><<<grid, kThreads, 0, st>>>((const uint4*)q, scales, (uint4*)out, units, rows, cols);
+        break;
+    case FPQ_NVFP4:
+        dequant_nvfp4_kernel<<<grid, kThreads, 0, st>>>((const uint2*)q, (const uint8_t*)scales, tensor_scale,
+                                                        (uint4*)out, units, rows * cols / 16);
+        break;
+    default:
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace fpq

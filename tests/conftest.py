@@ -22,3 +22,13 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def fpq():
+    """The CUDA library's Python binding.  GPU tests fail (never skip) when
+    the device or the built library is missing: there is no fallback."""
+    import torch
+    assert torch.cuda.is_available(), "GPU test run without a CUDA device"
+    import mxfp8_block_scaled_warp_b200 as lib
+    return lib
