@@ -3,9 +3,10 @@
 A thin ctypes binding over ``libfpq.so`` (C ABI: ``include/fpq.h``).  Every
 step of the computation runs in the library's CUDA kernels; this module only
 checks and marshals torch tensors (device memory, streams) into the C calls.
-There is no CPU fallback: importing fails loudly when ``libfpq.so`` is missing
-(build it with ``python -m mxfp8_block_scaled_warp_b200.build``), and every
-call fails with FPQ_ERR_UNSUPPORTED on a device that is not sm_100.
+There is no CPU fallback: the first call (or ``load()``) raises ImportError
+when ``libfpq.so`` is missing (build it with ``python -m
+mxfp8_block_scaled_warp_b200.build``), and every call fails with
+FPQ_ERR_UNSUPPORTED on a device that is not sm_100.
 
 The ``fpq_*`` functions mirror the C entry points one to one (tensors in
 place of pointers, the current torch stream by default).  ``quantize``,
@@ -21,7 +22,7 @@ import os
 import torch
 
 __all__ = [
-    "FP8_1x128", "FP8_128x128", "MXFP8", "NVFP4", "OUT_BF16", "OUT_F32", "FpqError", "lib_path",
+    "FP8_1x128", "FP8_128x128", "MXFP8", "NVFP4", "OUT_BF16", "OUT_F32", "FpqError", "lib_path", "load",
     "fpq_version", "fpq_quantize_workspace_bytes", "fpq_quantize_block", "fpq_dequantize",
     "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_grouped_scaled_gemm", "fpq_get_device_error",
     "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "grouped_scaled_gemm",
@@ -42,6 +43,17 @@ class FpqError(RuntimeError):
     def __init__(self, status: int, where: str, detail: str):
         self.status = status
         super().__init__(f"{where}: {STATUS.get(status, status)} ({detail})")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libfpq.so (once); ImportError if it has not been built."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
 
 
 def _load() -> ctypes.CDLL:
@@ -67,12 +79,9 @@ def _load() -> ctypes.CDLL:
     return L
 
 
-_lib = _load()
-
-
 def _check(status: int, where: str) -> None:
     if status != 0:
-        raise FpqError(status, where, _lib.fpq_last_error_detail().decode(errors="replace"))
+        raise FpqError(status, where, load().fpq_last_error_detail().decode(errors="replace"))
 
 
 def _ptr(t: torch.Tensor | None):
@@ -94,44 +103,44 @@ def _stream(stream) -> int | None:
 # ---------------------------------------------------------------- raw C entry points
 
 def fpq_version() -> int:
-    return _lib.fpq_version()
+    return load().fpq_version()
 
 
 def fpq_quantize_workspace_bytes(fmt: int, batch: int) -> int:
-    return _lib.fpq_quantize_workspace_bytes(fmt, batch)
+    return load().fpq_quantize_workspace_bytes(fmt, batch)
 
 
 def fpq_quantize_block(fmt, x, batch, rows, cols, q, scales, tensor_scale=None, workspace=None, stream=None):
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib.fpq_quantize_block(fmt, _ptr(x), batch, rows, cols, _ptr(q), _ptr(scales), _ptr(tensor_scale),
+    _check(load().fpq_quantize_block(fmt, _ptr(x), batch, rows, cols, _ptr(q), _ptr(scales), _ptr(tensor_scale),
                                    _ptr(workspace), wsb, _stream(stream)), "fpq_quantize_block")
 
 
 def fpq_dequantize(fmt, q, scales, tensor_scale, batch, rows, cols, out, stream=None):
-    _check(_lib.fpq_dequantize(fmt, _ptr(q), _ptr(scales), _ptr(tensor_scale), batch, rows, cols, _ptr(out),
+    _check(load().fpq_dequantize(fmt, _ptr(q), _ptr(scales), _ptr(tensor_scale), batch, rows, cols, _ptr(out),
                                _stream(stream)), "fpq_dequantize")
 
 
 def fpq_lora_merge_fakequant(w, lora_a, lora_b, n, k, r, alpha_over_r, wq, ws, w_fq=None, stream=None):
-    _check(_lib.fpq_lora_merge_fakequant(_ptr(w), _ptr(lora_a), _ptr(lora_b), n, k, r, float(alpha_over_r),
+    _check(load().fpq_lora_merge_fakequant(_ptr(w), _ptr(lora_a), _ptr(lora_b), n, k, r, float(alpha_over_r),
                                          _ptr(wq), _ptr(ws), _ptr(w_fq), _stream(stream)),
            "fpq_lora_merge_fakequant")
 
 
 def fpq_scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, m, n, k, c, c_dtype, stream=None):
-    _check(_lib.fpq_scaled_gemm(fmt_a, _ptr(aq), _ptr(as_), fmt_b, _ptr(bq), _ptr(bs), m, n, k, _ptr(c), c_dtype,
+    _check(load().fpq_scaled_gemm(fmt_a, _ptr(aq), _ptr(as_), fmt_b, _ptr(bq), _ptr(bs), m, n, k, _ptr(c), c_dtype,
                                 _stream(stream)), "fpq_scaled_gemm")
 
 
 def fpq_grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, groups, total_m, n, k, c, c_dtype, stream=None):
-    _check(_lib.fpq_grouped_scaled_gemm(fmt, _ptr(aq), _ptr(as_), _ptr(bq), _ptr(bs), _ptr(group_offsets), groups,
+    _check(load().fpq_grouped_scaled_gemm(fmt, _ptr(aq), _ptr(as_), _ptr(bq), _ptr(bs), _ptr(group_offsets), groups,
                                         total_m, n, k, _ptr(c), c_dtype, _stream(stream)),
            "fpq_grouped_scaled_gemm")
 
 
 def fpq_get_device_error(stream=None) -> int:
     code = ctypes.c_int32(0)
-    _check(_lib.fpq_get_device_error(_stream(stream), ctypes.byref(code)), "fpq_get_device_error")
+    _check(load().fpq_get_device_error(_stream(stream), ctypes.byref(code)), "fpq_get_device_error")
     return code.value
 
 

@@ -31,4 +31,5 @@ def fpq():
     import torch
     assert torch.cuda.is_available(), "GPU test run without a CUDA device"
     import mxfp8_block_scaled_warp_b200 as lib
+    lib.load()
     return lib
