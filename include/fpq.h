@@ -214,6 +214,27 @@ FPQ_API fpq_status fpq_grouped_scaled_gemm(fpq_format fmt, const void* aq, const
                                    int32_t c_dtype, void* stream);
 
 /*
+ * fpq_quantize_nvfp4_noalloc -- NVFP4 quantization (same outputs, layouts and
+ * errors as fpq_quantize_block with FPQ_NVFP4) for callers that cannot
+ * allocate device memory and so cannot pass the amax workspace, such as a
+ * plugin running inside a host application that owns the device memory pool.
+ * The pages describe no such entry point; it exists for these callers only.
+ *
+ * Scratch: a library-owned static device array of FPQ_NOALLOC_NVFP4_MAX_BATCH
+ * words (16 KiB) on every GPU that loads the library, held until the process
+ * exits.  No call allocates or frees anything.  batch > the maximum gives
+ * FPQ_ERR_INVALID_ARG.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  All calls on a device share the
+ * array, so calls that may overlap on the GPU (different streams, no
+ * ordering between them) race and must not be issued; calls on one stream
+ * are safe.
+ */
+#define FPQ_NOALLOC_NVFP4_MAX_BATCH 4096
+FPQ_API fpq_status fpq_quantize_nvfp4_noalloc(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                                              void* q, void* scales, float* tensor_scale, void* stream);
+
+/*
  * fpq_get_device_error -- synchronize `stream`, then read and clear the
  * current device's error word.  *code receives FPQ_OK or the first
  * FPQ_ERR_DEVICE_* raised by a kernel since the last read.  Returns

@@ -25,6 +25,7 @@ __all__ = [
     "FP8_1x128", "FP8_128x128", "MXFP8", "NVFP4", "OUT_BF16", "OUT_F32", "FpqError", "lib_path", "load",
     "fpq_version", "fpq_quantize_workspace_bytes", "fpq_quantize_block", "fpq_dequantize",
     "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_grouped_scaled_gemm", "fpq_get_device_error",
+    "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
     "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "grouped_scaled_gemm",
     "scale_shape", "code_shape",
 ]
@@ -72,6 +73,7 @@ def _load() -> ctypes.CDLL:
         "fpq_scaled_gemm": (I32, [I32, P, P, I32, P, P, I64, I64, I64, P, I32, P]),
         "fpq_grouped_scaled_gemm": (I32, [I32, P, P, P, P, P, I32, I64, I64, I64, P, I32, P]),
         "fpq_get_device_error": (I32, [P, ctypes.POINTER(I32)]),
+        "fpq_quantize_nvfp4_noalloc": (I32, [P, I64, I64, I64, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -136,6 +138,17 @@ def fpq_grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, groups, total_m
     _check(load().fpq_grouped_scaled_gemm(fmt, _ptr(aq), _ptr(as_), _ptr(bq), _ptr(bs), _ptr(group_offsets), groups,
                                         total_m, n, k, _ptr(c), c_dtype, _stream(stream)),
            "fpq_grouped_scaled_gemm")
+
+
+def fpq_quantize_nvfp4_noalloc(x, batch, rows, cols, q, scales, tensor_scale, stream=None):
+    """NVFP4 quantize without a workspace argument, for callers that cannot
+    allocate: the library keeps the scratch in a static device array (at most
+    NOALLOC_NVFP4_MAX_BATCH batch items; calls that overlap on the GPU race)."""
+    _check(load().fpq_quantize_nvfp4_noalloc(_ptr(x), batch, rows, cols, _ptr(q), _ptr(scales), _ptr(tensor_scale),
+                                           _stream(stream)), "fpq_quantize_nvfp4_noalloc")
+
+
+NOALLOC_NVFP4_MAX_BATCH = 4096
 
 
 def fpq_get_device_error(stream=None) -> int:

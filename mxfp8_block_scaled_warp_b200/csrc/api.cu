@@ -107,6 +107,12 @@ fpq_status check_quant_shape(fpq_format fmt, int64_t batch, int64_t rows, int64_
 
 }  // namespace
 
+namespace fpq {
+// Lets other translation units of the library report a detail string through
+// fpq_last_error_detail().
+void set_error_detail(const char* what) { set_detail(what); }
+}  // namespace fpq
+
 extern "C" {
 
 int32_t fpq_version(void) { return 10000; }

@@ -34,4 +34,7 @@ cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void
                                       int64_t total_m, int64_t n, int64_t k, void* c, int c_f32,
                                       uint32_t* err, int sms, cudaStream_t st);
 
+// Set the per-thread detail string returned by fpq_last_error_detail().
+void set_error_detail(const char* what);
+
 }  // namespace fpq
