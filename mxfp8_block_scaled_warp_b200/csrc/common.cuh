@@ -89,6 +89,45 @@ __device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t c2) {
                        __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
 }
 
+// ----------------------------------------------------------------- exact quotient codes
+//
+// The fp32-scale formats define a code as the rounding of the correctly
+// rounded fp32 quotient q(x) = fp32(x / s).  A division per element is the
+// slow part of the quantizers (it runs on the reciprocal unit), so the codes
+// are obtained from t = x * r with r = fp32(1/s) instead, and checked:
+//   |t - q(x)| < 3 ulp (ulp of the binade of x/s; at most 6 ulp of the binade
+//   below), because r and t each add at most half an ulp of relative error
+//   and q(x) itself is within half an ulp of x/s.
+// Rounding to a narrow format is monotone in the value, so if the magnitude
+// patterns |t| - 16 and |t| + 16 round to the same code, every value between
+// them -- q(x) included -- rounds to that code.  Otherwise (a quotient within
+// 16 ulp of a rounding boundary, rare) the code is taken from the IEEE
+// division itself.  The caller guarantees r is finite (s >= 2^-126).
+// The sign of the code is the sign of x (s > 0), so -0 keeps its sign.
+
+__device__ __forceinline__ uint32_t abs_pattern(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+// E4M3 codes of fp32(x0/s) (bits 0-7) and fp32(x1/s) (bits 8-15).
+__device__ __forceinline__ uint32_t e4m3x2_of_quotients(float x0, float x1, float s, float r) {
+    const uint32_t m0 = abs_pattern(x0 * r), m1 = abs_pattern(x1 * r);
+    uint32_t lo = f32x2_to_e4m3x2(__uint_as_float(m0 - min(m0, 16u)), __uint_as_float(m1 - min(m1, 16u)));
+    const uint32_t hi = f32x2_to_e4m3x2(__uint_as_float(m0 + 16u), __uint_as_float(m1 + 16u));
+    if (lo != hi) lo = f32x2_to_e4m3x2(fabsf(__fdiv_rn(x0, s)), fabsf(__fdiv_rn(x1, s)));
+    return lo | ((__float_as_uint(x0) >> 24) & 0x80u) | ((__float_as_uint(x1) >> 16) & 0x8000u);
+}
+
+// E2M1 codes of fp32(x0/s) (bits 0-3) and fp32(x1/s) (bits 4-7).
+__device__ __forceinline__ uint32_t e2m1x2_of_quotients(float x0, float x1, float s, float r) {
+    const uint32_t m0 = abs_pattern(x0 * r), m1 = abs_pattern(x1 * r);
+    uint32_t lo = f32x2_to_e2m1x2(__uint_as_float(m0 - min(m0, 16u)), __uint_as_float(m1 - min(m1, 16u)));
+    const uint32_t hi = f32x2_to_e2m1x2(__uint_as_float(m0 + 16u), __uint_as_float(m1 + 16u));
+    if (lo != hi) lo = f32x2_to_e2m1x2(fabsf(__fdiv_rn(x0, s)), fabsf(__fdiv_rn(x1, s)));
+    return lo | ((__float_as_uint(x0) >> 28) & 0x8u) | ((__float_as_uint(x1) >> 24) & 0x80u);
+}
+
+// Whether the multiply-and-check path applies for divisor s (1/s finite).
+__device__ __forceinline__ bool reciprocal_ok(float s) { return s >= 1.17549435e-38f; }
+
 // ----------------------------------------------------------------- absmax
 
 // Largest magnitude pattern of the two bf16 halves of each word, as a packed

@@ -10,9 +10,11 @@
 // before the final accumulation.  The MMA runs up to NBUF K blocks ahead of
 // the promotion.
 //
-// Per CTA one 128 x 128 output tile.  Warp roles: warp 0 TMA producer,
-// warp 2 TMEM allocator + MMA issuer, warps 4-11 promotion/epilogue (warp w
-// owns TMEM lane quadrant w % 4 and column half (w - 4) / 4).
+// Per CTA one 128 x 256 output tile (the wider N halves the shared-memory
+// operand bytes per FLOP against a 128 x 128 tile).  Warp roles: warp 0 TMA
+// producer, warp 1 TMEM allocator + MMA issuer, warps 2-9 promotion and
+// epilogue (warp w owns TMEM lane quadrant w % 4 and the 128-column half
+// (w - 2) / 4 of the tile, i.e. one 128-wide block of B and its scale).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -26,13 +28,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 128, BK = 128;
-constexpr int STAGES = 6;
-constexpr int NBUF = 4;
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int STAGES = 4;
+constexpr int NBUF = 2;
 constexpr int A_TILE = BM * BK, B_TILE = BN * BK;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 128 + 32 * NUM_EPI_WARPS;
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int EPI_COLS = 128;               // columns per promotion warp
+constexpr int CHUNK = 16;                   // columns per tcgen05.ld
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 struct __align__(1024) Smem {
@@ -64,6 +68,9 @@ __device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
     }
 }
 
+// 10 warps: two SM sub-partitions hold three warps each, so a thread gets at
+// most 168 registers (16 K registers per sub-partition); a promotion thread
+// keeps 128 fp32 accumulators plus one 16-column TMEM chunk.
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_fp8_f32scale_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const float* __restrict__ sA, const float* __restrict__ sB, int64_t M, int64_t N,
@@ -87,7 +94,7 @@ gemm_fp8_f32scale_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
         }
         fence_barrier_init();
     }
-    if (warp == 2) {
+    if (warp == 1) {
         tmem_alloc(&sm.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
@@ -109,7 +116,7 @@ gemm_fp8_f32scale_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                 tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)n0);
             }
         }
-    } else if (warp == 2) {
+    } else if (warp == 1) {
         if (elect_one()) {
             const uint32_t idesc = idesc_f8f6f4(BM, BN);
             for (int kt = 0; kt < KT; ++kt) {
@@ -130,22 +137,25 @@ gemm_fp8_f32scale_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                 mma_commit(&sm.acc_full[b]);
             }
         }
-    } else if (warp >= 4) {
-        const int ew = warp - 4;
+    } else {
+        const int ew = warp - 2;
         const int q = warp & 3, half = ew >> 2;
         const int64_t row = m0 + 32 * q + lane;
         const bool row_ok = row < M;
         const int64_t kts = K / 128;
+        const int64_t nb = n0 / 128 + half;                 // this warp's 128-wide block of B
+        const bool half_ok = nb * 128 < N;
         const float* sa_row = sA + (row_ok ? row : 0) * kts;
-        const float* sb_row = sB + (n0 / 128) * kts;
-        float acc[64];
+        const float* sb_row = sB + (half_ok ? nb : 0) * kts;
+        uint64_t acc[EPI_COLS / 2];          // pairs of fp32 accumulators (packed f32x2 FMAs)
 #pragma unroll
-        for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+        for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = 0ull;
         float sa_next = row_ok ? __ldg(sa_row) : 0.0f;
         float sb_next = __ldg(sb_row);
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
             const float sc = sa_next * sb_next;
+            const uint64_t sc2 = pack_f32x2(sc, sc);
             if (kt + 1 < KT) {
                 sa_next = row_ok ? __ldg(sa_row + kt + 1) : 0.0f;
                 sb_next = __ldg(sb_row + kt + 1);
@@ -154,44 +164,47 @@ gemm_fp8_f32scale_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             const uint32_t pb = (uint32_t)(kt / NBUF) & 1u;
             if (!wait_or_timeout(&sm.acc_full[b], pb, err)) { ok = false; break; }
             tc_fence_after();
-            uint32_t p0[32], p1[32];
-            const uint32_t t = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN + 64 * half);
-            tmem_ld_32x32b_x32(t, p0);
-            tmem_ld_32x32b_x32(t + 32, p1);
-            tmem_ld_wait();
+            const uint32_t t = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN + EPI_COLS * half);
+#pragma unroll
+            for (int c = 0; c < EPI_COLS / CHUNK; ++c) {
+                uint32_t p[CHUNK];
+                tmem_ld_32x32b_x16(t + (uint32_t)(CHUNK * c), p);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < CHUNK / 2; ++j)
+                    acc[CHUNK / 2 * c + j] = fma_f32x2(pack_u32x2(p[2 * j], p[2 * j + 1]), sc2, acc[CHUNK / 2 * c + j]);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.acc_empty[b]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] = __fmaf_rn(__uint_as_float(p0[j]), sc, acc[j]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[32 + j] = __fmaf_rn(__uint_as_float(p1[j]), sc, acc[32 + j]);
         }
-        const int64_t col0 = n0 + 64 * half;
+        const int64_t col0 = n0 + EPI_COLS * half;
         if (ok && row_ok && col0 < N) {
             if (c_f32) {
                 float* out = reinterpret_cast<float*>(C) + row * N + col0;
 #pragma unroll
-                for (int v = 0; v < 16; ++v)
+                for (int v = 0; v < EPI_COLS / 4; ++v)
                     if (col0 + 4 * v < N)
-                        st_v4(out + 4 * v, make_uint4(__float_as_uint(acc[4 * v]), __float_as_uint(acc[4 * v + 1]),
-                                                      __float_as_uint(acc[4 * v + 2]), __float_as_uint(acc[4 * v + 3])));
+                        st_v4(out + 4 * v, make_uint4((uint32_t)acc[2 * v], (uint32_t)(acc[2 * v] >> 32),
+                                                      (uint32_t)acc[2 * v + 1], (uint32_t)(acc[2 * v + 1] >> 32)));
             } else {
                 uint16_t* out = reinterpret_cast<uint16_t*>(C) + row * N + col0;
 #pragma unroll
-                for (int v = 0; v < 8; ++v)
-                    if (col0 + 8 * v < N)
-                        st_v4(out + 8 * v, make_uint4(f32x2_to_bf16x2(acc[8 * v], acc[8 * v + 1]),
-                                                      f32x2_to_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
-                                                      f32x2_to_bf16x2(acc[8 * v + 4], acc[8 * v + 5]),
-                                                      f32x2_to_bf16x2(acc[8 * v + 6], acc[8 * v + 7])));
+                for (int v = 0; v < EPI_COLS / 8; ++v) {
+                    uint32_t h[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        h[j] = f32x2_to_bf16x2(__uint_as_float((uint32_t)acc[4 * v + j]),
+                                               __uint_as_float((uint32_t)(acc[4 * v + j] >> 32)));
+                    if (col0 + 8 * v < N) st_v4(out + 8 * v, make_uint4(h[0], h[1], h[2], h[3]));
+                }
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }

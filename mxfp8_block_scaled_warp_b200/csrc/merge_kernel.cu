@@ -14,7 +14,7 @@ namespace {
 
 constexpr int kMaxRank = 64;
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict__ a,
                      const uint16_t* __restrict__ b, int64_t n, int64_t k, int r, float alpha_over_r,
                      uint8_t* __restrict__ wq, float* __restrict__ ws, uint16_t* __restrict__ w_fq) {
@@ -24,6 +24,15 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     const int64_t bj = blockIdx.x, bi = blockIdx.y;
     const int64_t row0 = bi * 128, col0 = bj * 128;
     const int rmax = (int)min64(128, n - row0);
+
+    // this thread's 8 chunks of W, loaded before the shared-memory staging so
+    // the HBM latency overlaps it
+    uint4 wv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int c = threadIdx.x + 256 * i, rr = c >> 4, c8 = (c & 15) * 8;
+        wv[i] = rr < rmax ? ld_stream(w + (row0 + rr) * k + col0 + c8) : make_uint4(0, 0, 0, 0);
+    }
 
     for (int i = threadIdx.x; i < 128 * r; i += 256) {
         int rr = i / r, j = i - rr * r;
@@ -40,10 +49,10 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     for (int i = 0; i < 8; ++i) {
         const int c = threadIdx.x + 256 * i, rr = c >> 4, c8 = (c & 15) * 8;
         if (rr < rmax) {
-            const uint4 wv = ld_stream(w + (row0 + rr) * k + col0 + c8);
             float d[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) d[e] = 0.0f;
+#pragma unroll 4
             for (int j = 0; j < r; ++j) {
                 const float bj_ = sB[rr * r + j];
                 const float4 a0 = *reinterpret_cast<const float4*>(sA + j * 128 + c8);
@@ -53,7 +62,7 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
                 d[4] = __fmaf_rn(bj_, a1.x, d[4]); d[5] = __fmaf_rn(bj_, a1.y, d[5]);
                 d[6] = __fmaf_rn(bj_, a1.z, d[6]); d[7] = __fmaf_rn(bj_, a1.w, d[7]);
             }
-            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+            const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 float lo = __fmaf_rn(alpha_over_r, d[2 * e], bf16_lo(ww[e]));
@@ -81,6 +90,8 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     }
     __syncthreads();
     const float sc = sc_sh;
+    const bool fast = reciprocal_ok(sc);
+    const float rc = fast ? __frcp_rn(sc) : 0.0f;
 
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -89,7 +100,8 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
             uint32_t e[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                e[j] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(v[i][j]), sc), __fdiv_rn(bf16_hi(v[i][j]), sc));
+                e[j] = fast ? e4m3x2_of_quotients(bf16_lo(v[i][j]), bf16_hi(v[i][j]), sc, rc)
+                            : f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(v[i][j]), sc), __fdiv_rn(bf16_hi(v[i][j]), sc));
             const int64_t off = (row0 + rr) * k + col0 + c8;
             st_v2(wq + off, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
             if (w_fq) {

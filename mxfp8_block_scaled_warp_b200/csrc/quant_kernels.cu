@@ -71,11 +71,18 @@ __device__ __forceinline__ uint4 scale_to_e4m3(const Unit& v, float mul) {
     return make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
 }
 
+// E4M3 codes of fp32(x / s) for the 16 elements of a unit.
 __device__ __forceinline__ uint4 divide_to_e4m3(const Unit& v, float s) {
     uint32_t c[8];
+    if (reciprocal_ok(s)) {
+        const float r = __frcp_rn(s);
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-        c[i] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(v.w[i]), s), __fdiv_rn(bf16_hi(v.w[i]), s));
+        for (int i = 0; i < 8; ++i) c[i] = e4m3x2_of_quotients(bf16_lo(v.w[i]), bf16_hi(v.w[i]), s, r);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            c[i] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(v.w[i]), s), __fdiv_rn(bf16_hi(v.w[i]), s));
+    }
     return make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
 }
 
@@ -86,7 +93,7 @@ __device__ __forceinline__ float fp32_scale(uint32_t a) {
 
 // ----------------------------------------------------------------- MXFP8
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* __restrict__ s,
                    int64_t units) {
     const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
@@ -116,7 +123,7 @@ quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* 
 
 // ----------------------------------------------------------------- FP8 1x128
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 quant_fp8_1x128_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
                        float* __restrict__ s, int64_t units) {
     const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
@@ -175,15 +182,22 @@ quant_fp8_128x128_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ q
     }
     __syncthreads();
     const float sc = sc_sh;
+    const bool fast = reciprocal_ok(sc);
+    const float rc = fast ? __frcp_rn(sc) : 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         int c = threadIdx.x + 256 * i, r = c >> 4, c8 = (c & 15) * 8;
         if (r < rmax) {
-            uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
             uint32_t e[4];
+            if (fast) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                e[j] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[j]), sc), __fdiv_rn(bf16_hi(w[j]), sc));
+                for (int j = 0; j < 4; ++j) e[j] = e4m3x2_of_quotients(bf16_lo(w[j]), bf16_hi(w[j]), sc, rc);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    e[j] = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[j]), sc), __fdiv_rn(bf16_hi(w[j]), sc));
+            }
             st_v2(qb + r * cols + c8, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
         }
     }
@@ -193,7 +207,7 @@ quant_fp8_128x128_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ q
 
 // Pass 1: per-matrix amax as a 15-bit magnitude pattern, atomicMax into
 // amax_bits[b] (zeroed by the launcher).  grid = (slices, matrices).
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 tensor_amax_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, uint32_t* __restrict__ amax_bits) {
     const int64_t b = blockIdx.y;
     const uint4* xb = x + 2 * b * units_per_matrix;
@@ -222,7 +236,7 @@ __device__ __forceinline__ float nvfp4_tensor_scale(uint32_t a) {
 }
 
 // Pass 2: one lane per 16-element block.  grid = (slices, matrices).
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, const uint32_t* __restrict__ amax_bits,
                    uint2* __restrict__ q, uint8_t* __restrict__ s, float* __restrict__ g_out) {
     const int64_t b = blockIdx.y;
@@ -249,11 +263,19 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, const 
             const float S = e4m3_to_f32(code) * g;
             uint32_t packed[2] = {0u, 0u};
             if (S != 0.0f) {
+                if (reciprocal_ok(S)) {
+                    const float rS = __frcp_rn(S);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(bf16_lo(v[i].w[j]), S),
-                                                    __fdiv_rn(bf16_hi(v[i].w[j]), S));
-                    packed[j >> 2] |= byte << (8 * (j & 3));
+                    for (int j = 0; j < 8; ++j)
+                        packed[j >> 2] |= e2m1x2_of_quotients(bf16_lo(v[i].w[j]), bf16_hi(v[i].w[j]), S, rS)
+                                          << (8 * (j & 3));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(bf16_lo(v[i].w[j]), S),
+                                                        __fdiv_rn(bf16_hi(v[i].w[j]), S));
+                        packed[j >> 2] |= byte << (8 * (j & 3));
+                    }
                 }
             }
             st_v2(qb + u, make_uint2(packed[0], packed[1]));
@@ -275,7 +297,7 @@ __device__ __forceinline__ void store_bf16x16(uint4* out, int64_t u, const float
 // fmt: 0 = 1x128 (fp32 scale per 8 units), 2 = MXFP8 (E8M0 per 2 units),
 // 1 = 128x128 (fp32 scale per 128x128 block).
 template <int kFmt>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales, uint4* __restrict__ out,
                    int64_t units, int64_t rows, int64_t cols) {
     const int64_t stride = (int64_t)gridDim.x * kThreads;
@@ -307,7 +329,7 @@ dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales,
     }
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 dequant_nvfp4_kernel(const uint2* __restrict__ q, const uint8_t* __restrict__ s, const float* __restrict__ g,
                      uint4* __restrict__ out, int64_t units, int64_t units_per_matrix) {
     const int64_t stride = (int64_t)gridDim.x * kThreads;
