@@ -154,7 +154,7 @@ fpq_status fpq_quantize_block(fpq_format fmt, const void* x, int64_t batch, int6
     const DeviceState* d = device_state(&st);
     if (!d) return st;
     return from_cuda(fpq::launch_quantize(fmt, x, batch, rows, cols, q, scales, tensor_scale, workspace,
-                                          d->sms, (cudaStream_t)stream), "quantize launch");
+                                          d->err, d->sms, (cudaStream_t)stream), "quantize launch");
 }
 
 fpq_status fpq_dequantize(fpq_format fmt, const void* q, const void* scales, const float* tensor_scale,

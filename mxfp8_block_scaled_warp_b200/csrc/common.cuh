@@ -92,40 +92,46 @@ __device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t c2) {
 // ----------------------------------------------------------------- exact quotient codes
 //
 // The fp32-scale formats define a code as the rounding of the correctly
-// rounded fp32 quotient q(x) = fp32(x / s).  A division per element is the
-// slow part of the quantizers (it runs on the reciprocal unit), so the codes
-// are obtained from t = x * r with r = fp32(1/s) instead, and checked:
-//   |t - q(x)| < 3 ulp (ulp of the binade of x/s; at most 6 ulp of the binade
-//   below), because r and t each add at most half an ulp of relative error
-//   and q(x) itself is within half an ulp of x/s.
-// Rounding to a narrow format is monotone in the value, so if the magnitude
-// patterns |t| - 16 and |t| + 16 round to the same code, every value between
-// them -- q(x) included -- rounds to that code.  Otherwise (a quotient within
-// 16 ulp of a rounding boundary, rare) the code is taken from the IEEE
-// division itself.  The caller guarantees r is finite (s >= 2^-126).
-// The sign of the code is the sign of x (s > 0), so -0 keeps its sign.
+// rounded fp32 quotient q = fp32(x / s).  Instead of a division per element
+// (which runs on the reciprocal unit), the code is read off two products
+// that bracket q:
+//   r = fp32(1/s), r_lo = fp32(r (1 - 2^-20)), r_hi = fp32(r (1 + 2^-20))
+// give r_lo < (1/s)(1 - 2^-21) and r_hi > (1/s)(1 + 2^-21), so for x > 0
+//   fp32(x r_lo) < (x/s)(1 - 2^-24) <= q <= (x/s)(1 + 2^-24) < fp32(x r_hi)
+// (mirrored for x < 0; all zero for x = 0).  Rounding to a narrow format is
+// monotone in the value, so when both bracket ends round to the same code,
+// q rounds to it too.  Otherwise (q within about 2^-20 relative of a
+// rounding boundary, rare) the code is taken from the IEEE division itself.
+// Values so small that the products are fp32-subnormal are far below the
+// smallest nonzero code and round to signed zero on every path.  The caller
+// guarantees 1/s is a normal fp32 number (s >= 2^-126, see reciprocal_ok).
 
-__device__ __forceinline__ uint32_t abs_pattern(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+struct QuotientBracket {
+    float s, lo, hi;
+};
+
+__device__ __forceinline__ QuotientBracket quotient_bracket(float s) {
+    const float r = __frcp_rn(s);
+    return QuotientBracket{s, __fmul_rn(r, 1.0f - 0x1p-20f), __fmul_rn(r, 1.0f + 0x1p-20f)};
+}
 
 // E4M3 codes of fp32(x0/s) (bits 0-7) and fp32(x1/s) (bits 8-15).
-__device__ __forceinline__ uint32_t e4m3x2_of_quotients(float x0, float x1, float s, float r) {
-    const uint32_t m0 = abs_pattern(x0 * r), m1 = abs_pattern(x1 * r);
-    uint32_t lo = f32x2_to_e4m3x2(__uint_as_float(m0 - min(m0, 16u)), __uint_as_float(m1 - min(m1, 16u)));
-    const uint32_t hi = f32x2_to_e4m3x2(__uint_as_float(m0 + 16u), __uint_as_float(m1 + 16u));
-    if (lo != hi) lo = f32x2_to_e4m3x2(fabsf(__fdiv_rn(x0, s)), fabsf(__fdiv_rn(x1, s)));
-    return lo | ((__float_as_uint(x0) >> 24) & 0x80u) | ((__float_as_uint(x1) >> 16) & 0x8000u);
+__device__ __forceinline__ uint32_t e4m3x2_of_quotients(float x0, float x1, const QuotientBracket& b) {
+    uint32_t lo = f32x2_to_e4m3x2(__fmul_rn(x0, b.lo), __fmul_rn(x1, b.lo));
+    const uint32_t hi = f32x2_to_e4m3x2(__fmul_rn(x0, b.hi), __fmul_rn(x1, b.hi));
+    if (lo != hi) lo = f32x2_to_e4m3x2(__fdiv_rn(x0, b.s), __fdiv_rn(x1, b.s));
+    return lo;
 }
 
 // E2M1 codes of fp32(x0/s) (bits 0-3) and fp32(x1/s) (bits 4-7).
-__device__ __forceinline__ uint32_t e2m1x2_of_quotients(float x0, float x1, float s, float r) {
-    const uint32_t m0 = abs_pattern(x0 * r), m1 = abs_pattern(x1 * r);
-    uint32_t lo = f32x2_to_e2m1x2(__uint_as_float(m0 - min(m0, 16u)), __uint_as_float(m1 - min(m1, 16u)));
-    const uint32_t hi = f32x2_to_e2m1x2(__uint_as_float(m0 + 16u), __uint_as_float(m1 + 16u));
-    if (lo != hi) lo = f32x2_to_e2m1x2(fabsf(__fdiv_rn(x0, s)), fabsf(__fdiv_rn(x1, s)));
-    return lo | ((__float_as_uint(x0) >> 28) & 0x8u) | ((__float_as_uint(x1) >> 24) & 0x80u);
+__device__ __forceinline__ uint32_t e2m1x2_of_quotients(float x0, float x1, const QuotientBracket& b) {
+    uint32_t lo = f32x2_to_e2m1x2(__fmul_rn(x0, b.lo), __fmul_rn(x1, b.lo));
+    const uint32_t hi = f32x2_to_e2m1x2(__fmul_rn(x0, b.hi), __fmul_rn(x1, b.hi));
+    if (lo != hi) lo = f32x2_to_e2m1x2(__fdiv_rn(x0, b.s), __fdiv_rn(x1, b.s));
+    return lo;
 }
 
-// Whether the multiply-and-check path applies for divisor s (1/s finite).
+// Whether the bracket applies for divisor s (1/s a normal fp32 number).
 __device__ __forceinline__ bool reciprocal_ok(float s) { return s >= 1.17549435e-38f; }
 
 // ----------------------------------------------------------------- absmax

@@ -10,7 +10,7 @@ namespace fpq {
 // Quantize `batch` dense row-major bf16 matrices [rows, cols] (fmt: fpq_format).
 cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows, int64_t cols,
                             void* q, void* scales, float* tensor_scale, void* workspace,
-                            int sms, cudaStream_t st);
+                            uint32_t* err, int sms, cudaStream_t st);
 
 cudaError_t launch_dequantize(int fmt, const void* q, const void* scales, const float* tensor_scale,
                               int64_t batch, int64_t rows, int64_t cols, void* out, int sms,

@@ -14,66 +14,112 @@ namespace {
 
 constexpr int kMaxRank = 64;
 
+// One CTA per 128x128 block of W, 256 threads as a 16 x 16 grid: thread
+// (ty, tx) owns rows 8 ty .. 8 ty + 7 and columns 8 tx .. 8 tx + 7 of the
+// block, so each rank step j costs it two 32-byte shared loads (B column j of
+// its rows, A row j of its columns) for 64 fused multiply-adds.  The delta is
+// accumulated in fp32 with j ascending from zero, exactly as the definition
+// states, then merged into W and rounded to bf16; the block's amax, scale and
+// E4M3 codes follow, and optionally the fake-quantized bf16 copy.
 __global__ void __launch_bounds__(256, 2)
 lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict__ a,
                      const uint16_t* __restrict__ b, int64_t n, int64_t k, int r, float alpha_over_r,
                      uint8_t* __restrict__ wq, float* __restrict__ ws, uint16_t* __restrict__ w_fq) {
-    extern __shared__ float sm[];
-    float* sB = sm;                 // [128][r]   rows of B for this block row
-    float* sA = sm + 128 * r;       // [r][128]   columns of A for this block column
+    extern __shared__ __align__(16) float sm[];
+    float* sBt = sm;                // [r][128]  B^T for this block row: sBt[j][i] = B[row0 + i][j]
+    float* sA = sm + 128 * r;       // [r][128]  A for this block column: sA[j][c] = A[j][col0 + c]
     const int64_t bj = blockIdx.x, bi = blockIdx.y;
     const int64_t row0 = bi * 128, col0 = bj * 128;
     const int rmax = (int)min64(128, n - row0);
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 
-    // this thread's 8 chunks of W, loaded before the shared-memory staging so
-    // the HBM latency overlaps it
+    // this thread's 8 rows x 8 columns of W (one 16-byte load per row), issued
+    // first so the HBM latency overlaps the staging and the rank-r product
     uint4 wv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int c = threadIdx.x + 256 * i, rr = c >> 4, c8 = (c & 15) * 8;
-        wv[i] = rr < rmax ? ld_stream(w + (row0 + rr) * k + col0 + c8) : make_uint4(0, 0, 0, 0);
+        const int rr = 8 * ty + i;
+        wv[i] = rr < rmax ? ld_stream(w + (row0 + rr) * k + col0 + 8 * tx) : make_uint4(0, 0, 0, 0);
     }
-
-    for (int i = threadIdx.x; i < 128 * r; i += 256) {
-        int rr = i / r, j = i - rr * r;
-        sB[i] = rr < rmax ? __uint_as_float((uint32_t)b[(row0 + rr) * r + j] << 16) : 0.0f;
-        int jj = i >> 7, cc = i & 127;
-        sA[i] = __uint_as_float((uint32_t)a[(int64_t)jj * k + col0 + cc] << 16);
+    // stage the block's B rows ([128, r] contiguous) transposed, and A's r rows
+    // of 128 columns, as fp32; every 16-byte load is issued before any store
+    constexpr int kMaxChunks = 128 * kMaxRank * 2 / 16 / 256;         // 4 per operand at r = 64
+    const int chunks = 128 * r * 2 / 16;                               // 16-byte chunks per operand
+    uint4 bc[kMaxChunks], ac[kMaxChunks];
+#pragma unroll
+    for (int i = 0; i < kMaxChunks; ++i) {
+        const int c = threadIdx.x + 256 * i;
+        if (c < chunks) {
+            // B elements e .. e+7 of the block (row (e+h) / r, rank (e+h) % r);
+            // only the block's first rmax * r elements exist
+            const int e = 8 * c, valid = rmax * r;
+            if (e + 8 <= valid) {
+                bc[i] = ld_stream(b + row0 * r + e);
+            } else {
+                uint16_t h[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) h[t] = (e + t < valid) ? b[row0 * r + e + t] : (uint16_t)0;
+                bc[i] = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16),
+                                   h[4] | ((uint32_t)h[5] << 16), h[6] | ((uint32_t)h[7] << 16));
+            }
+            const int jj = c >> 4, cc = 8 * (c & 15);                  // A row jj, columns cc .. cc + 7
+            ac[i] = ld_stream(a + (int64_t)jj * k + col0 + cc);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxChunks; ++i) {
+        const int c = threadIdx.x + 256 * i;
+        if (c < chunks) {
+            const uint32_t bw[4] = {bc[i].x, bc[i].y, bc[i].z, bc[i].w};
+            const int e = 8 * c;
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const int rr = (e + h) / r, j = (e + h) - rr * r;
+                sBt[j * 128 + rr] = (h & 1) ? bf16_hi(bw[h >> 1]) : bf16_lo(bw[h >> 1]);
+            }
+            const uint32_t aw[4] = {ac[i].x, ac[i].y, ac[i].z, ac[i].w};
+            float* dst = sA + (c >> 4) * 128 + 8 * (c & 15);
+            *reinterpret_cast<float4*>(dst) = make_float4(bf16_lo(aw[0]), bf16_hi(aw[0]), bf16_lo(aw[1]), bf16_hi(aw[1]));
+            *reinterpret_cast<float4*>(dst + 4) = make_float4(bf16_lo(aw[2]), bf16_hi(aw[2]), bf16_lo(aw[3]), bf16_hi(aw[3]));
+        }
     }
     __syncthreads();
 
-    // merged bf16 weight of this thread's 8 chunks of 8 elements
+    float d[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d[i][e] = 0.0f;
+#pragma unroll 2
+    for (int j = 0; j < r; ++j) {
+        const float4 b0 = *reinterpret_cast<const float4*>(sBt + j * 128 + 8 * ty);
+        const float4 b1 = *reinterpret_cast<const float4*>(sBt + j * 128 + 8 * ty + 4);
+        const float4 a0 = *reinterpret_cast<const float4*>(sA + j * 128 + 8 * tx);
+        const float4 a1 = *reinterpret_cast<const float4*>(sA + j * 128 + 8 * tx + 4);
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) d[i][e] = __fmaf_rn(bv[i], av[e], d[i][e]);
+    }
+
+    // merge, round to bf16, block amax
     uint32_t v[8][4];
     uint32_t m = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int c = threadIdx.x + 256 * i, rr = c >> 4, c8 = (c & 15) * 8;
-        if (rr < rmax) {
-            float d[8];
+        const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) d[e] = 0.0f;
-#pragma unroll 4
-            for (int j = 0; j < r; ++j) {
-                const float bj_ = sB[rr * r + j];
-                const float4 a0 = *reinterpret_cast<const float4*>(sA + j * 128 + c8);
-                const float4 a1 = *reinterpret_cast<const float4*>(sA + j * 128 + c8 + 4);
-                d[0] = __fmaf_rn(bj_, a0.x, d[0]); d[1] = __fmaf_rn(bj_, a0.y, d[1]);
-                d[2] = __fmaf_rn(bj_, a0.z, d[2]); d[3] = __fmaf_rn(bj_, a0.w, d[3]);
-                d[4] = __fmaf_rn(bj_, a1.x, d[4]); d[5] = __fmaf_rn(bj_, a1.y, d[5]);
-                d[6] = __fmaf_rn(bj_, a1.z, d[6]); d[7] = __fmaf_rn(bj_, a1.w, d[7]);
-            }
-            const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float lo = __fmaf_rn(alpha_over_r, d[2 * e], bf16_lo(ww[e]));
-                float hi = __fmaf_rn(alpha_over_r, d[2 * e + 1], bf16_hi(ww[e]));
-                v[i][e] = f32x2_to_bf16x2(lo, hi);
-                m = max2(m, abs2(v[i][e]));
-            }
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __fmaf_rn(alpha_over_r, d[i][2 * e], bf16_lo(ww[e]));
+            const float hi = __fmaf_rn(alpha_over_r, d[i][2 * e + 1], bf16_hi(ww[e]));
+            v[i][e] = f32x2_to_bf16x2(lo, hi);
         }
+        if (8 * ty + i < rmax)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m = max2(m, abs2(v[i][e]));
     }
-
-    // 128x128 block amax -> fp32 scale
     m = hmax2(m);
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -91,18 +137,18 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     __syncthreads();
     const float sc = sc_sh;
     const bool fast = reciprocal_ok(sc);
-    const float rc = fast ? __frcp_rn(sc) : 0.0f;
+    const QuotientBracket br = quotient_bracket(fast ? sc : 1.0f);
 
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int c = threadIdx.x + 256 * i, rr = c >> 4, c8 = (c & 15) * 8;
+        const int rr = 8 * ty + i;
         if (rr < rmax) {
             uint32_t e[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                e[j] = fast ? e4m3x2_of_quotients(bf16_lo(v[i][j]), bf16_hi(v[i][j]), sc, rc)
+                e[j] = fast ? e4m3x2_of_quotients(bf16_lo(v[i][j]), bf16_hi(v[i][j]), br)
                             : f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(v[i][j]), sc), __fdiv_rn(bf16_hi(v[i][j]), sc));
-            const int64_t off = (row0 + rr) * k + col0 + c8;
+            const int64_t off = (row0 + rr) * k + col0 + 8 * tx;
             st_v2(wq + off, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
             if (w_fq) {
                 uint32_t h[4];

@@ -42,4 +42,21 @@ inline cudaError_t make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// General 2-D row-major tensor map: [rows, cols] elements of `elem_bytes`,
+// row pitch `pitch` bytes, box box_rows x box_cols elements.
+inline cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint32_t elem_bytes,
+                                uint64_t rows, uint64_t cols, uint64_t pitch, uint32_t box_rows, uint32_t box_cols,
+                                CUtensorMapSwizzle swizzle) {
+    (void)elem_bytes;
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {pitch};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace fpq

@@ -223,7 +223,7 @@ def test_moe_prequant_full_size_batch(fpq, orc):
 
 # ------------------------------------------------------------------ LoRA merge + fake-quant
 
-@pytest.mark.parametrize("n,k,r", [(256, 384, 16), (200, 256, 1), (130, 512, 64), (1, 128, 3)])
+@pytest.mark.parametrize("n,k,r", [(256, 384, 16), (200, 256, 1), (130, 512, 64), (1, 128, 3), (133, 256, 3), (200, 384, 5)])
 def test_lora_merge_fakequant_small(fpq, orc, n, k, r):
     w = rand((n, k), 40, std=0.02)
     a = rand((r, k), 41, std=0.01)
