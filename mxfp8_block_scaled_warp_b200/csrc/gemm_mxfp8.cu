@@ -15,8 +15,13 @@
 //           tcgen05.cp of the scales, then 4 x tcgen05.mma kind::mxf8f6f4
 //           (K = 32 each, scale byte selected per MMA), tcgen05.commit
 //   warps 4-7 epilogue: tcgen05.ld of the accumulator, convert, store
-// Every wait on an mbarrier is bounded by wall time; on expiry the kernel
-// records FPQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
+// Every wait on an mbarrier is bounded by wall time (4 s, or
+// FPQ_WAIT_TIMEOUT_MS); on expiry the kernel records FPQ_ERR_DEVICE_TIMEOUT in
+// the device error word and unwinds (TMEM freed, no store).  For testing
+// that path, FPQ_DEBUG_GEMM_STALL=1 makes the producer declare more TMA bytes
+// per stage than it loads, so the stage barriers never complete: every load
+// it issues still lands, and the waits run out instead of hanging.
+#include <cstdlib>
 #include <cuda.h>
 
 #include "common.cuh"
@@ -38,7 +43,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = BN;            // scale columns follow the accumulator
 constexpr uint32_t SF_COLS_PER_STAGE = 16;  // 4 (A) + 8 (B), padded
 constexpr int NUM_THREADS = 256;
-constexpr uint64_t kTimeoutNs = 4000000000ull;
+constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
 
 struct __align__(1024) Smem {
     uint8_t a[STAGES][A_TILE];
@@ -61,13 +66,13 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
-__device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
+__device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err, uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > kTimeoutNs) {
+        if (globaltimer() - t0 > timeout_ns) {
             raise_device_error(err, FPQ_ERR_DEVICE_TIMEOUT);
             return false;
         }
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
                   const int32_t* __restrict__ offsets, int groups, int64_t M, int64_t N, int64_t K,
-                  void* __restrict__ C, int c_f32, uint32_t* err) {
+                  void* __restrict__ C, int c_f32, uint32_t* err, uint64_t timeout_ns, uint32_t extra_tx) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -177,8 +182,8 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             for (int kt = 0; kt < KT; ++kt) {
                 const int s = kt % STAGES;
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
-                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
-                mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE);
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err, timeout_ns)) break;
+                mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE + extra_tx);
                 tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)a_row0);
                 tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)b_row0);
             }
@@ -213,7 +218,7 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 if (kt >= KT) break;
                 const int s = kt % STAGES;
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
-                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) { alive = false; break; }
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err, timeout_ns)) { alive = false; break; }
                 *reinterpret_cast<uint4*>(sm.sfa[s] + lane * 16) =
                     make_uint4(pick(ca[0], j), pick(ca[1], j), pick(ca[2], j), pick(ca[3], j));
                 *reinterpret_cast<uint4*>(sm.sfb[s] + lane * 16) =
@@ -236,7 +241,7 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             for (int kt = 0; kt < KT; ++kt) {
                 const int s = kt % STAGES;
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
-                if (!wait_or_timeout(&sm.full[s], ph, err)) { ok = false; break; }
+                if (!wait_or_timeout(&sm.full[s], ph, err, timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sf_col = tmem + SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
                 tmem_cp_32x128b_warpx4(sf_col + 0, smem_desc(smem_u32(sm.sfa[s]), 0, 128, kLayoutNone));
@@ -259,7 +264,7 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int q = warp & 3;                       // TMEM lane quadrant of this warp
         const int64_t row = a_row0 + 32 * q + lane;
         const bool row_ok = row < a_rows_end;
-        if (wait_or_timeout(&sm.tmem_full, 0, err)) {
+        if (wait_or_timeout(&sm.tmem_full, 0, err, timeout_ns)) {
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
@@ -296,6 +301,17 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
 int smem_bytes() { return (int)sizeof(Smem) + 1024; }
 
+// Wait limit and the stall switch for the timeout test (see the file header).
+uint64_t wait_timeout_ns() {
+    const char* v = std::getenv("FPQ_WAIT_TIMEOUT_MS");
+    const long ms = v ? std::atol(v) : 0;
+    return ms > 0 ? (uint64_t)ms * 1000000ull : kDefaultTimeoutNs;
+}
+uint32_t debug_extra_tx() {
+    const char* v = std::getenv("FPQ_DEBUG_GEMM_STALL");
+    return (v && v[0] == '1') ? 16u : 0u;
+}
+
 cudaError_t launch(const void* aq, const void* as, const void* bq, const void* bs, const int32_t* offsets,
                    int groups, int64_t M, int64_t N, int64_t K, void* c, int c_f32, uint32_t* err,
                    int64_t grid, cudaStream_t st) {
@@ -308,7 +324,8 @@ cudaError_t launch(const void* aq, const void* as, const void* bq, const void* b
     if (e != cudaSuccess) return e;
     if (grid < 1) return cudaSuccess;
     gemm_mxfp8_kernel<<<(unsigned)grid, NUM_THREADS, smem_bytes(), st>>>(
-        ta, tb, (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err);
+        ta, tb, (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err, wait_timeout_ns(),
+        debug_extra_tx());
     return cudaGetLastError();
 }
 
