@@ -89,6 +89,16 @@ __device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t c2) {
                        __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
 }
 
+// ----------------------------------------------------------------- dependent launch
+
+// Wait until the grids this one depends on (programmatic dependent launch)
+// have completed and their memory operations are visible; a no-op for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow dependent grids to be scheduled; they still wait (pdl_wait) for this
+// grid's completion before touching its results.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------- exact quotient codes
 //
 // The fp32-scale formats define a code as the rounding of the correctly

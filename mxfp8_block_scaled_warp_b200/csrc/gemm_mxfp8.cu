@@ -113,6 +113,7 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int sf_pitch = (int)(K / 32);
 
     if (threadIdx.x == 0) {
+        pdl_wait();    // the group offsets may come from the preceding grid
         // map this CTA to (group, m tile, n tile)
         int valid = 0, g = 0, mt = 0, nt = 0;
         int32_t rb = 0, re = (int32_t)M;
@@ -168,6 +169,9 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // Everything above touched only shared memory and TMEM; global inputs
+    // and the output are accessed after the preceding grids complete.
+    pdl_wait();
 
     const int64_t a_row0 = (int64_t)sm.row_begin + (int64_t)sm.m_tile * BM;   // first A row of the tile
     const int64_t a_rows_end = sm.row_end;                                     // rows >= this are masked
@@ -323,10 +327,9 @@ cudaError_t launch(const void* aq, const void* as, const void* bq, const void* b
     e = cudaFuncSetAttribute(gemm_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
     if (e != cudaSuccess) return e;
     if (grid < 1) return cudaSuccess;
-    gemm_mxfp8_kernel<<<(unsigned)grid, NUM_THREADS, smem_bytes(), st>>>(
-        ta, tb, (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err, wait_timeout_ns(),
-        debug_extra_tx());
-    return cudaGetLastError();
+    return launch_pdl(gemm_mxfp8_kernel, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta, tb,
+                      (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err,
+                      wait_timeout_ns(), debug_extra_tx());
 }
 
 }  // namespace

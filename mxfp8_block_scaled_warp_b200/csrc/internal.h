@@ -37,4 +37,24 @@ cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void
 // Set the per-thread detail string returned by fpq_last_error_detail().
 void set_error_detail(const char* what);
 
+// Launch with programmatic dependent launch allowed: the kernel may become
+// resident while the previous kernel in the stream is still finishing, so it
+// must execute pdl_wait() (griddepcontrol.wait) before it touches global
+// memory that earlier work writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace fpq

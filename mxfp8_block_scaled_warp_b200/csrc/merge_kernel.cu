@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(256, 2)
 lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict__ a,
                      const uint16_t* __restrict__ b, int64_t n, int64_t k, int r, float alpha_over_r,
                      uint8_t* __restrict__ wq, float* __restrict__ ws, uint16_t* __restrict__ w_fq) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     extern __shared__ __align__(16) float sm[];
     float* sBt = sm;                // [r][128]  B^T for this block row: sBt[j][i] = B[row0 + i][j]
     float* sA = sm + 128 * r;       // [r][128]  A for this block column: sA[j][c] = A[j][col0 + c]

@@ -99,6 +99,7 @@ __device__ __forceinline__ float fp32_scale(uint32_t a) {
 __global__ void __launch_bounds__(kThreads, 3)
 quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* __restrict__ s,
                    int64_t units) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
     for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units; base += stride) {
         Unit v[kUnroll];
@@ -129,6 +130,7 @@ quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* 
 __global__ void __launch_bounds__(kThreads, 3)
 quant_fp8_1x128_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
                        float* __restrict__ s, int64_t units) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
     for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units; base += stride) {
         Unit v[kUnroll];
@@ -223,6 +225,7 @@ __device__ __forceinline__ void qb_issue(const CUtensorMap* map, int64_t idx, in
 __global__ void __launch_bounds__(256, 2)
 quant_fp8_128x128_kernel(const __grid_constant__ CUtensorMap tmX, uint8_t* __restrict__ q, float* __restrict__ s,
                          int64_t batch, int64_t rows, int64_t cols, uint32_t* err) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     extern __shared__ __align__(128) uint8_t qb_smem[];
     __shared__ __align__(8) uint64_t full[QB_STAGES];
     __shared__ uint32_t red[8];
@@ -300,6 +303,7 @@ quant_fp8_128x128_kernel(const __grid_constant__ CUtensorMap tmX, uint8_t* __res
 // amax_bits[b] (zeroed by the launcher).  grid = (slices, matrices).
 __global__ void __launch_bounds__(kThreads, 3)
 tensor_amax_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, uint32_t* __restrict__ amax_bits) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t b = blockIdx.y;
     const uint4* xb = x + 2 * b * units_per_matrix;
     uint32_t m = 0;
@@ -330,6 +334,7 @@ __device__ __forceinline__ float nvfp4_tensor_scale(uint32_t a) {
 __global__ void __launch_bounds__(kThreads, 3)
 quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, const uint32_t* __restrict__ amax_bits,
                    uint2* __restrict__ q, uint8_t* __restrict__ s, float* __restrict__ g_out) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t b = blockIdx.y;
     const uint4* xb = x + 2 * b * units_per_matrix;
     uint2* qb = q + b * units_per_matrix;
@@ -391,6 +396,7 @@ template <int kFmt>
 __global__ void __launch_bounds__(kThreads, 3)
 dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales, uint4* __restrict__ out,
                    int64_t units, int64_t rows, int64_t cols) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     const int64_t units_per_row = cols / 16;
     for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
@@ -423,6 +429,7 @@ dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales,
 __global__ void __launch_bounds__(kThreads, 3)
 dequant_nvfp4_kernel(const uint2* __restrict__ q, const uint8_t* __restrict__ s, const float* __restrict__ g,
                      uint4* __restrict__ out, int64_t units, int64_t units_per_matrix) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
         uint2 c = q[u];
