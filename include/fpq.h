@@ -111,7 +111,8 @@ FPQ_API const char* fpq_status_string(fpq_status status);
 FPQ_API const char* fpq_last_error_detail(void);
 
 /* Bytes of device workspace fpq_quantize_block needs for `fmt` and `batch`
- * (NVFP4: 4 bytes per batch item for the tensor amax; 0 otherwise). */
+ * (NVFP4: 16 + 8 * batch bytes -- a work-item counter, and per batch item
+ * the tensor amax and a progress counter of the amax pass; 0 otherwise). */
 FPQ_API size_t fpq_quantize_workspace_bytes(fpq_format fmt, int64_t batch);
 
 /*
@@ -220,8 +221,10 @@ FPQ_API fpq_status fpq_grouped_scaled_gemm(fpq_format fmt, const void* aq, const
  * plugin running inside a host application that owns the device memory pool.
  * The pages describe no such entry point; it exists for these callers only.
  *
- * Scratch: a library-owned static device array of FPQ_NOALLOC_NVFP4_MAX_BATCH
- * words (16 KiB) on every GPU that loads the library, held until the process
+ * Scratch: a library-owned static device array of 4 + 2 *
+ * FPQ_NOALLOC_NVFP4_MAX_BATCH 32-bit words (32 KiB + 16 bytes: the NVFP4
+ * workspace for the largest batch) on every GPU that loads the library, held
+ * until the process
  * exits.  No call allocates or frees anything.  batch > the maximum gives
  * FPQ_ERR_INVALID_ARG.  The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current; make that

@@ -134,7 +134,7 @@ const char* fpq_status_string(fpq_status s) {
 const char* fpq_last_error_detail(void) { return t_detail; }
 
 size_t fpq_quantize_workspace_bytes(fpq_format fmt, int64_t batch) {
-    return (fmt == FPQ_NVFP4 && batch > 0) ? sizeof(uint32_t) * (size_t)batch : 0;
+    return (fmt == FPQ_NVFP4 && batch > 0) ? sizeof(uint32_t) * (size_t)fpq::nvfp4_workspace_words(batch) : 0;
 }
 
 fpq_status fpq_quantize_block(fpq_format fmt, const void* x, int64_t batch, int64_t rows, int64_t cols,

@@ -141,6 +141,47 @@ __device__ __forceinline__ uint32_t e2m1x2_of_quotients(float x0, float x1, cons
     return lo;
 }
 
+// ----------------------------------------------------------------- per-block scale tables
+//
+// For a bf16 amax a = (1 + m/128) 2^(E-127) (m: 7-bit mantissa field, E:
+// exponent field) the quotient a / d by a constant d is
+// fp32((1 + m/128) / d) 2^(E-127) exactly whenever the result is a normal
+// fp32 number (scaling by a power of two commutes with rounding there), and
+// likewise the reciprocal and the bracket ends of a scale.  So the per-block
+// divisions reduce to 128-entry tables indexed by m plus an exponent add.
+
+struct ScaleTables {
+    uint32_t s[128];     // fp32((1 + m/128) / d)
+    uint32_t lo[128];    // bracket ends for quotients by s: r (1 - 2^-20), r (1 + 2^-20), r = fp32(1 / s)
+    uint32_t hi[128];
+};
+
+// Threads 0..127 each fill one entry; the caller synchronizes afterwards.
+__device__ __forceinline__ void init_scale_tables(ScaleTables& t, float d) {
+    const int m = threadIdx.x;
+    if (m < 128) {
+        const float sm = __fdiv_rn(1.0f + (float)m * 0x1p-7f, d);
+        const float r = __frcp_rn(sm);
+        t.s[m] = __float_as_uint(sm);
+        t.lo[m] = __float_as_uint(__fmul_rn(r, 1.0f - 0x1p-20f));
+        t.hi[m] = __float_as_uint(__fmul_rn(r, 1.0f + 0x1p-20f));
+    }
+}
+
+// Scale s = fp32(a / d) of a bf16 magnitude pattern a and its bracket ends,
+// when E is in [e_min, 254] (the caller's e_min keeps s and 1/s normal);
+// false otherwise (zero, tiny, infinite or NaN amax: use the division path).
+__device__ __forceinline__ bool table_scale(const ScaleTables& t, uint32_t a, int e_min, float& s, float& lo,
+                                            float& hi) {
+    const int E = (int)(a >> 7), m = (int)(a & 0x7Fu);
+    if (E < e_min || E > 254) return false;
+    const int k = (E - 127) << 23;
+    s = __uint_as_float(t.s[m] + (uint32_t)k);
+    lo = __uint_as_float(t.lo[m] - (uint32_t)k);
+    hi = __uint_as_float(t.hi[m] - (uint32_t)k);
+    return true;
+}
+
 // Whether the bracket applies for divisor s (1/s a normal fp32 number).
 __device__ __forceinline__ bool reciprocal_ok(float s) { return s >= 1.17549435e-38f; }
 

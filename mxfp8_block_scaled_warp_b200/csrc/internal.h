@@ -7,6 +7,11 @@
 
 namespace fpq {
 
+// 32-bit words of NVFP4 quantize workspace for `batch` matrices: a 64-bit
+// work-item counter (4 words with padding), one amax word and one progress
+// counter per matrix.
+inline int64_t nvfp4_workspace_words(int64_t batch) { return 4 + 2 * batch; }
+
 // Quantize `batch` dense row-major bf16 matrices [rows, cols] (fmt: fpq_format).
 cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows, int64_t cols,
                             void* q, void* scales, float* tensor_scale, void* workspace,

@@ -16,8 +16,11 @@
 
 namespace {
 
-// One amax word per batch item; FPQ_NOALLOC_NVFP4_MAX_BATCH words (16 KiB).
-__device__ __align__(256) uint32_t g_noalloc_amax[FPQ_NOALLOC_NVFP4_MAX_BATCH];
+// The NVFP4 quantize workspace for up to FPQ_NOALLOC_NVFP4_MAX_BATCH
+// matrices: a work-item counter plus one amax word and one progress counter
+// per matrix (4 + 2 * 4096 words, 32 KiB + 16 bytes).
+constexpr int kScratchWords = 4 + 2 * FPQ_NOALLOC_NVFP4_MAX_BATCH;
+__device__ __align__(256) uint32_t g_noalloc_amax[kScratchWords];
 
 constexpr int kMaxDevices = 64;
 void* g_scratch[kMaxDevices] = {};
@@ -57,7 +60,7 @@ extern "C" FPQ_API fpq_status fpq_quantize_nvfp4_noalloc(const void* x, int64_t 
     void* scratch = nullptr;
     fpq_status st = scratch_on_current_device(&scratch);
     if (st != FPQ_OK) return st;
-    // The quantizer zeroes the amax words it uses before the amax pass.
+    // The quantizer zeroes the workspace words it uses before it starts.
     return fpq_quantize_block(FPQ_NVFP4, x, batch, rows, cols, q, scales, tensor_scale, scratch,
-                              sizeof(uint32_t) * (size_t)FPQ_NOALLOC_NVFP4_MAX_BATCH, stream);
+                              sizeof(uint32_t) * (size_t)kScratchWords, stream);
 }

@@ -127,27 +127,46 @@ quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* 
 
 // ----------------------------------------------------------------- FP8 1x128
 
-__global__ void __launch_bounds__(kThreads, 3)
+// One unit per thread per iteration, with the next iteration's unit loaded
+// before this one is encoded; few registers let six CTAs share an SM, and
+// the grid is sized to exactly that residency (grid-stride loop).
+constexpr int Q1_MIN_BLOCKS = 6;
+
+__global__ void __launch_bounds__(kThreads, Q1_MIN_BLOCKS)
 quant_fp8_1x128_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
                        float* __restrict__ s, int64_t units) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
-    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units; base += stride) {
-        Unit v[kUnroll];
+    __shared__ ScaleTables tab;                      // s = fp32(amax / 448) and its bracket, by mantissa
+    init_scale_tables(tab, 448.0f);
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    Unit cur;
+    if (u < units) cur = load_unit(x, u);
+    __syncthreads();
+    // The 8 lanes of a block are in range or out of range together (units
+    // and stride are multiples of 8), so the shuffles stay converged.
+    for (; u - threadIdx.x < units; u += stride) {
+        Unit nxt;
+        if (u + stride < units) nxt = load_unit(x, u + stride);
+        const uint32_t a = group_max<8>(u < units ? unit_absmax(cur) : 0u);
+        if (u < units) {
+            // exponent field >= 10 keeps s = fp32(amax / 448) and 1/s normal
+            float sc, lo, hi;
+            uint4 out;
+            if (table_scale(tab, a, 10, sc, lo, hi)) {
+                const QuotientBracket br{sc, lo, hi};
+                uint32_t c[8];
 #pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            int64_t u = base + i * kThreads + threadIdx.x;
-            if (u < units) v[i] = load_unit(x, u);
-        }
-#pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            int64_t u = base + i * kThreads + threadIdx.x;
-            uint32_t a = group_max<8>(u < units ? unit_absmax(v[i]) : 0u);
-            if (u >= units) continue;
-            float sc = fp32_scale(a);
-            st_v4(q + u, divide_to_e4m3(v[i], sc));
+                for (int j = 0; j < 8; ++j) c[j] = e4m3x2_of_quotients(bf16_lo(cur.w[j]), bf16_hi(cur.w[j]), br);
+                out = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+            } else {
+                sc = fp32_scale(a);
+                out = divide_to_e4m3(cur, sc);
+            }
+            st_v4(q + u, out);
             if ((u & 7) == 0) s[u >> 3] = sc;
         }
+        cur = nxt;
     }
 }
 
@@ -298,85 +317,200 @@ quant_fp8_128x128_kernel(const __grid_constant__ CUtensorMap tmX, uint8_t* __res
 }
 
 // ----------------------------------------------------------------- NVFP4
-
-// Pass 1: per-matrix amax as a 15-bit magnitude pattern, atomicMax into
-// amax_bits[b] (zeroed by the launcher).  grid = (slices, matrices).
-__global__ void __launch_bounds__(kThreads, 3)
-tensor_amax_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, uint32_t* __restrict__ amax_bits) {
-    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
-    const int64_t b = blockIdx.y;
-    const uint4* xb = x + 2 * b * units_per_matrix;
-    uint32_t m = 0;
-    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units_per_matrix; base += stride) {
-        Unit v[kUnroll];
-#pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            int64_t u = base + i * kThreads + threadIdx.x;
-            if (u < units_per_matrix) v[i] = load_unit(xb, u);
-        }
-#pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            int64_t u = base + i * kThreads + threadIdx.x;
-            if (u < units_per_matrix) m = max(m, unit_absmax(v[i]));
-        }
-    }
-    m = group_max<32>(m);
-    if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax_bits + b, m);
-}
+//
+// One persistent kernel per call.  The per-tensor scale g needs the amax of
+// the whole matrix before any block of it can be encoded, so every matrix
+// is read twice: once for its amax ("A" tiles) and once to encode it ("B"
+// tiles).  Work items (tiles of 1024 units = 32 KB of input) are handed out
+// from a global counter in the order
+//   A(0), A(1), B(0), A(2), B(1), ..., A(n-1), B(n-2), B(n-1)
+// (each a run over all tiles of the matrix), so the encode of matrix b
+// starts one matrix of amax work after its own amax, and its second read is
+// mostly served by L2.  A B tile of matrix b waits (bounded) until all A
+// tiles of b have published their amax.  An item only waits on items with
+// smaller indices, and the smallest unfinished item is always being run by
+// some CTA (the next index is fetched only once the current item is done),
+// so the order cannot deadlock whatever the residency.
+//
+// Workspace (32-bit words, zeroed by the launcher): [0, 2) item counter
+// (64-bit), [4, 4 + batch) amax patterns, [4 + batch, 4 + 2 batch) number of
+// finished A tiles per matrix.
+constexpr int NV_TILE_UNITS = kThreads * kUnroll;
 
 // Per-tensor scale g = fp32(amax_T / 2688), 1 for an all-zero tensor.
 __device__ __forceinline__ float nvfp4_tensor_scale(uint32_t a) {
     return a == 0 ? 1.0f : __fdiv_rn(__uint_as_float(a << 16), 2688.0f);
 }
 
-// Pass 2: one lane per 16-element block.  grid = (slices, matrices).
-__global__ void __launch_bounds__(kThreads, 3)
-quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t units_per_matrix, const uint32_t* __restrict__ amax_bits,
-                   uint2* __restrict__ q, uint8_t* __restrict__ s, float* __restrict__ g_out) {
-    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
-    const int64_t b = blockIdx.y;
-    const uint4* xb = x + 2 * b * units_per_matrix;
-    uint2* qb = q + b * units_per_matrix;
-    uint8_t* sb = s + b * units_per_matrix;
-    const float g = nvfp4_tensor_scale(amax_bits[b]);
-    if (blockIdx.x == 0 && threadIdx.x == 0) g_out[b] = g;
-    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units_per_matrix; base += stride) {
-        Unit v[kUnroll];
-#pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            int64_t u = base + i * kThreads + threadIdx.x;
-            if (u < units_per_matrix) v[i] = load_unit(xb, u);
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait until *count >= target; false (and a device error) after ~4 s.
+__device__ bool wait_count(const uint32_t* count, uint32_t target, uint32_t* err) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (ld_acquire_u32(count) >= target) return true;
+        uint64_t now;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+        if (it == 0) t0 = now;
+        else if (now - t0 > 4000000000ull) {
+            raise_device_error(err, FPQ_ERR_DEVICE_TIMEOUT);
+            return false;
         }
+        __nanosleep(128);
+    }
+}
+
+// Bracket for quotients by s from an approximation r of 1/s with relative
+// error at most 2^-21: r (1 -+ 2^-20) still lands strictly outside
+// (1/s)(1 -+ 2^-21), which is what the bracket argument needs.
+__device__ __forceinline__ QuotientBracket bracket_from_reciprocal(float s, float r) {
+    return QuotientBracket{s, __fmul_rn(r, 1.0f - 0x1p-20f), __fmul_rn(r, 1.0f + 0x1p-20f)};
+}
+
+struct NvItem {
+    bool is_a;
+    int64_t b, t;
+};
+
+__device__ __forceinline__ NvItem nv_decode(unsigned long long item, int64_t batch, int64_t nT) {
+    NvItem r;
+    const int64_t i = (int64_t)item;
+    if (i < nT) {
+        r.is_a = true; r.b = 0; r.t = i;
+        return r;
+    }
+    const int64_t j = i - nT, blk = j / nT;
+    r.t = j - blk * nT;
+    if (blk == 2 * (batch - 1)) { r.is_a = false; r.b = batch - 1; }
+    else if ((blk & 1) == 0) { r.is_a = true; r.b = blk / 2 + 1; }
+    else { r.is_a = false; r.b = (blk - 1) / 2; }
+    return r;
+}
+
+// Within an item each thread encodes its units one at a time, loading the
+// next before encoding the current; few registers let NV_MIN_BLOCKS CTAs
+// share an SM.
+constexpr int NV_MIN_BLOCKS = 4;
+
+__device__ __forceinline__ void nvfp4_encode_unit(const Unit& v, float g, bool g_ok, const QuotientBracket& gb,
+                                                  float rg, const ScaleTables& tab6, const float* s_dec,
+                                                  const float* s_inv, uint2* qdst, uint8_t* sdst) {
+    // block scale code = E4M3(fp32(fp32(amax_b / 6) / g)), S = fp32(dec(code) g)
+    const uint32_t a = unit_absmax(v);
+    float tq, unused_lo, unused_hi;
+    if (!table_scale(tab6, a, 4, tq, unused_lo, unused_hi)) tq = __fdiv_rn(__uint_as_float(a << 16), 6.0f);
+    uint32_t code;
+    if (g_ok) {
+        code = f32x2_to_e4m3x2(__fmul_rn(tq, gb.lo), __fmul_rn(tq, gb.hi));
+        code = ((code & 0xFFu) == (code >> 8)) ? (code & 0xFFu) : (f32x2_to_e4m3x2(__fdiv_rn(tq, g), 0.0f) & 0xFFu);
+    } else {
+        code = f32x2_to_e4m3x2(__fdiv_rn(tq, g), 0.0f) & 0xFFu;
+    }
+    const float S = code < 127u ? __fmul_rn(s_dec[code], g) : __fmul_rn(e4m3_to_f32(code), g);
+    uint32_t packed[2] = {0u, 0u};
+    if (S != 0.0f) {
+        if (g_ok && reciprocal_ok(S) && code < 127u) {
+            // fp32(inv(code) * fp32(1/g)) is within 2^-22 of 1/S, close
+            // enough for the bracket (bracket_from_reciprocal)
+            const QuotientBracket br = bracket_from_reciprocal(S, __fmul_rn(s_inv[code], rg));
 #pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            int64_t u = base + i * kThreads + threadIdx.x;
-            if (u >= units_per_matrix) continue;
-            const uint32_t a = unit_absmax(v[i]);
-            const float t = __fdiv_rn(__uint_as_float(a << 16), 6.0f);
-            const uint32_t code = f32x2_to_e4m3x2(__fdiv_rn(t, g), 0.0f) & 0xFFu;
-            const float S = e4m3_to_f32(code) * g;
-            uint32_t packed[2] = {0u, 0u};
-            if (S != 0.0f) {
-                if (reciprocal_ok(S)) {
-                    const QuotientBracket br = quotient_bracket(S);
+            for (int j = 0; j < 8; ++j)
+                packed[j >> 2] |= e2m1x2_of_quotients(bf16_lo(v.w[j]), bf16_hi(v.w[j]), br) << (8 * (j & 3));
+        } else {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        packed[j >> 2] |= e2m1x2_of_quotients(bf16_lo(v[i].w[j]), bf16_hi(v[i].w[j]), br)
-                                          << (8 * (j & 3));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(bf16_lo(v[i].w[j]), S),
-                                                        __fdiv_rn(bf16_hi(v[i].w[j]), S));
-                        packed[j >> 2] |= byte << (8 * (j & 3));
-                    }
-                }
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(bf16_lo(v.w[j]), S), __fdiv_rn(bf16_hi(v.w[j]), S));
+                packed[j >> 2] |= byte << (8 * (j & 3));
             }
-            st_v2(qb + u, make_uint2(packed[0], packed[1]));
-            sb[u] = (uint8_t)code;
         }
+    }
+    st_v2(qdst, make_uint2(packed[0], packed[1]));
+    *sdst = (uint8_t)code;
+}
+
+__global__ void __launch_bounds__(kThreads, NV_MIN_BLOCKS)
+quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint2* __restrict__ q,
+                   uint8_t* __restrict__ s, float* __restrict__ g_out, uint32_t* __restrict__ ws,
+                   uint32_t* err) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
+    __shared__ ScaleTables tab6;                 // fp32(amax_b / 6) by mantissa
+    __shared__ float s_dec[128];                 // dec(c) for E4M3 codes c = 0..126
+    __shared__ float s_inv[128];                 // fp32(1 / dec(c)) for c = 1..126
+    __shared__ uint32_t s_wmax[kThreads / 32];
+    __shared__ unsigned long long s_item;
+    __shared__ int s_ok;
+    unsigned long long* counter = reinterpret_cast<unsigned long long*>(ws);
+    uint32_t* amax = ws + 4;
+    uint32_t* done = ws + 4 + batch;
+    const int64_t nT = (upm + NV_TILE_UNITS - 1) / NV_TILE_UNITS;
+    const unsigned long long total = (unsigned long long)(2 * batch * nT);
+    init_scale_tables(tab6, 6.0f);
+    if (threadIdx.x < 128) {
+        const uint32_t c = threadIdx.x;
+        const float d = c == 127 ? 0.0f : e4m3_to_f32(c);
+        s_dec[c] = d;
+        s_inv[c] = (c == 0 || c == 127) ? 0.0f : __frcp_rn(d);
+    }
+    if (threadIdx.x == 0) s_item = atomicAdd(counter, 1ull);
+    __syncthreads();
+    unsigned long long item = s_item;
+    while (item < total) {
+        const NvItem w = nv_decode(item, batch, nT);
+        const uint4* xb = x + 2 * w.b * upm;
+        const int64_t u0 = w.t * NV_TILE_UNITS + threadIdx.x;
+        if (w.is_a) {
+            uint32_t m = 0;
+            Unit cur;
+            if (u0 < upm) cur = load_unit(xb, u0);
+#pragma unroll
+            for (int i = 0; i < kUnroll; ++i) {
+                const int64_t u = u0 + i * kThreads;
+                Unit nxt;
+                if (i + 1 < kUnroll && u + kThreads < upm) nxt = load_unit(xb, u + kThreads);
+                if (u < upm) m = max(m, unit_absmax(cur));
+                cur = nxt;
+            }
+            m = group_max<32>(m);
+            if ((threadIdx.x & 31) == 0) s_wmax[threadIdx.x >> 5] = m;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                uint32_t mm = 0;
+#pragma unroll
+                for (int k = 0; k < kThreads / 32; ++k) mm = max(mm, s_wmax[k]);
+                if (mm) atomicMax(amax + w.b, mm);
+                __threadfence();                     // publish the amax before the count
+                atomicAdd(done + w.b, 1u);
+            }
+        } else {
+            Unit cur;
+            if (u0 < upm) cur = load_unit(xb, u0);  // the input is ready; only g must wait
+            if (threadIdx.x == 0) s_ok = wait_count(done + w.b, (uint32_t)nT, err) ? 1 : 0;
+            __syncthreads();
+            if (!s_ok) return;
+            const float g = nvfp4_tensor_scale(__ldcg(amax + w.b));
+            if (w.t == 0 && threadIdx.x == 0) g_out[w.b] = g;
+            const bool g_ok = reciprocal_ok(g);
+            const QuotientBracket gb = quotient_bracket(g_ok ? g : 1.0f);
+            const float rg = __frcp_rn(g_ok ? g : 1.0f);
+            uint2* qb = q + w.b * upm;
+            uint8_t* sb = s + w.b * upm;
+#pragma unroll 1
+            for (int i = 0; i < kUnroll; ++i) {
+                const int64_t u = u0 + i * kThreads;
+                Unit nxt;
+                if (i + 1 < kUnroll && u + kThreads < upm) nxt = load_unit(xb, u + kThreads);
+                if (u < upm) nvfp4_encode_unit(cur, g, g_ok, gb, rg, tab6, s_dec, s_inv, qb + u, sb + u);
+                cur = nxt;
+            }
+        }
+        __syncthreads();                             // every thread is done with s_item / s_ok
+        if (threadIdx.x == 0) s_item = atomicAdd(counter, 1ull);
+        __syncthreads();
+        item = s_item;
     }
 }
 
@@ -466,7 +600,8 @@ cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows,
             (const uint4*)x, (uint4*)q, (uint8_t*)scales, units);
         break;
     case FPQ_FP8_1x128:
-        quant_fp8_1x128_kernel<<<grid_for(units, kThreads * kUnroll, sms), kThreads, 0, st>>>(
+        quant_fp8_1x128_kernel<<<(int)max64(1, min64((units + kThreads - 1) / kThreads, (int64_t)sms * Q1_MIN_BLOCKS)),
+                                 kThreads, 0, st>>>(
             (const uint4*)x, (uint4*)q, (float*)scales, units);
         break;
     case FPQ_FP8_128x128: {
@@ -484,23 +619,13 @@ cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows,
     }
     case FPQ_NVFP4: {
         const int64_t upm = rows * cols / 16;
-        uint32_t* amax = (uint32_t*)workspace;
-        cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t) * batch, st);
+        uint32_t* ws = (uint32_t*)workspace;
+        cudaError_t e = cudaMemsetAsync(ws, 0, nvfp4_workspace_words(batch) * sizeof(uint32_t), st);
         if (e != cudaSuccess) return e;
-        // Matrices are processed in chunks small enough that the amax pass
-        // leaves the chunk resident in L2 for the quantize pass.
-        const int64_t chunk_bytes = 64ll << 20;
-        int64_t per_chunk = max64(1, chunk_bytes / max64(1, rows * cols * 2));
-        for (int64_t b0 = 0; b0 < batch; b0 += per_chunk) {
-            int64_t nb = min(per_chunk, batch - b0);
-            int slices = (int)max64(1, min64((sms * 8 + nb - 1) / nb,
-                                                           (upm + kThreads * kUnroll - 1) / (kThreads * kUnroll)));
-            dim3 grid((unsigned)slices, (unsigned)nb);
-            tensor_amax_kernel<<<grid, kThreads, 0, st>>>((const uint4*)x + 2 * b0 * upm, upm, amax + b0);
-            quant_nvfp4_kernel<<<grid, kThreads, 0, st>>>((const uint4*)x + 2 * b0 * upm, upm, amax + b0,
-                                                          (uint2*)q + b0 * upm, (uint8_t*)scales + b0 * upm,
-                                                          tensor_scale + b0);
-        }
+        const int64_t items = 2 * batch * ((upm + NV_TILE_UNITS - 1) / NV_TILE_UNITS);
+        const int grid = (int)max64(1, min64(items, (int64_t)sms * NV_MIN_BLOCKS));
+        quant_nvfp4_kernel<<<grid, kThreads, 0, st>>>((const uint4*)x, batch, upm, (uint2*)q, (uint8_t*)scales,
+                                                      tensor_scale, ws, err);
         break;
     }
     default:

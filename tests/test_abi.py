@@ -89,3 +89,17 @@ def test_status_strings(lib):
         assert L.fpq_status_string(code)
     L.fpq_version.restype = ctypes.c_int32
     assert L.fpq_version() >= 10000
+
+
+def test_nvfp4_workspace_size(lib):
+    """NVFP4 needs a 64-bit work counter (16 bytes with padding) plus an amax
+    word and a progress counter per matrix; the other formats need none."""
+    L, _ = lib
+    import mxfp8_block_scaled_warp_b200 as f
+    L.fpq_quantize_workspace_bytes.restype = ctypes.c_size_t
+    L.fpq_quantize_workspace_bytes.argtypes = [ctypes.c_int32, ctypes.c_int64]
+    for b in (1, 2, 64, 4096):
+        assert L.fpq_quantize_workspace_bytes(f.NVFP4, b) == 16 + 8 * b
+    assert L.fpq_quantize_workspace_bytes(f.NVFP4, 0) == 0
+    for fmt in (f.MXFP8, f.FP8_1x128, f.FP8_128x128):
+        assert L.fpq_quantize_workspace_bytes(fmt, 8) == 0
