@@ -169,6 +169,44 @@ def test_ds_fp8_full_size(fpq, orc):
     assert_same(host(sb), f32_bits(osb), "B scales")
 
 
+def amax_sweep_blocks(exponents, block: int, seed: int) -> np.ndarray:
+    """One block per (exponent field, mantissa field) pair: the block's
+    largest magnitude is exactly that bf16 pattern (random sign), the other
+    elements random patterns of no larger magnitude.  The quantizers derive
+    a block scale from the amax through a per-mantissa table whenever the
+    result is a normal fp32 number and by IEEE division otherwise, so the
+    sweep covers every table entry on both sides of that boundary."""
+    rng = np.random.default_rng(seed)
+    pats = [(e << 7) | m for e in exponents for m in range(128)]
+    out = np.empty((len(pats), block), np.uint16)
+    for i, p in enumerate(pats):
+        mags = rng.integers(0, p + 1, block)
+        mags[rng.integers(0, block)] = p
+        out[i] = (mags | (rng.integers(0, 2, block) << 15)).astype(np.uint16)
+    return out
+
+
+def test_fp8_1x128_every_amax_mantissa(fpq, orc):
+    # amax / 448 is a normal fp32 number from exponent field 10 upwards
+    x = amax_sweep_blocks(list(range(1, 14)) + list(range(120, 136)) + list(range(245, 255)), 128, 40)
+    q, s = fpq.quantize(dev(x), fpq.FP8_1x128)
+    oq, os_ = orc.quant_fp8_1x128(x)
+    assert_same(host(q), oq, "codes")
+    assert_same(host(s), f32_bits(os_), "fp32 scales")
+
+
+def test_nvfp4_every_amax_mantissa(fpq, orc):
+    # amax_b / 6 is a normal fp32 number from exponent field 4 upwards; one
+    # matrix per exponent range, so that each has its own tensor scale
+    groups = [range(2, 13), range(20, 31), range(100, 111), range(244, 255)]
+    x = np.stack([amax_sweep_blocks(list(g), 16, 41 + i).reshape(88, 256) for i, g in enumerate(groups)])
+    q, s, g = fpq.quantize(dev(x), fpq.NVFP4)
+    oq, os_, og = orc.quant_nvfp4(x)
+    assert_same(host(g), f32_bits(og), "tensor scales")
+    assert_same(host(s), os_, "E4M3 block scales")
+    assert_same(host(q), oq, "packed E2M1 codes")
+
+
 # ------------------------------------------------------------------ NVFP4
 
 NV_CASES = {
