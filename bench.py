@@ -339,6 +339,36 @@ def run_reference(args, rank, world):
     print(json.dumps(line))
 
 
+# ------------------------------------------------------------------ replicas
+
+def init_replicas(world: int, backend: str = "nccl", device=None):
+    """One process per GPU, no data-path collective: the process group only
+    carries the barriers around the timed region and the max over ranks.
+    Returns the torch.distributed module, or None for a single process."""
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    from datetime import timedelta
+    kw = {"device_id": device} if backend == "nccl" and device is not None else {}
+    dist.init_process_group(backend, timeout=timedelta(seconds=120), **kw)
+    return dist
+
+
+def max_over_ranks(value: float, pg, device=None) -> float:
+    """The slowest rank's time (every rank takes this collective in step)."""
+    if pg is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, steps: int, total_ms: float) -> float:
+    """Weak scaling: every rank runs the same step on its own data, so the
+    job's throughput is all ranks' work over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (total_ms * 1e-3) / 1e12
+
+
 METRIC = "quantize GB/s vs HBM peak; block-scaled FP8 GEMM TFLOPS vs FP8 tensor peak"
 
 
@@ -363,12 +393,7 @@ def main():
     import mxfp8_block_scaled_warp_b200 as fpq
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import torch.distributed as dist
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-        pg = dist
+    pg = init_replicas(world, "nccl", dev)
 
     step = STEPS[args.workload](fpq, dev)
     stream = torch.cuda.current_stream()
@@ -429,13 +454,9 @@ def main():
     if status != 0:
         raise SystemExit(f"device error word {status} after the timed steps")
     del graph
-    total_ms = sum(step_ms)
-    if pg:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), pg, dev)
     ms_per_step = total_ms / args.steps
-    value = world * step.flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, step.flops, args.steps, total_ms)
 
     peaks = _peaks()
     fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
@@ -467,12 +488,8 @@ def main():
             hb, db = step.e2e_step(stream)
         e1.record(stream)
         e1.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / reps
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * step.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": hb,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / reps, pg, dev)
+        e2e = {"value": whole_job_tflops(world, step.flops, 1, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": hb,
                "d2h_bytes_per_step": db, "ms_per_step": e2e_ms}
 
     cpu = None
