@@ -415,22 +415,39 @@ def main():
     torch.cuda.synchronize()
     assert fpq.fpq_get_device_error() == 0
 
-    # The step is captured once as a CUDA graph (its launches and the event
-    # records between them) and replayed, so that host-side launch work never
-    # leaves the GPU idle inside the timed kernels.  The L2 flush runs outside
-    # the graph before every replay; each replay's events are read before the
-    # next one overwrites them.
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in kern]
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    cap.wait_stream(stream)
-    with torch.cuda.stream(cap):
-        with torch.cuda.graph(graph, stream=cap):
-            one_step(ev)
-    stream.wait_stream(cap)
+    # The step is captured as CUDA graphs and replayed, so that host-side
+    # launch work never leaves the GPU idle inside the timed region.  Two
+    # graphs of the same launches: `whole` records events only before the
+    # first and after the last kernel, so consecutive kernels keep their
+    # programmatic-dependent-launch overlap (the step time and the headline
+    # value come from it); `split` records events around every kernel (the
+    # per-kernel times and the roofline come from it).  The L2 flush runs
+    # outside the graphs before every replay; each replay's events are read
+    # before the next replay overwrites them.
+    def capture(events_per_kernel):
+        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+              for _ in (kern if events_per_kernel else [None])]
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap):
+                if events_per_kernel:
+                    one_step(ev)
+                else:
+                    ev[0][0].record()
+                    one_step()
+                    ev[0][1].record()
+        stream.wait_stream(cap)
+        return g, ev
+
+    whole, ev_whole = capture(False)
+    split, ev_split = capture(True)
     for _ in range(args.warmup):
         flush.zero_()
-        graph.replay()
+        whole.replay()
+        flush.zero_()
+        split.replay()
     torch.cuda.synchronize()
     assert fpq.fpq_get_device_error() == 0
 
@@ -442,18 +459,23 @@ def main():
     with ClockSampler(local) as clk:
         for s in range(args.steps):
             flush.zero_()
-            graph.replay()
-            ev[-1][1].synchronize()
-            for i, n in enumerate(names):
-                per_kernel[n].append(ev[i][0].elapsed_time(ev[i][1]))
-            step_ms.append(ev[0][0].elapsed_time(ev[-1][1]))
+            whole.replay()
+            ev_whole[0][1].synchronize()
+            step_ms.append(ev_whole[0][0].elapsed_time(ev_whole[0][1]))
         torch.cuda.synchronize()
     if pg:
         pg.barrier()
+    for s in range(args.steps):
+        flush.zero_()
+        split.replay()
+        ev_split[-1][1].synchronize()
+        for i, n in enumerate(names):
+            per_kernel[n].append(ev_split[i][0].elapsed_time(ev_split[i][1]))
+    torch.cuda.synchronize()
     status = fpq.fpq_get_device_error()
     if status != 0:
         raise SystemExit(f"device error word {status} after the timed steps")
-    del graph
+    del whole, split
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(world, step.flops, args.steps, total_ms)
@@ -499,7 +521,7 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3xe4m3->f32 (bf16 in/out)", "data": "synthetic",
-            "config": dict(step.config, launch="one CUDA graph per step (kernels + event records), replayed"), "quantize_gbs": quant_gbs, "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"],
+            "config": dict(step.config, launch="CUDA graph of the step replayed per timed step; per-kernel times from a second graph with events around each kernel"), "quantize_gbs": quant_gbs, "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"],
             "kernels": kernels_out, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.launches * args.steps, "clocks": clk.summary(),
             "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp8_tflops": fp8_peak_burst, "source": peaks["source"]}}
