@@ -108,6 +108,13 @@ class Step:
     quant_bytes = 0.0
     launches = 0
     dominant = ""
+    unit = "TFLOP/s"           # the rate `value` is reported in: flops (GEMM steps) or bytes
+    dtype = "e4m3xe4m3->f32 (bf16 in/out)"
+
+    @property
+    def work(self) -> float:
+        """Work of one step in the unit's numerator (flops, or bytes for GB/s)."""
+        return self.flops
 
     def kernels(self):  # list of (label, callable)
         raise NotImplementedError
@@ -244,7 +251,91 @@ class QatForward(Step):
                 "gemm_fp8_f32scale": ("TFLOP/s", self.flops)}
 
 
-STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": QatForward}
+
+
+class MoePrequant(Step):
+    """MoE expert prequantization: 64 experts x {gate, up [2048, 7168]; down
+    [7168, 2048]} bf16 N(0, 0.02), each projection's 64 matrices quantized by
+    one batched call, to MXFP8 (1x32, E8M0) and to NVFP4 (1x16 E4M3 + a
+    per-matrix fp32 scale).  The step's work is the algorithmic bytes."""
+    name = "moe_prequant"
+    dominant = "quant_nvfp4"
+    unit = "GB/s"
+    dtype = "bf16 -> e4m3 / e2m1 codes (fp32 scale arithmetic)"
+
+    def __init__(self, fpq, dev, experts=64):
+        self.f = fpq
+        self.e = experts
+        shapes = {"gate": (2048, 7168), "up": (2048, 7168), "down": (7168, 2048)}
+        self.x, self.mx, self.nv, self.host = {}, {}, {}, {}
+        for i, (nm, (r, c)) in enumerate(shapes.items()):
+            g = torch.Generator(device=dev)
+            g.manual_seed(4000 + i)
+            x = torch.empty((experts, r, c), dtype=torch.bfloat16, device=dev)
+            for e in range(experts):
+                x[e] = (torch.randn(r, c, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+            self.x[nm] = (x, r, c)
+            self.mx[nm] = (torch.empty((experts, r, c), dtype=torch.uint8, device=dev),
+                           torch.empty((experts, r, c // 32), dtype=torch.uint8, device=dev))
+            wsb = fpq.fpq_quantize_workspace_bytes(fpq.NVFP4, experts)
+            self.nv[nm] = (torch.empty((experts, r, c // 2), dtype=torch.uint8, device=dev),
+                           torch.empty((experts, r, c // 16), dtype=torch.uint8, device=dev),
+                           torch.empty((experts,), dtype=torch.float32, device=dev),
+                           torch.empty(((wsb + 15) // 16 * 16,), dtype=torch.uint8, device=dev))
+        elems = sum(experts * r * c for _, r, c in self.x.values())
+        self.mx_bytes = elems * (2 + 1 + 1 / 32)
+        self.nv_bytes = elems * (2 + 0.5 + 1 / 16) + 4 * 3 * experts
+        self.quant_bytes = self.mx_bytes + self.nv_bytes
+        self.launches = 6
+        self.config = {"workload": "moe_prequant: 64 experts x {gate, up 2048x7168; down 7168x2048} bf16 N(0,0.02) "
+                                   "-> MXFP8 (1x32 E8M0) and NVFP4 (1x16 E4M3 + fp32 per matrix); one batched call "
+                                   "per projection and format",
+                       "elements": elems, "l2": "flushed before every step (256 MiB write)"}
+
+    @property
+    def work(self) -> float:
+        return self.quant_bytes
+
+    def kernels(self):
+        f = self.f
+
+        def mx():
+            for nm, (x, r, c) in self.x.items():
+                q, s_ = self.mx[nm]
+                f.fpq_quantize_block(f.MXFP8, x, self.e, r, c, q, s_)
+
+        def nv():
+            for nm, (x, r, c) in self.x.items():
+                q, s_, g, ws = self.nv[nm]
+                f.fpq_quantize_block(f.NVFP4, x, self.e, r, c, q, s_, g, ws)
+
+        return [("quant_mxfp8", mx), ("quant_nvfp4", nv)]
+
+    def kernel_work(self):
+        return {"quant_mxfp8": ("GB/s", self.mx_bytes), "quant_nvfp4": ("GB/s", self.nv_bytes)}
+
+    def e2e_step(self, stream):
+        """bf16 expert stacks in pinned host memory in, every code and scale
+        back to pinned host memory, copies inside the timed region."""
+        if not self.host:
+            for nm, (x, r, c) in self.x.items():
+                outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (*self.mx[nm], *self.nv[nm][:3])]
+                self.host[nm] = (x.cpu().pin_memory(), outs)
+        hb = db = 0
+        for nm, (x, r, c) in self.x.items():
+            x.copy_(self.host[nm][0], non_blocking=True)
+            hb += x.numel() * 2
+        for _, fn in self.kernels():
+            fn()
+        for nm in self.x:
+            for h, d in zip(self.host[nm][1], (*self.mx[nm], *self.nv[nm][:3])):
+                h.copy_(d, non_blocking=True)
+                db += d.numel() * d.element_size()
+        return hb, db
+
+
+STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": QatForward,
+         "moe_prequant": MoePrequant}
 
 
 # ------------------------------------------------------------------ traffic from committed ncu summaries
@@ -281,6 +372,8 @@ def cpu_baseline(workload: str, budget_s: float = 12.0):
     the workload and extrapolate to the whole step in TFLOP/s."""
     import oracle
     oracle.build()
+    if workload == "moe_prequant":
+        return _cpu_baseline_prequant(oracle, budget_s)
     if workload != "ds_fp8_gemm":
         return None
     m, n, k = 4096, 2048, 7168
@@ -308,10 +401,37 @@ def cpu_baseline(workload: str, budget_s: float = 12.0):
     oracle.gemm_entries(0, qa, sa, 1, qb, sb, rr, cc)
     per = (time.perf_counter() - t0) / count
     step_s = t_qa * m * k + t_qb * n * k + per * m * n
-    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "work": 2.0 * m * n * k, "cores": 1,
+            "kind": "oracle",
             "sample": f"1x128 quantize of {rows_a} rows and 128x128 quantize of 256 rows of the 7168-wide "
                       f"operands, {count} fp64 GEMM entries (K=7168); extrapolated to the full 4096x2048x7168 "
                       f"step ({step_s:.1f} s per step on one core)"}
+
+
+def _cpu_baseline_prequant(oracle, budget_s: float):
+    """The oracle's MXFP8 and NVFP4 quantizers on leading rows of one
+    2048x7168 expert matrix (rows sized to the budget), extrapolated to the
+    whole 64-expert step at their per-byte rates."""
+    k = 7168
+    x = workloads.as_u16(workloads.normal_bf16((2048, k), 0.02, 4000))
+    rates = {}
+    for fmt, bpe in (("mxfp8", 3 + 1 / 32), ("nvfp4", 2.5 + 1 / 16)):
+        fn = oracle.quant_mxfp8 if fmt == "mxfp8" else oracle.quant_nvfp4
+        rows = 16
+        t0 = time.perf_counter()
+        fn(x[:rows])
+        per_row = (time.perf_counter() - t0) / rows
+        rows = int(max(16, min(2048, budget_s / 2 / max(per_row, 1e-9))))
+        t0 = time.perf_counter()
+        fn(x[:rows])
+        rates[fmt] = (rows * k * bpe, time.perf_counter() - t0, rows, bpe)
+    elems = 64 * 3 * 2048 * 7168
+    work = sum(elems * bpe for (_, _, _, bpe) in rates.values())
+    step_s = sum(elems * bpe * t / b for (b, t, _, bpe) in rates.values())
+    return {"value": work / step_s / 1e9, "unit": "GB/s", "work": work, "cores": 1, "kind": "oracle",
+            "sample": f"MXFP8 quantize of {rates['mxfp8'][2]} rows and NVFP4 quantize of {rates['nvfp4'][2]} rows "
+                      f"of one 2048x7168 expert matrix; extrapolated to the 64-expert step ({step_s:.1f} s per step "
+                      f"on one core)"}
 
 
 # ------------------------------------------------------------------ main
@@ -320,8 +440,11 @@ def run_reference(args, rank, world):
     """The reference arm: the CPU oracle timed as it stands."""
     if rank != 0:
         return
+    if cpu_baseline(args.workload, budget_s=1.0) is None:
+        print(json.dumps({"impl": "reference", "unavailable": f"no oracle timing defined for {args.workload}"}))
+        return
     vals = []
-    for _ in range(args.warmup):
+    for _ in range(args.warmup - 1):
         cpu_baseline(args.workload, budget_s=1.0)
     t_total = 0.0
     for _ in range(args.steps):
@@ -330,12 +453,14 @@ def run_reference(args, rank, world):
         t_total += time.perf_counter() - t0
         vals.append(r["value"])
     v = statistics.median(vals)
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 2.0 * 4096 * 2048 * 7168 / (v * 1e12) * 1e3,
+    unit, work = r["unit"], r["work"]
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": work / (v * scale) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": args.workload},
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": r["sample"]},
-            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle", "sample": r["sample"]},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
 
@@ -367,6 +492,12 @@ def whole_job_tflops(world: int, flops_per_rank_step: float, steps: int, total_m
     """Weak scaling: every rank runs the same step on its own data, so the
     job's throughput is all ranks' work over the slowest rank's time."""
     return world * flops_per_rank_step * steps / (total_ms * 1e-3) / 1e12
+
+
+def whole_job_rate(world: int, work_per_rank_step: float, steps: int, total_ms: float, unit: str) -> float:
+    """whole_job_tflops for either unit: TFLOP/s (flops) or GB/s (bytes)."""
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    return world * work_per_rank_step * steps / (total_ms * 1e-3) / scale
 
 
 METRIC = "quantize GB/s vs HBM peak; block-scaled FP8 GEMM TFLOPS vs FP8 tensor peak"
@@ -478,7 +609,7 @@ def main():
     del whole, split
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
     ms_per_step = total_ms / args.steps
-    value = whole_job_tflops(world, step.flops, args.steps, total_ms)
+    value = whole_job_rate(world, step.work, args.steps, total_ms, step.unit)
 
     peaks = _peaks()
     fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
@@ -491,9 +622,14 @@ def main():
         kernels_out[n] = {"ms": ms, "achieved": ach, "unit": unit, "frac_of_peak": ach / pk}
     dom = kernels_out[step.dominant]
     traffic = _traffic(step.dominant, step.name)
-    roofline = {"kernel": step.dominant, "bound": "tensor", "achieved": dom["achieved"], "peak": fp8_peak_burst,
-                "unit": "TFLOP/s", "frac": dom["achieved"] / fp8_peak_burst, "traffic": traffic,
-                "peak_note": f"fp8 = 2 x {peaks['source']} cuBLAS bf16 burst ({peaks['bf16_tflops']} TFLOP/s)"}
+    if dom["unit"] == "GB/s":
+        roofline = {"kernel": step.dominant, "bound": "hbm", "achieved": dom["achieved"], "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": dom["achieved"] / peaks["hbm_gbs"], "traffic": traffic,
+                    "peak_note": f"{peaks['source']} HBM copy bandwidth"}
+    else:
+        roofline = {"kernel": step.dominant, "bound": "tensor", "achieved": dom["achieved"], "peak": fp8_peak_burst,
+                    "unit": "TFLOP/s", "frac": dom["achieved"] / fp8_peak_burst, "traffic": traffic,
+                    "peak_note": f"fp8 = 2 x {peaks['source']} cuBLAS bf16 burst ({peaks['bf16_tflops']} TFLOP/s)"}
     quant_ms = sum(statistics.mean(per_kernel[n]) for n in names if not n.startswith("gemm"))
     quant_gbs = step.quant_bytes / (quant_ms * 1e-3) / 1e9
 
@@ -511,16 +647,16 @@ def main():
         e1.record(stream)
         e1.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / reps, pg, dev)
-        e2e = {"value": whole_job_tflops(world, step.flops, 1, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": hb,
+        e2e = {"value": whole_job_rate(world, step.work, 1, e2e_ms, step.unit), "unit": step.unit, "h2d_bytes_per_step": hb,
                "d2h_bytes_per_step": db, "ms_per_step": e2e_ms}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(step.name)
 
-    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+    line = {"metric": METRIC, "value": value, "unit": step.unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3xe4m3->f32 (bf16 in/out)", "data": "synthetic",
+            "vs_baseline": None, "dtype": step.dtype, "data": "synthetic",
             "config": dict(step.config, launch="CUDA graph of the step replayed per timed step; per-kernel times from a second graph with events around each kernel"), "quantize_gbs": quant_gbs, "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"],
             "kernels": kernels_out, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.launches * args.steps, "clocks": clk.summary(),
