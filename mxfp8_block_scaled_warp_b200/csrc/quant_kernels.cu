@@ -321,7 +321,7 @@ quant_fp8_128x128_kernel(const __grid_constant__ CUtensorMap tmX, uint8_t* __res
 // One persistent kernel per call.  The per-tensor scale g needs the amax of
 // the whole matrix before any block of it can be encoded, so every matrix
 // is read twice: once for its amax ("A" tiles) and once to encode it ("B"
-// tiles).  Work items (tiles of 1024 units = 32 KB of input) are handed out
+// tiles).  Work items (tiles of 4096 units = 128 KB of input) are handed out
 // from a global counter in the order
 //   A(0), A(1), B(0), A(2), B(1), ..., A(n-1), B(n-2), B(n-1)
 // (each a run over all tiles of the matrix), so the encode of matrix b
@@ -335,7 +335,8 @@ quant_fp8_128x128_kernel(const __grid_constant__ CUtensorMap tmX, uint8_t* __res
 // Workspace (32-bit words, zeroed by the launcher): [0, 2) item counter
 // (64-bit), [4, 4 + batch) amax patterns, [4 + batch, 4 + 2 batch) number of
 // finished A tiles per matrix.
-constexpr int NV_TILE_UNITS = kThreads * kUnroll;
+constexpr int NV_UNITS_PER_THREAD = 16;        // units of one item per thread
+constexpr int NV_TILE_UNITS = kThreads * NV_UNITS_PER_THREAD;
 
 // Per-tensor scale g = fp32(amax_T / 2688), 1 for an all-zero tensor.
 __device__ __forceinline__ float nvfp4_tensor_scale(uint32_t a) {
@@ -394,7 +395,7 @@ __device__ __forceinline__ NvItem nv_decode(unsigned long long item, int64_t bat
 // Within an item each thread encodes its units one at a time, loading the
 // next before encoding the current; few registers let NV_MIN_BLOCKS CTAs
 // share an SM.
-constexpr int NV_MIN_BLOCKS = 4;
+constexpr int NV_MIN_BLOCKS = 5;
 
 __device__ __forceinline__ void nvfp4_encode_unit(const Unit& v, float g, bool g_ok, const QuotientBracket& gb,
                                                   float rg, const ScaleTables& tab6, const float* s_dec,
@@ -460,18 +461,22 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
     unsigned long long item = s_item;
     while (item < total) {
         const NvItem w = nv_decode(item, batch, nT);
-        const uint4* xb = x + 2 * w.b * upm;
-        const int64_t u0 = w.t * NV_TILE_UNITS + threadIdx.x;
+        // this item's units: [base, base + n) of matrix w.b, addressed by
+        // 32-bit offsets from the item's first unit
+        const int64_t base = w.b * upm + w.t * NV_TILE_UNITS;
+        const int n = (int)min64(NV_TILE_UNITS, upm - w.t * NV_TILE_UNITS);
+        const uint4* xi = x + 2 * base;
+        const int u0 = threadIdx.x;
         if (w.is_a) {
             uint32_t m = 0;
             Unit cur;
-            if (u0 < upm) cur = load_unit(xb, u0);
+            if (u0 < n) cur = load_unit(xi, u0);
 #pragma unroll
-            for (int i = 0; i < kUnroll; ++i) {
-                const int64_t u = u0 + i * kThreads;
+            for (int i = 0; i < NV_UNITS_PER_THREAD; ++i) {
+                const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < kUnroll && u + kThreads < upm) nxt = load_unit(xb, u + kThreads);
-                if (u < upm) m = max(m, unit_absmax(cur));
+                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit(xi, u + kThreads);
+                if (u < n) m = max(m, unit_absmax(cur));
                 cur = nxt;
             }
             m = group_max<32>(m);
@@ -487,7 +492,7 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
             }
         } else {
             Unit cur;
-            if (u0 < upm) cur = load_unit(xb, u0);  // the input is ready; only g must wait
+            if (u0 < n) cur = load_unit(xi, u0);    // the input is ready; only g must wait
             if (threadIdx.x == 0) s_ok = wait_count(done + w.b, (uint32_t)nT, err) ? 1 : 0;
             __syncthreads();
             if (!s_ok) return;
@@ -496,14 +501,14 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
             const bool g_ok = reciprocal_ok(g);
             const QuotientBracket gb = quotient_bracket(g_ok ? g : 1.0f);
             const float rg = __frcp_rn(g_ok ? g : 1.0f);
-            uint2* qb = q + w.b * upm;
-            uint8_t* sb = s + w.b * upm;
+            uint2* qi = q + base;
+            uint8_t* si = s + base;
 #pragma unroll 1
-            for (int i = 0; i < kUnroll; ++i) {
-                const int64_t u = u0 + i * kThreads;
+            for (int i = 0; i < NV_UNITS_PER_THREAD; ++i) {
+                const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < kUnroll && u + kThreads < upm) nxt = load_unit(xb, u + kThreads);
-                if (u < upm) nvfp4_encode_unit(cur, g, g_ok, gb, rg, tab6, s_dec, s_inv, qb + u, sb + u);
+                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit(xi, u + kThreads);
+                if (u < n) nvfp4_encode_unit(cur, g, g_ok, gb, rg, tab6, s_dec, s_inv, qi + u, si + u);
                 cur = nxt;
             }
         }
