@@ -211,6 +211,21 @@ class MoeGrouped(Step):
     def kernel_work(self):
         return {"quant_mxfp8": ("GB/s", self.qx_bytes), "gemm_grouped_mxfp8": ("TFLOP/s", self.flops)}
 
+    def e2e_step(self, stream):
+        """Permuted tokens and the group offsets from pinned host memory in,
+        the expert outputs back to pinned host memory, copies inside the
+        timed region (the expert weights stay resident: serving)."""
+        if not hasattr(self, "x_host"):
+            self.x_host = self.x.cpu().pin_memory()
+            self.off_host = self.offsets.cpu().pin_memory()
+            self.c_host = torch.empty(self.c.shape, dtype=self.c.dtype).pin_memory()
+        self.x.copy_(self.x_host, non_blocking=True)
+        self.offsets.copy_(self.off_host, non_blocking=True)
+        for _, fn in self.kernels():
+            fn()
+        self.c_host.copy_(self.c, non_blocking=True)
+        return self.x.numel() * 2 + self.offsets.numel() * 4, self.c.numel() * 2
+
 
 class QatForward(Step):
     name = "qat_forward"
@@ -250,7 +265,19 @@ class QatForward(Step):
         return {"lora_merge_fq": ("GB/s", self.merge_bytes), "quant_fp8_1x128": ("GB/s", self.xq_bytes),
                 "gemm_fp8_f32scale": ("TFLOP/s", self.flops)}
 
-
+    def e2e_step(self, stream):
+        """Base weight, LoRA factors and activations from pinned host memory
+        in, the GEMM output back to pinned host memory, copies inside the
+        timed region."""
+        if not hasattr(self, "host"):
+            self.host = [t.cpu().pin_memory() for t in (self.w, self.la, self.lb, self.x)]
+            self.c_host = torch.empty(self.c.shape, dtype=self.c.dtype).pin_memory()
+        for d, h in zip((self.w, self.la, self.lb, self.x), self.host):
+            d.copy_(h, non_blocking=True)
+        for _, fn in self.kernels():
+            fn()
+        self.c_host.copy_(self.c, non_blocking=True)
+        return sum(h.numel() * 2 for h in self.host), self.c.numel() * 2
 
 
 class MoePrequant(Step):

@@ -45,6 +45,8 @@ constexpr uint32_t SF_COLS_PER_STAGE = 16;  // 4 (A) + 8 (B), padded
 constexpr int NUM_THREADS = 256;
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
 
+constexpr int kMaxGroups = 1024;   // the C ABI rejects more groups
+
 struct __align__(1024) Smem {
     uint8_t a[STAGES][A_TILE];
     uint8_t b[STAGES][B_TILE];
@@ -58,6 +60,7 @@ struct __align__(1024) Smem {
     int32_t group;
     int32_t row_begin, row_end;   // A rows owned by this tile's group
     int32_t m_tile, n_tile;
+    int32_t off[kMaxGroups + 1];  // grouped: the group offsets, staged once per CTA
 };
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -112,51 +115,73 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int KT = (int)(K / BK);
     const int sf_pitch = (int)(K / 32);
 
-    if (threadIdx.x == 0) {
+    // Map this CTA to (group, m tile, n tile).  Grouped: all threads stage
+    // the offsets in shared memory with one coalesced read, then warp 0
+    // scans the groups 32 at a time (tile counts, inclusive prefix sum over
+    // the warp, ballot for the group holding tile blockIdx.x) and validates
+    // every group: offsets must rise from 0 to M.
+    if (offsets != nullptr) {
         pdl_wait();    // the group offsets may come from the preceding grid
-        // map this CTA to (group, m tile, n tile)
-        int valid = 0, g = 0, mt = 0, nt = 0;
-        int32_t rb = 0, re = (int32_t)M;
-        if (offsets == nullptr) {
-            const int t = blockIdx.x;
-            mt = t / n_tiles;
-            nt = t - mt * n_tiles;
-            valid = (int64_t)mt * BM < M;
-        } else {
-            bool ok = offsets[0] == 0 && offsets[groups] == (int32_t)M;
-            int t = blockIdx.x;
-            for (int e = 0; e < groups && ok; ++e) {
-                const int32_t b0 = offsets[e], b1 = offsets[e + 1];
-                if (b1 < b0) { ok = false; break; }
-                const int tiles_e = ((b1 - b0 + BM - 1) / BM) * n_tiles;
-                if (!valid && t < tiles_e) {
-                    valid = 1;
-                    g = e;
-                    mt = t / n_tiles;
-                    nt = t - mt * n_tiles;
-                    rb = b0;
-                    re = b1;
-                } else if (!valid) {
-                    t -= tiles_e;
-                }
-            }
-            if (!ok) {
-                if (blockIdx.x == 0) raise_device_error(err, FPQ_ERR_DEVICE_BAD_INPUT);
-                valid = 0;
-            }
-        }
-        sm.tile_valid = valid;
-        sm.group = g;
-        sm.m_tile = mt;
-        sm.n_tile = nt;
-        sm.row_begin = rb;
-        sm.row_end = re;
+        for (int i = threadIdx.x; i <= groups; i += NUM_THREADS) sm.off[i] = offsets[i];
+    }
+    if (threadIdx.x == 32) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.full[s], 2);     // TMA bytes + scale-factor warp
             mbar_init(&sm.empty[s], 1);    // tcgen05.commit
         }
         mbar_init(&sm.tmem_full, 1);
         fence_barrier_init();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int valid = 0, g = 0, mt = 0, nt = 0;
+        int32_t rb = 0, re = (int32_t)M;
+        const int t = blockIdx.x;
+        if (offsets == nullptr) {
+            mt = t / n_tiles;
+            nt = t - mt * n_tiles;
+            valid = (int64_t)mt * BM < M;
+        } else {
+            bool bad = sm.off[0] != 0 || sm.off[groups] != (int32_t)M;
+            int before = 0;                          // tiles of the groups in earlier chunks
+            for (int c0 = 0; c0 < groups; c0 += 32) {
+                const int e = c0 + lane;
+                const int32_t b0 = e < groups ? sm.off[e] : 0, b1 = e < groups ? sm.off[e + 1] : 0;
+                if (b1 < b0) bad = true;
+                const int tiles = b1 > b0 ? ((b1 - b0 + BM - 1) / BM) * n_tiles : 0;
+                int incl = tiles;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                const int lo = before + incl - tiles;
+                const unsigned hit = __ballot_sync(0xFFFFFFFFu, tiles > 0 && t >= lo && t < lo + tiles);
+                if (hit) {
+                    const int src = __ffs(hit) - 1;
+                    const int tt = t - __shfl_sync(0xFFFFFFFFu, lo, src);
+                    g = c0 + src;
+                    rb = __shfl_sync(0xFFFFFFFFu, b0, src);
+                    re = __shfl_sync(0xFFFFFFFFu, b1, src);
+                    mt = tt / n_tiles;
+                    nt = tt - mt * n_tiles;
+                    valid = 1;
+                }
+                before += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            }
+            if (__any_sync(0xFFFFFFFFu, bad)) {
+                if (blockIdx.x == 0 && lane == 0) raise_device_error(err, FPQ_ERR_DEVICE_BAD_INPUT);
+                valid = 0;
+            }
+        }
+        if (lane == 0) {
+            sm.tile_valid = valid;
+            sm.group = g;
+            sm.m_tile = mt;
+            sm.n_tile = nt;
+            sm.row_begin = rb;
+            sm.row_end = re;
+        }
     }
     __syncthreads();
     if (!sm.tile_valid) return;
@@ -265,32 +290,52 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         }
     } else if (warp >= 4) {
         // ---------------------------------------------------------- epilogue
+        // Once the last MMA has completed the operand ring is free: each warp
+        // stages its 32 x 256 block of C there (row l of the block at l *
+        // row_bytes, 16-byte chunk c at position c ^ l, so neither the
+        // writes by rows nor the reads along a row conflict), then writes C
+        // one full row at a time (512 or 1024 contiguous bytes per store
+        // instruction), skipping rows outside the group and columns past N.
         const int q = warp & 3;                       // TMEM lane quadrant of this warp
-        const int64_t row = a_row0 + 32 * q + lane;
-        const bool row_ok = row < a_rows_end;
+        const int64_t row0 = a_row0 + 32 * q;
         if (wait_or_timeout(&sm.tmem_full, 0, err, timeout_ns)) {
             tc_fence_after();
+            uint8_t* stage = &sm.a[0][0] + (warp - 4) * (32 * BN * 4);
+            const int row_bytes = c_f32 ? BN * 4 : BN * 2;
+            uint8_t* my_row = stage + lane * row_bytes;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
                 tmem_ld_wait();
-                const int64_t col0 = n0 + 32 * c;
-                if (!row_ok || col0 >= N) continue;
                 if (c_f32) {
-                    float* out = reinterpret_cast<float*>(C) + row * N + col0;
 #pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        if (col0 + 4 * v < N) st_v4(out + 4 * v, make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]));
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(my_row + 16 * ((8 * c + j) ^ lane)) =
+                            make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
                 } else {
-                    uint16_t* out = reinterpret_cast<uint16_t*>(C) + row * N + col0;
-                    uint32_t h[16];
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) h[v] = f32x2_to_bf16x2(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t h[4];
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        if (col0 + 8 * v < N) st_v4(out + 8 * v, make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]));
+                        for (int e = 0; e < 4; ++e)
+                            h[e] = f32x2_to_bf16x2(__uint_as_float(r[8 * j + 2 * e]), __uint_as_float(r[8 * j + 2 * e + 1]));
+                        *reinterpret_cast<uint4*>(my_row + 16 * ((4 * c + j) ^ lane)) = make_uint4(h[0], h[1], h[2], h[3]);
+                    }
                 }
+            }
+            __syncwarp();
+            const int chunks = row_bytes / 16;                    // 32 (bf16) or 64 (fp32) per row
+            const int cols_per_chunk = c_f32 ? 4 : 8;
+#pragma unroll 1
+            for (int rr = 0; rr < 32; ++rr) {
+                const int64_t row = row0 + rr;
+                if (row >= a_rows_end) break;
+                const uint8_t* src_row = stage + rr * row_bytes;
+                uint8_t* dst_row = reinterpret_cast<uint8_t*>(C) + (row * N + n0) * (c_f32 ? 4 : 2);
+                for (int ch = lane; ch < chunks; ch += 32)
+                    if (n0 + (int64_t)ch * cols_per_chunk < N)
+                        st_v4(dst_row + 16 * ch, *reinterpret_cast<const uint4*>(src_row + 16 * (ch ^ rr)));
             }
         }
     }
