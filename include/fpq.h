@@ -192,6 +192,28 @@ FPQ_API fpq_status fpq_scaled_gemm(fpq_format fmt_a, const void* aq, const void*
                            void* stream);
 
 /*
+ * fpq_scaled_gemm_nvfp4 -- C = gA gB (A * B^T) on NVFP4 operands with fp32
+ * accumulation ["fireworks-prequant 0.1.0" Formats: nvfp4 = packed FP4 +
+ * FP8 block scales]:
+ *   C[m,n] = gA gB sum_k e2m1(A[m,k]) sA[m,k/16] e2m1(B[n,k]) sB[n,k/16].
+ *
+ *   aq   uint8 [m, k/2] packed E2M1 (element 2i in the low nibble of byte i)
+ *   as   uint8 E4M3 [m, k/16] block scales
+ *   ag   fp32 device scalar: A's tensor scale g (as written by
+ *        fpq_quantize_block with FPQ_NVFP4)
+ *   bq, bs, bg   the same for B [n, k] (weights, K-major)
+ *   c    [m, n] bf16 (FPQ_OUT_BF16, round-to-nearest-even) or fp32
+ *
+ * The tensor cores multiply the codes with their block scales exactly and
+ * accumulate in fp32; the epilogue multiplies by fp32(gA gB).  Requires
+ * k % 128 == 0, n % 16 == 0, m >= 1; ag and bg 4-byte aligned, the other
+ * pointers 16-byte aligned.  Errors: as fpq_scaled_gemm.
+ */
+FPQ_API fpq_status fpq_scaled_gemm_nvfp4(const void* aq, const void* as, const float* ag, const void* bq,
+                                         const void* bs, const float* bg, int64_t m, int64_t n, int64_t k,
+                                         void* c, int32_t c_dtype, void* stream);
+
+/*
  * fpq_grouped_scaled_gemm -- per-expert product over a token-permuted
  * activation matrix (MoE routed experts) [FP "Quick start": routed MoE
  * expert projections; DS "Как FP8 связан с MoE-архитектурой DeepSeek V3"]:

@@ -24,9 +24,10 @@ import torch
 __all__ = [
     "FP8_1x128", "FP8_128x128", "MXFP8", "NVFP4", "OUT_BF16", "OUT_F32", "FpqError", "lib_path", "load",
     "fpq_version", "fpq_quantize_workspace_bytes", "fpq_quantize_block", "fpq_dequantize",
-    "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_grouped_scaled_gemm", "fpq_get_device_error",
+    "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_scaled_gemm_nvfp4", "fpq_grouped_scaled_gemm",
+    "fpq_get_device_error",
     "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
-    "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "grouped_scaled_gemm",
+    "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "scaled_gemm_nvfp4", "grouped_scaled_gemm",
     "scale_shape", "code_shape",
 ]
 
@@ -71,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "fpq_dequantize": (I32, [I32, P, P, P, I64, I64, I64, P, P]),
         "fpq_lora_merge_fakequant": (I32, [P, P, P, I64, I64, I32, F, P, P, P, P]),
         "fpq_scaled_gemm": (I32, [I32, P, P, I32, P, P, I64, I64, I64, P, I32, P]),
+        "fpq_scaled_gemm_nvfp4": (I32, [P, P, P, P, P, P, I64, I64, I64, P, I32, P]),
         "fpq_grouped_scaled_gemm": (I32, [I32, P, P, P, P, P, I32, I64, I64, I64, P, I32, P]),
         "fpq_get_device_error": (I32, [P, ctypes.POINTER(I32)]),
         "fpq_quantize_nvfp4_noalloc": (I32, [P, I64, I64, I64, P, P, P, P]),
@@ -132,6 +134,11 @@ def fpq_lora_merge_fakequant(w, lora_a, lora_b, n, k, r, alpha_over_r, wq, ws, w
 def fpq_scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, m, n, k, c, c_dtype, stream=None):
     _check(load().fpq_scaled_gemm(fmt_a, _ptr(aq), _ptr(as_), fmt_b, _ptr(bq), _ptr(bs), m, n, k, _ptr(c), c_dtype,
                                 _stream(stream)), "fpq_scaled_gemm")
+
+
+def fpq_scaled_gemm_nvfp4(aq, as_, ag, bq, bs, bg, m, n, k, c, c_dtype, stream=None):
+    _check(load().fpq_scaled_gemm_nvfp4(_ptr(aq), _ptr(as_), _ptr(ag), _ptr(bq), _ptr(bs), _ptr(bg), m, n, k,
+                                      _ptr(c), c_dtype, _stream(stream)), "fpq_scaled_gemm_nvfp4")
 
 
 def fpq_grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, groups, total_m, n, k, c, c_dtype, stream=None):
@@ -230,6 +237,18 @@ def scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, out_dtype=torch.bfloat16, stream=
     c = torch.empty((m, n), dtype=out_dtype, device=aq.device)
     fpq_scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, m, n, k, c, OUT_F32 if out_dtype == torch.float32 else OUT_BF16,
                     stream)
+    return c
+
+
+def scaled_gemm_nvfp4(aq, as_, ag, bq, bs, bg, out_dtype=torch.bfloat16, stream=None):
+    """C = ag bg (A B^T) for NVFP4 operands as returned by quantize(x, NVFP4):
+    aq [m, k/2] packed codes, as_ [m, k/16] E4M3 scales, ag a one-element
+    fp32 tensor (likewise for B [n, k])."""
+    m, k = aq.shape[0], aq.shape[1] * 2
+    n = bq.shape[0]
+    c = torch.empty((m, n), dtype=out_dtype, device=aq.device)
+    fpq_scaled_gemm_nvfp4(aq, as_, ag, bq, bs, bg, m, n, k, c, OUT_F32 if out_dtype == torch.float32 else OUT_BF16,
+                          stream)
     return c
 
 

@@ -212,6 +212,28 @@ fpq_status fpq_scaled_gemm(fpq_format fmt_a, const void* aq, const void* as, fpq
     return FPQ_ERR_UNSUPPORTED;
 }
 
+fpq_status fpq_scaled_gemm_nvfp4(const void* aq, const void* as, const float* ag, const void* bq, const void* bs,
+                                 const float* bg, int64_t m, int64_t n, int64_t k, void* c, int32_t c_dtype,
+                                 void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (m < 1 || n < 16 || n % 16 || k < 128 || k % 128 || (c_dtype != FPQ_OUT_BF16 && c_dtype != FPQ_OUT_F32) ||
+        m > (1 << 30) || n > (1 << 30) || k > (1 << 30)) {
+        set_detail("need m >= 1, n a positive multiple of 16, k a positive multiple of 128, c_dtype BF16|F32");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if ((st = check_ptrs({aq, as, bq, bs, c})) != FPQ_OK) return st;
+    if (!ag || !bg) { set_detail("null tensor scale pointer"); return FPQ_ERR_INVALID_ARG; }
+    if ((reinterpret_cast<uintptr_t>(ag) & 3) || (reinterpret_cast<uintptr_t>(bg) & 3)) {
+        set_detail("tensor scale pointers must be 4-byte aligned");
+        return FPQ_ERR_ALIGNMENT;
+    }
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_gemm_nvfp4(aq, as, ag, bq, bs, bg, m, n, k, c, c_dtype == FPQ_OUT_F32, d->err,
+                                            (cudaStream_t)stream), "nvfp4 gemm launch");
+}
+
 fpq_status fpq_grouped_scaled_gemm(fpq_format fmt, const void* aq, const void* as, const void* bq,
                                    const void* bs, const int32_t* group_offsets, int32_t groups,
                                    int64_t total_m, int64_t n, int64_t k, void* c, int32_t c_dtype,

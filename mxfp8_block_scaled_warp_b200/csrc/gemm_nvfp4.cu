@@ -1,0 +1,323 @@
+// gemm_nvfp4.cu -- block-scaled NVFP4 GEMM on the 5th-generation tensor
+// cores: C = gA gB (A * B^T) with A [M, K], B [N, K] packed E2M1 codes (two
+// per byte, element 2i in the low nibble), one E4M3 scale per 16 K-elements
+// of every row and one fp32 tensor scale per operand ("fireworks-prequant
+// 0.1.0", Formats: packed FP4 + FP8 block scales); fp32 accumulation in
+// TMEM, bf16 (round-to-nearest-even) or fp32 output.
+//
+// Per CTA one 128 x 256 output tile; the K loop runs over 256-wide K tiles
+// (128 bytes of codes per row) through a STAGES-deep shared-memory ring.
+// One tcgen05.mma kind::mxf4nvf4 covers K = 64 and reads, for row m of its
+// operand, the 32-bit TMEM word holding the row's four block scales of those
+// 64 elements: lane m mod 32 of the scale columns, column base + m / 32.  A
+// K tile therefore needs four such scale atoms for A (4 columns each) and
+// four for B (8 columns each: 256 rows).
+//
+// Warp roles:
+//   warp 0  TMA producer: A and B code tiles (128-byte swizzle, no multicast)
+//   warp 2  TMEM allocator and MMA issuer (one elected thread): tcgen05.cp of
+//           the scale atoms, 4 x tcgen05.mma per K tile, tcgen05.commit
+//   warps 4-7 during the K loop, scale loaders: warp 4 + i serves ring stage
+//           i (K tiles i, i + 4, ...), reading the row-major E4M3 scales of
+//           the tile's rows one K tile ahead and writing them in the
+//           shared-memory atom layout the shared->TMEM copy expects (lane l:
+//           rows l, l+32, l+64, l+96), so four K tiles of scale loads are in
+//           flight; afterwards, the epilogue: tcgen05.ld of the accumulator,
+//           times gA gB, convert, stage in the freed operand ring, store C a
+//           row at a time
+// Every wait on an mbarrier is bounded by wall time (4 s); on expiry the
+// kernel records FPQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace fpq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 256;          // BK in elements (128 bytes of codes)
+constexpr int BKB = BK / 2;                          // code bytes per row per K tile
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BKB, B_TILE = BN * BKB;
+constexpr int MMAS_PER_TILE = BK / 64;               // K = 64 per instruction
+constexpr int ATOM_BYTES = 512;                      // 128 rows x 4 scale bytes
+constexpr int SFA_BYTES = MMAS_PER_TILE * ATOM_BYTES;          // 4 atoms
+constexpr int SFB_BYTES = MMAS_PER_TILE * 2 * ATOM_BYTES;      // 8 atoms (256 rows)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL0 = BN;                     // scale columns follow the accumulator
+constexpr uint32_t SFA_COLS = 4 * MMAS_PER_TILE;     // per stage
+constexpr uint32_t SFB_COLS = 8 * MMAS_PER_TILE;
+constexpr uint32_t SF_COLS_PER_STAGE = SFA_COLS + SFB_COLS;
+static_assert(SF_COL0 + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM columns");
+constexpr int NUM_THREADS = 256;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+
+struct __align__(1024) Smem {
+    uint8_t a[STAGES][A_TILE];
+    uint8_t b[STAGES][B_TILE];
+    uint8_t sfa[STAGES][SFA_BYTES];
+    uint8_t sfb[STAGES][SFB_BYTES];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tmem_full;
+    uint32_t tmem_base;
+};
+static_assert(4 * 32 * BN * 4 <= STAGES * (A_TILE + B_TILE), "epilogue staging exceeds the ring");
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > kTimeoutNs) {
+            raise_device_error(err, FPQ_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int j) {
+    return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+// The 16 scale bytes of row `row` for K tile kt (K elements [256 kt, 256 kt
+// + 256)); rows outside [0, nrows) and bytes past the row's end read as 0.
+__device__ __forceinline__ uint4 load_sf_tile(const uint8_t* sf, int64_t row, int64_t nrows, int64_t pitch, int kt,
+                                              bool vec16) {
+    if (row < 0 || row >= nrows) return make_uint4(0, 0, 0, 0);
+    const uint8_t* p = sf + row * pitch + (int64_t)kt * 16;
+    if (vec16) return *reinterpret_cast<const uint4*>(p);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        w[j] = ((int64_t)kt * 16 + 4 * j + 4 <= pitch) ? *reinterpret_cast<const uint32_t*>(p + 4 * j) : 0u;
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const uint8_t* __restrict__ sfa, const float* __restrict__ ga, const uint8_t* __restrict__ sfb,
+                  const float* __restrict__ gb, int64_t M, int64_t N, int64_t K, void* __restrict__ C, int c_f32,
+                  uint32_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = (int)((N + BN - 1) / BN);
+    const int mt = blockIdx.x / n_tiles, nt = blockIdx.x - mt * n_tiles;
+    const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
+    const int KT = (int)((K + BK - 1) / BK);
+    const int64_t sf_pitch = K / 16;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 2);     // TMA bytes + scale loader
+            mbar_init(&sm.empty[s], 1);    // tcgen05.commit
+        }
+        mbar_init(&sm.tmem_full, 1);
+        fence_barrier_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    // Everything above touched only shared memory and TMEM; global inputs
+    // and the output are accessed after the preceding grids complete.
+    pdl_wait();
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
+                mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE);
+                tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BKB, (int32_t)m0);
+                tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BKB, (int32_t)n0);
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------------------------------------------------- MMA issuer
+        if (elect_one()) {
+            const uint32_t idesc = idesc_mxf4nvf4(BM, BN);
+            bool ok = true;
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!wait_or_timeout(&sm.full[s], ph, err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t col_a = tmem + SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
+                const uint32_t col_b = col_a + SFA_COLS;
+#pragma unroll
+                for (int j = 0; j < MMAS_PER_TILE; ++j) {
+                    tmem_cp_32x128b_warpx4(col_a + 4 * j,
+                                           smem_desc(smem_u32(sm.sfa[s] + j * ATOM_BYTES), 0, 128, kLayoutNone));
+                    tmem_cp_32x128b_warpx4(col_b + 8 * j,
+                                           smem_desc(smem_u32(sm.sfb[s] + 2 * j * ATOM_BYTES), 0, 128, kLayoutNone));
+                    tmem_cp_32x128b_warpx4(col_b + 8 * j + 4,
+                                           smem_desc(smem_u32(sm.sfb[s] + (2 * j + 1) * ATOM_BYTES), 0, 128,
+                                                     kLayoutNone));
+                }
+                const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
+#pragma unroll
+                for (int j = 0; j < MMAS_PER_TILE; ++j)
+                    mma_mxf4nvf4(tmem, desc_kmajor_sw128(a_base + 32 * j), desc_kmajor_sw128(b_base + 32 * j), idesc,
+                                 col_a + 4 * j, col_b + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                mma_commit(&sm.empty[s]);
+            }
+            if (ok) mma_commit(&sm.tmem_full);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------- scale loader
+        // Lane l holds rows l + 32 i of A (i < 4) and of B (i < 8); atom j of a
+        // K tile (the scales of MMA j) is, per lane, the j-th 32-bit word of
+        // each of its rows: 16 bytes = rows l, l+32, l+64, l+96.
+        {
+            const int s = warp - 4;                   // this warp's ring stage
+            const bool vec16 = (sf_pitch % 16) == 0;
+            uint4 ca[4], cb[8];
+            if (s < KT) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ca[i] = load_sf_tile(sfa, m0 + lane + 32 * i, M, sf_pitch, s, vec16);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cb[i] = load_sf_tile(sfb, n0 + lane + 32 * i, N, sf_pitch, s, vec16);
+            }
+            for (int kt = s; kt < KT; kt += STAGES) {
+                uint4 na[4], nb[8];
+                if (kt + STAGES < KT) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        na[i] = load_sf_tile(sfa, m0 + lane + 32 * i, M, sf_pitch, kt + STAGES, vec16);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        nb[i] = load_sf_tile(sfb, n0 + lane + 32 * i, N, sf_pitch, kt + STAGES, vec16);
+                }
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!__all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.empty[s], ph ^ 1u, err))) break;
+#pragma unroll
+                for (int j = 0; j < MMAS_PER_TILE; ++j) {
+                    *reinterpret_cast<uint4*>(sm.sfa[s] + j * ATOM_BYTES + lane * 16) =
+                        make_uint4(word(ca[0], j), word(ca[1], j), word(ca[2], j), word(ca[3], j));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        *reinterpret_cast<uint4*>(sm.sfb[s] + (2 * j + h) * ATOM_BYTES + lane * 16) =
+                            make_uint4(word(cb[4 * h], j), word(cb[4 * h + 1], j), word(cb[4 * h + 2], j),
+                                       word(cb[4 * h + 3], j));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.full[s]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ca[i] = na[i];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cb[i] = nb[i];
+            }
+        }
+        // ---------------------------------------------------------- epilogue
+        // Once the last MMA has completed the operand ring is free: each warp
+        // stages its 32 x 256 block of C there (row l at l * row_bytes,
+        // 16-byte chunk c at position c ^ l), then writes C one full row at a
+        // time, skipping rows past M and columns past N.
+        const int q = warp & 3;                       // TMEM lane quadrant of this warp
+        const int64_t row0 = m0 + 32 * q;
+        if (wait_or_timeout(&sm.tmem_full, 0, err)) {
+            tc_fence_after();
+            const float gab = __fmul_rn(__ldg(ga), __ldg(gb));
+            uint8_t* stage = &sm.a[0][0] + (warp - 4) * (32 * BN * 4);
+            const int row_bytes = c_f32 ? BN * 4 : BN * 2;
+            uint8_t* my_row = stage + lane * row_bytes;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
+                tmem_ld_wait();
+                float f[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(__uint_as_float(r[e]), gab);
+                if (c_f32) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(my_row + 16 * ((8 * c + j) ^ lane)) =
+                            make_uint4(__float_as_uint(f[4 * j]), __float_as_uint(f[4 * j + 1]),
+                                       __float_as_uint(f[4 * j + 2]), __float_as_uint(f[4 * j + 3]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t h[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) h[e] = f32x2_to_bf16x2(f[8 * j + 2 * e], f[8 * j + 2 * e + 1]);
+                        *reinterpret_cast<uint4*>(my_row + 16 * ((4 * c + j) ^ lane)) = make_uint4(h[0], h[1], h[2], h[3]);
+                    }
+                }
+            }
+            __syncwarp();
+            const int chunks = row_bytes / 16;
+            const int cols_per_chunk = c_f32 ? 4 : 8;
+#pragma unroll 1
+            for (int rr = 0; rr < 32; ++rr) {
+                const int64_t row = row0 + rr;
+                if (row >= M) break;
+                const uint8_t* src_row = stage + rr * row_bytes;
+                uint8_t* dst_row = reinterpret_cast<uint8_t*>(C) + (row * N + n0) * (c_f32 ? 4 : 2);
+                for (int ch = lane; ch < chunks; ch += 32)
+                    if (n0 + (int64_t)ch * cols_per_chunk < N)
+                        st_v4(dst_row + 16 * ch, *reinterpret_cast<const uint4*>(src_row + 16 * (ch ^ rr)));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+int smem_bytes() { return (int)sizeof(Smem) + 1024; }
+
+
+}  // namespace
+
+cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, const void* bq, const void* bs,
+                              const float* bg, int64_t m, int64_t n, int64_t k, void* c, int c_f32, uint32_t* err,
+                              cudaStream_t st) {
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e != cudaSuccess) return e;
+        configured[dev] = 1;
+    }
+    CUtensorMap ta, tb;
+    e = make_tmap_u8_2d(&ta, aq, (uint64_t)m, (uint64_t)(k / 2), (uint64_t)(k / 2), BM, BKB);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_u8_2d(&tb, bq, (uint64_t)n, (uint64_t)(k / 2), (uint64_t)(k / 2), BN, BKB);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
+    return launch_pdl(gemm_nvfp4_kernel, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta, tb,
+                      (const uint8_t*)as, ag, (const uint8_t*)bs, bg, m, n, k, c, c_f32, err);
+}
+
+}  // namespace fpq

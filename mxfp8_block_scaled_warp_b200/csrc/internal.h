@@ -34,6 +34,11 @@ cudaError_t launch_gemm_fp8_f32scale(const void* aq, const float* as, const void
                                      const float* bs, int64_t m, int64_t n, int64_t k, void* c,
                                      int c_f32, uint32_t* err, int sms, cudaStream_t st);
 
+// NVFP4 GEMM: C = ga gb sum_k A[m,k] B[n,k] (packed E2M1, E4M3 per 16).
+cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, const void* bq, const void* bs,
+                              const float* bg, int64_t m, int64_t n, int64_t k, void* c, int c_f32, uint32_t* err,
+                              cudaStream_t st);
+
 cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void* bq,
                                       const void* bs, const int32_t* offsets, int groups,
                                       int64_t total_m, int64_t n, int64_t k, void* c, int c_f32,

@@ -272,6 +272,17 @@ __host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int m, int n, uint32_t sfa
          | ((sfa_id & 3u) << 29);
 }
 
+// Instruction descriptor, kind::mxf4nvf4 with one UE4M3 scale per 16
+// K-elements (NVFP4): A, B packed E2M1 (format code 1), K-major, dense
+// K = 64 per instruction, scale-factor ids 0 (each MMA consumes the four
+// scale bytes of its row's 32-bit TMEM word).
+__host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int m, int n) {
+    return (1u << 7) | (1u << 10)           // A, B: E2M1
+         | ((uint32_t)(n >> 3) << 17)
+         | (0u << 23)                       // scale format: UE4M3
+         | ((uint32_t)(m >> 4) << 24);
+}
+
 // ----------------------------------------------------------------- MMA
 
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -289,6 +300,18 @@ __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, u
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %6, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// D (+)= A * B with E2M1 operands and UE4M3 scales per 16 K-elements taken
+// from TMEM (K = 64 per instruction).
+__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
         :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
         : "memory");
 }
