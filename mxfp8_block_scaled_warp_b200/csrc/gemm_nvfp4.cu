@@ -29,6 +29,8 @@
 // kernel records FPQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
 #include <cuda.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -62,7 +64,8 @@ struct __align__(1024) Smem {
     uint8_t b[STAGES][B_TILE];
     uint8_t sfa[STAGES][SFA_BYTES];
     uint8_t sfb[STAGES][SFB_BYTES];
-    uint64_t full[STAGES];
+    uint64_t full[STAGES];     // operand tiles (and, with TMA scales, the scale rows) have landed
+    uint64_t sfr[STAGES];      // scale atoms written
     uint64_t empty[STAGES];
     uint64_t tmem_full;
     uint32_t tmem_base;
@@ -106,8 +109,30 @@ __device__ __forceinline__ uint4 load_sf_tile(const uint8_t* sf, int64_t row, in
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Writes the scale atoms of one ring stage from 16-byte row chunks: ca[i] =
+// the K tile's scales of A row lane + 32 i, cb[i] those of B row lane + 32 i.
+__device__ __forceinline__ void write_atoms(uint8_t* sfa_s, uint8_t* sfb_s, const uint4 (&ca)[4],
+                                            const uint4 (&cb)[8], int lane) {
+#pragma unroll
+    for (int j = 0; j < MMAS_PER_TILE; ++j) {
+        *reinterpret_cast<uint4*>(sfa_s + j * ATOM_BYTES + lane * 16) =
+            make_uint4(word(ca[0], j), word(ca[1], j), word(ca[2], j), word(ca[3], j));
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            *reinterpret_cast<uint4*>(sfb_s + (2 * j + h) * ATOM_BYTES + lane * 16) =
+                make_uint4(word(cb[4 * h], j), word(cb[4 * h + 1], j), word(cb[4 * h + 2], j),
+                           word(cb[4 * h + 3], j));
+    }
+}
+
+// TMA_SF: the scale rows of each K tile arrive by TMA with the operand tiles
+// (dense, row r at 16 r) and the stage's loader warp rearranges them in place
+// into atoms; otherwise (scale rows not 16-byte aligned) the loader warps
+// read them from global memory themselves.
+template <bool TMA_SF>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                   const uint8_t* __restrict__ sfa, const float* __restrict__ ga, const uint8_t* __restrict__ sfb,
                   const float* __restrict__ gb, int64_t M, int64_t N, int64_t K, void* __restrict__ C, int c_f32,
                   uint32_t* err) {
@@ -122,7 +147,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sm.full[s], 2);     // TMA bytes + scale loader
+            mbar_init(&sm.full[s], 1);     // TMA bytes
+            mbar_init(&sm.sfr[s], 1);      // scale loader
             mbar_init(&sm.empty[s], 1);    // tcgen05.commit
         }
         mbar_init(&sm.tmem_full, 1);
@@ -145,13 +171,21 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         if (elect_one()) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
+            if (TMA_SF) {
+                tma_prefetch_desc(&tmSA);
+                tma_prefetch_desc(&tmSB);
+            }
             for (int kt = 0; kt < KT; ++kt) {
                 const int s = kt % STAGES;
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
                 if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
-                mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE);
+                mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE + (TMA_SF ? SFA_BYTES + SFB_BYTES : 0));
                 tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BKB, (int32_t)m0);
                 tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BKB, (int32_t)n0);
+                if (TMA_SF) {
+                    tma_load_2d(sm.sfa[s], &tmSA, &sm.full[s], kt * 16, (int32_t)m0);
+                    tma_load_2d(sm.sfb[s], &tmSB, &sm.full[s], kt * 16, (int32_t)n0);
+                }
             }
         }
     } else if (warp == 2) {
@@ -162,7 +196,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             for (int kt = 0; kt < KT; ++kt) {
                 const int s = kt % STAGES;
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
-                if (!wait_or_timeout(&sm.full[s], ph, err)) { ok = false; break; }
+                if (!wait_or_timeout(&sm.full[s], ph, err) || !wait_or_timeout(&sm.sfr[s], ph, err)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t col_a = tmem + SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
                 const uint32_t col_b = col_a + SFA_COLS;
@@ -190,8 +227,24 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         // Lane l holds rows l + 32 i of A (i < 4) and of B (i < 8); atom j of a
         // K tile (the scales of MMA j) is, per lane, the j-th 32-bit word of
         // each of its rows: 16 bytes = rows l, l+32, l+64, l+96.
-        {
+        if (TMA_SF) {
             const int s = warp - 4;                   // this warp's ring stage
+            for (int kt = s; kt < KT; kt += STAGES) {
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!__all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.full[s], ph, err))) break;
+                uint4 ca[4], cb[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ca[i] = *reinterpret_cast<const uint4*>(sm.sfa[s] + (lane + 32 * i) * 16);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cb[i] = *reinterpret_cast<const uint4*>(sm.sfb[s] + (lane + 32 * i) * 16);
+                __syncwarp();
+                write_atoms(sm.sfa[s], sm.sfb[s], ca, cb, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sfr[s]);
+            }
+        } else {
+            const int s = warp - 4;
             const bool vec16 = (sf_pitch % 16) == 0;
             uint4 ca[4], cb[8];
             if (s < KT) {
@@ -212,19 +265,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 }
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
                 if (!__all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.empty[s], ph ^ 1u, err))) break;
-#pragma unroll
-                for (int j = 0; j < MMAS_PER_TILE; ++j) {
-                    *reinterpret_cast<uint4*>(sm.sfa[s] + j * ATOM_BYTES + lane * 16) =
-                        make_uint4(word(ca[0], j), word(ca[1], j), word(ca[2], j), word(ca[3], j));
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        *reinterpret_cast<uint4*>(sm.sfb[s] + (2 * j + h) * ATOM_BYTES + lane * 16) =
-                            make_uint4(word(cb[4 * h], j), word(cb[4 * h + 1], j), word(cb[4 * h + 2], j),
-                                       word(cb[4 * h + 3], j));
-                }
+                write_atoms(sm.sfa[s], sm.sfb[s], ca, cb, lane);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.full[s]);
+                if (lane == 0) mbar_arrive(&sm.sfr[s]);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) ca[i] = na[i];
 #pragma unroll
@@ -301,12 +345,17 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
                               const float* bg, int64_t m, int64_t n, int64_t k, void* c, int c_f32, uint32_t* err,
                               cudaStream_t st) {
     static int configured[64] = {0};
+    // Scale rows can come by TMA when every row starts on a 16-byte boundary
+    // (the matrices themselves are 16-byte aligned).
+    const bool tma_sf = (k / 16) % 16 == 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        e = cudaFuncSetAttribute(gemm_nvfp4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(gemm_nvfp4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
         if (e != cudaSuccess) return e;
         configured[dev] = 1;
     }
@@ -315,9 +364,21 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
     if (e != cudaSuccess) return e;
     e = make_tmap_u8_2d(&tb, bq, (uint64_t)n, (uint64_t)(k / 2), (uint64_t)(k / 2), BN, BKB);
     if (e != cudaSuccess) return e;
+    CUtensorMap tsa, tsb;
+    std::memset(&tsa, 0, sizeof(tsa));
+    std::memset(&tsb, 0, sizeof(tsb));
+    if (tma_sf) {
+        e = make_tmap_2d(&tsa, as, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)m, (uint64_t)(k / 16), (uint64_t)(k / 16),
+                         BM, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (e != cudaSuccess) return e;
+        e = make_tmap_2d(&tsb, bs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n, (uint64_t)(k / 16), (uint64_t)(k / 16),
+                         BN, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (e != cudaSuccess) return e;
+    }
     const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
-    return launch_pdl(gemm_nvfp4_kernel, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta, tb,
-                      (const uint8_t*)as, ag, (const uint8_t*)bs, bg, m, n, k, c, c_f32, err);
+    return launch_pdl(tma_sf ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>, dim3((unsigned)grid),
+                      dim3(NUM_THREADS), smem_bytes(), st, ta, tb, tsa, tsb, (const uint8_t*)as, ag,
+                      (const uint8_t*)bs, bg, m, n, k, c, c_f32, err);
 }
 
 }  // namespace fpq

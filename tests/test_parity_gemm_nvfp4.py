@@ -34,8 +34,10 @@ def pack(codes: np.ndarray) -> np.ndarray:
     return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
 
 
+# K a multiple of 256 takes the path whose scale rows arrive by TMA (rows of
+# K/16 bytes on 16-byte boundaries); other K read the scale rows directly.
 @pytest.mark.parametrize("m,n,k", [(128, 256, 256), (200, 272, 384), (1, 16, 128), (300, 512, 1024),
-                                   (257, 256, 640)])
+                                   (257, 256, 640), (160, 256, 896), (384, 512, 1152)])
 def test_nvfp4_gemm_random(fpq, orc, m, n, k):
     a = rand((m, k), 700 + m, std=0.02, outliers=0.01)
     b = rand((n, k), 800 + n, std=0.02, outliers=0.01)
@@ -108,3 +110,4 @@ def test_nvfp4_gemm_full_size_sampled(fpq, orc):
     got = c[torch.from_numpy(rr.ravel()).cuda(), torch.from_numpy(cc.ravel()).cuda()]
     check(got, ref, orc, "nvfp4 full size", rms=float(np.sqrt(np.mean(ref ** 2))))
     assert fpq.fpq_get_device_error() == 0
+
