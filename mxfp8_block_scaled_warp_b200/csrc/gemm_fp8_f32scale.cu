@@ -101,12 +101,6 @@ __device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
     }
 }
 
-// Byte offset of 16-byte chunk j (0-7) of row r in a 32-row box of 128-byte
-// rows stored with the 128-byte swizzle (chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t sw128_offset(int r, int j) {
-    return (uint32_t)(r * 128 + 16 * (j ^ (r & 7)));
-}
-
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_fp8_f32scale_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmC, const float* __restrict__ sA,

@@ -70,7 +70,8 @@ struct __align__(1024) Smem {
     uint64_t tmem_full;
     uint32_t tmem_base;
 };
-static_assert(4 * 32 * BN * 4 <= STAGES * (A_TILE + B_TILE), "epilogue staging exceeds the ring");
+constexpr int EPI_WARP_BYTES = 32 * 128 * 4;       // a warp's 32 x 128 block of C, fp32
+static_assert(8 * EPI_WARP_BYTES <= STAGES * (A_TILE + B_TILE), "epilogue staging exceeds the ring");
 
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
@@ -133,6 +134,7 @@ template <bool TMA_SF>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                  const __grid_constant__ CUtensorMap tmC,
                   const uint8_t* __restrict__ sfa, const float* __restrict__ ga, const uint8_t* __restrict__ sfb,
                   const float* __restrict__ gb, int64_t M, int64_t N, int64_t K, void* __restrict__ C, int c_f32,
                   uint32_t* err) {
@@ -171,6 +173,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         if (elect_one()) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmC);
             if (TMA_SF) {
                 tma_prefetch_desc(&tmSA);
                 tma_prefetch_desc(&tmSB);
@@ -275,56 +278,61 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 for (int i = 0; i < 8; ++i) cb[i] = nb[i];
             }
         }
-        // ---------------------------------------------------------- epilogue
-        // Once the last MMA has completed the operand ring is free: each warp
-        // stages its 32 x 256 block of C there (row l at l * row_bytes,
-        // 16-byte chunk c at position c ^ l), then writes C one full row at a
-        // time, skipping rows past M and columns past N.
-        const int q = warp & 3;                       // TMEM lane quadrant of this warp
-        const int64_t row0 = m0 + 32 * q;
-        if (wait_or_timeout(&sm.tmem_full, 0, err)) {
+    }
+
+    // -------------------------------------------------------------- epilogue
+    // All eight warps, once the last MMA has completed (the operand ring is
+    // then free): warp w reads TMEM lanes 32 (w & 3) .. + 31 (rows of C) and
+    // columns 128 (w >> 2) .. + 127, multiplies by gA gB, stages the 32 x 128
+    // block in 128-byte-swizzled boxes and writes them with TMA stores (which
+    // clip rows past M and columns past N).
+    __syncwarp();     // the role warps' other lanes wait here for the elected lane, without polling
+    {
+        const int q = warp & 3, half = warp >> 2;
+        const int64_t row0 = m0 + 32 * q, col0 = n0 + 128 * half;
+        const bool ok = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.tmem_full, 0, err));
+        if (ok && row0 < M && col0 < N) {
             tc_fence_after();
             const float gab = __fmul_rn(__ldg(ga), __ldg(gb));
-            uint8_t* stage = &sm.a[0][0] + (warp - 4) * (32 * BN * 4);
-            const int row_bytes = c_f32 ? BN * 4 : BN * 2;
-            uint8_t* my_row = stage + lane * row_bytes;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
-                tmem_ld_wait();
+            uint8_t* stage = &sm.a[0][0] + warp * EPI_WARP_BYTES;
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half + 32 * c), r[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
                 float f[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(__uint_as_float(r[e]), gab);
-                if (c_f32) {
+                for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(__uint_as_float(r[c][e]), gab);
+                if (c_f32) {     // columns 32c .. 32c + 31 = box c, chunks 0..7
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4*>(my_row + 16 * ((8 * c + j) ^ lane)) =
+                        *reinterpret_cast<uint4*>(stage + c * 4096 + sw128_offset(lane, j)) =
                             make_uint4(__float_as_uint(f[4 * j]), __float_as_uint(f[4 * j + 1]),
                                        __float_as_uint(f[4 * j + 2]), __float_as_uint(f[4 * j + 3]));
-                } else {
+                } else {         // columns 32c .. 32c + 31 = box c / 2, chunks 4 (c % 2) .. + 3
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t h[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) h[e] = f32x2_to_bf16x2(f[8 * j + 2 * e], f[8 * j + 2 * e + 1]);
-                        *reinterpret_cast<uint4*>(my_row + 16 * ((4 * c + j) ^ lane)) = make_uint4(h[0], h[1], h[2], h[3]);
+                        *reinterpret_cast<uint4*>(stage + (c / 2) * 4096 + sw128_offset(lane, 4 * (c % 2) + j)) =
+                            make_uint4(h[0], h[1], h[2], h[3]);
                     }
                 }
             }
+            fence_proxy_async_smem();
             __syncwarp();
-            const int chunks = row_bytes / 16;
-            const int cols_per_chunk = c_f32 ? 4 : 8;
-#pragma unroll 1
-            for (int rr = 0; rr < 32; ++rr) {
-                const int64_t row = row0 + rr;
-                if (row >= M) break;
-                const uint8_t* src_row = stage + rr * row_bytes;
-                uint8_t* dst_row = reinterpret_cast<uint8_t*>(C) + (row * N + n0) * (c_f32 ? 4 : 2);
-                for (int ch = lane; ch < chunks; ch += 32)
-                    if (n0 + (int64_t)ch * cols_per_chunk < N)
-                        st_v4(dst_row + 16 * ch, *reinterpret_cast<const uint4*>(src_row + 16 * (ch ^ rr)));
+            if (lane == 0) {
+                const int boxes = c_f32 ? 4 : 2, box_cols = c_f32 ? 32 : 64;
+                for (int x = 0; x < boxes; ++x)
+                    if (col0 + x * box_cols < N)
+                        tma_store_2d(&tmC, stage + x * 4096, (int32_t)(col0 + x * box_cols), (int32_t)row0);
+                bulk_commit_group();
+                bulk_wait_group_read0();     // the staging must stay valid until read
             }
+            __syncwarp();
         }
     }
 
@@ -375,9 +383,17 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
                          BN, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (e != cudaSuccess) return e;
     }
+    CUtensorMap tc;
+    if (c_f32)
+        e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)m, (uint64_t)n, (uint64_t)n * 4, 32, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)n, (uint64_t)n * 2, 32, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
     const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
     return launch_pdl(tma_sf ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>, dim3((unsigned)grid),
-                      dim3(NUM_THREADS), smem_bytes(), st, ta, tb, tsa, tsb, (const uint8_t*)as, ag,
+                      dim3(NUM_THREADS), smem_bytes(), st, ta, tb, tsa, tsb, tc, (const uint8_t*)as, ag,
                       (const uint8_t*)bs, bg, m, n, k, c, c_f32, err);
 }
 

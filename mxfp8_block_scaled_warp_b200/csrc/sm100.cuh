@@ -283,6 +283,12 @@ __host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int m, int n) {
          | ((uint32_t)(m >> 4) << 24);
 }
 
+// Byte offset of 16-byte chunk j (0-7) of row r in a box of 128-byte
+// rows stored with the 128-byte swizzle (chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t sw128_offset(int r, int j) {
+    return (uint32_t)(r * 128 + 16 * (j ^ (r & 7)));
+}
+
 // ----------------------------------------------------------------- MMA
 
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
