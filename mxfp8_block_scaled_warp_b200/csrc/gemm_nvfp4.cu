@@ -126,6 +126,48 @@ __device__ __forceinline__ void write_atoms(uint8_t* sfa_s, uint8_t* sfb_s, cons
     }
 }
 
+// Epilogue of one warp: its 32 accumulator rows x 128 columns (r[c] = TMEM
+// columns 32c .. 32c + 31 of the warp's half, row = lane) times gab, staged in
+// 128-byte-swizzled boxes of 32 rows (fp32: 32 columns, bf16: 64) and
+// written by TMA stores at (col0, row0); the stores clip at M and N.
+__device__ __forceinline__ void stage_and_store(uint8_t* stage, const uint32_t (&r)[4][32], float gab, int c_f32,
+                                                int lane, const CUtensorMap* tmC, int64_t col0, int64_t row0,
+                                                int64_t N) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(__uint_as_float(r[c][e]), gab);
+        if (c_f32) {     // columns 32c .. 32c + 31 = box c, chunks 0..7
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(stage + c * 4096 + sw128_offset(lane, j)) =
+                    make_uint4(__float_as_uint(f[4 * j]), __float_as_uint(f[4 * j + 1]),
+                               __float_as_uint(f[4 * j + 2]), __float_as_uint(f[4 * j + 3]));
+        } else {         // columns 32c .. 32c + 31 = box c / 2, chunks 4 (c % 2) .. + 3
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t h[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) h[e] = f32x2_to_bf16x2(f[8 * j + 2 * e], f[8 * j + 2 * e + 1]);
+                *reinterpret_cast<uint4*>(stage + (c / 2) * 4096 + sw128_offset(lane, 4 * (c % 2) + j)) =
+                    make_uint4(h[0], h[1], h[2], h[3]);
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        const int boxes = c_f32 ? 4 : 2, box_cols = c_f32 ? 32 : 64;
+        for (int x = 0; x < boxes; ++x)
+            if (col0 + x * box_cols < N)
+                tma_store_2d(tmC, stage + x * 4096, (int32_t)(col0 + x * box_cols), (int32_t)row0);
+        bulk_commit_group();
+        bulk_wait_group_read0();     // the staging must stay valid until read
+    }
+    __syncwarp();
+}
+
 // TMA_SF: the scale rows of each K tile arrive by TMA with the operand tiles
 // (dense, row r at 16 r) and the stage's loader warp rearranges them in place
 // into atoms; otherwise (scale rows not 16-byte aligned) the loader warps
@@ -300,39 +342,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             for (int c = 0; c < 4; ++c)
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half + 32 * c), r[c]);
             tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float f[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) f[e] = __fmul_rn(__uint_as_float(r[c][e]), gab);
-                if (c_f32) {     // columns 32c .. 32c + 31 = box c, chunks 0..7
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4*>(stage + c * 4096 + sw128_offset(lane, j)) =
-                            make_uint4(__float_as_uint(f[4 * j]), __float_as_uint(f[4 * j + 1]),
-                                       __float_as_uint(f[4 * j + 2]), __float_as_uint(f[4 * j + 3]));
-                } else {         // columns 32c .. 32c + 31 = box c / 2, chunks 4 (c % 2) .. + 3
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t h[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) h[e] = f32x2_to_bf16x2(f[8 * j + 2 * e], f[8 * j + 2 * e + 1]);
-                        *reinterpret_cast<uint4*>(stage + (c / 2) * 4096 + sw128_offset(lane, 4 * (c % 2) + j)) =
-                            make_uint4(h[0], h[1], h[2], h[3]);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                const int boxes = c_f32 ? 4 : 2, box_cols = c_f32 ? 32 : 64;
-                for (int x = 0; x < boxes; ++x)
-                    if (col0 + x * box_cols < N)
-                        tma_store_2d(&tmC, stage + x * 4096, (int32_t)(col0 + x * box_cols), (int32_t)row0);
-                bulk_commit_group();
-                bulk_wait_group_read0();     // the staging must stay valid until read
-            }
-            __syncwarp();
+            stage_and_store(stage, r, gab, c_f32, lane, &tmC, col0, row0, N);
         }
     }
 
@@ -345,6 +355,228 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 }
 
 int smem_bytes() { return (int)sizeof(Smem) + 1024; }
+
+// ============================================================== CTA pair
+// A cluster of two CTAs computes one 256 x 256 tile with tcgen05 cta_group::2:
+// CTA r holds A rows m0 + 128 r .. + 127 and B rows (output columns)
+// n0 + 128 r .. + 127 of each K tile in its own shared memory, and receives
+// its 128 accumulator rows x 256 columns in its own TMEM.  Per SM a K tile
+// is then 16 + 16 KB of codes instead of 16 + 32 KB.
+//
+// Scales come in chunks of SF_CH K tiles, SF_BUFS chunks in flight: one TMA
+// box of (16 SF_CH)-byte scale rows for this CTA's 128 A rows and one for
+// all 256 B rows of the tile (its accumulator rows meet every output
+// column).  Per-row TMA requests are costly, so wider rows and fewer boxes
+// matter.  Two loader warps per chunk, one per K tile, rearrange a landed
+// chunk in place into the atoms of its K tiles, make them visible to the
+// async proxy and arrive on the leader's sfr barrier; the leader's copy
+// instruction (cta_group::2) moves each CTA's atoms into that CTA's TMEM.
+// The leader's single thread issues all copies and MMAs and commits to the
+// barriers of both CTAs.
+//
+// Warp roles in both CTAs: warp 0 code-tile TMA producer; warp 1 scale-chunk
+// TMA producer; warp 2 TMEM allocator (and, in the leader, MMA issuer);
+// warps 4-7 scale loaders (4-5 even chunks, 6-7 odd); then all eight warps
+// run the epilogue.
+constexpr int PSTAGES = 5;
+constexpr int P_A_TILE = 128 * BKB, P_B_TILE = 128 * BKB;
+constexpr int SF_CH = 2;                                   // K tiles per scale chunk
+constexpr int SF_BUFS = 4;                                 // scale chunks in flight
+constexpr int SFC_A_BYTES = 128 * 16 * SF_CH;              // dense: row r at r * 64
+constexpr int SFC_BYTES = SFC_A_BYTES + 256 * 16 * SF_CH;  // + 256 B rows
+constexpr int SF_TILE_ATOM_BYTES = SFA_BYTES + SFB_BYTES;  // a K tile's atoms (A then B)
+static_assert(SF_CH * SF_TILE_ATOM_BYTES == SFC_BYTES, "in-place rearrangement");
+constexpr uint32_t P_SF_COL0 = 256;
+static_assert(P_SF_COL0 + PSTAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM columns (pair)");
+static_assert(SF_CH == 2 && SF_BUFS % 2 == 0, "loader warps 4-5 take even chunks, 6-7 odd ones");
+
+struct __align__(1024) PairSmem {
+    uint8_t a[PSTAGES][P_A_TILE];
+    uint8_t b[PSTAGES][P_B_TILE];
+    uint8_t sfc[SF_BUFS][SFC_BYTES];
+    uint64_t full[PSTAGES];    // leader's copy used: code tiles of both CTAs
+    uint64_t empty[PSTAGES];   // both CTAs: the leader's commit after the stage's MMAs
+    uint64_t sff[SF_BUFS];      // this CTA's scale chunk has landed
+    uint64_t sfr[SF_BUFS];      // leader's copy used: atoms of both CTAs written
+    uint64_t sf_empty[SF_BUFS]; // both CTAs: the leader's commit after a chunk's last MMAs
+    uint64_t tmem_full;        // both CTAs: the leader's commit after the last MMA
+    uint32_t tmem_base;
+};
+static_assert(8 * EPI_WARP_BYTES <= PSTAGES * (P_A_TILE + P_B_TILE), "epilogue staging exceeds the ring (pair)");
+
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                       const __grid_constant__ CUtensorMap tmC, const float* __restrict__ ga,
+                       const float* __restrict__ gb, int64_t M, int64_t N, int64_t K, int c_f32, uint32_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    PairSmem& sm = *reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int n_tiles = (int)((N + 255) / 256);
+    const int pair = blockIdx.x >> 1;
+    const int mt = pair / n_tiles, nt = pair - mt * n_tiles;
+    const int64_t m0 = (int64_t)mt * 256 + 128 * rank;    // this CTA's A rows and accumulator rows
+    const int64_t n0 = (int64_t)nt * 256;                 // the tile's first output column
+    const int64_t nb0 = n0 + 128 * rank;                  // this CTA's B rows
+    const int KT = (int)(K / BK);
+    const int NC = (KT + SF_CH - 1) / SF_CH;              // scale chunks
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PSTAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < SF_BUFS; ++b) {
+            mbar_init(&sm.sff[b], 1);
+            mbar_init(&sm.sfr[b], 2 * SF_CH);     // SF_CH loader warps in each CTA
+            mbar_init(&sm.sf_empty[b], 1);
+        }
+        mbar_init(&sm.tmem_full, 1);
+        fence_barrier_init();
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    pdl_wait();
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- code-tile TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmC);
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % PSTAGES;
+                const uint32_t ph = (uint32_t)(kt / PSTAGES) & 1u;
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
+                if (leader) mbar_arrive_expect_tx(&sm.full[s], 2 * (P_A_TILE + P_B_TILE));
+                tma_load_2d_pair(sm.a[s], &tmA, &sm.full[s], kt * BKB, (int32_t)m0);
+                tma_load_2d_pair(sm.b[s], &tmB, &sm.full[s], kt * BKB, (int32_t)nb0);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- scale-chunk TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmSA);
+            tma_prefetch_desc(&tmSB);
+            for (int c = 0; c < NC; ++c) {
+                const int b = c % SF_BUFS;
+                const uint32_t ph = (uint32_t)(c / SF_BUFS) & 1u;
+                if (!wait_or_timeout(&sm.sf_empty[b], ph ^ 1u, err)) break;
+                mbar_arrive_expect_tx(&sm.sff[b], SFC_BYTES);
+                tma_load_2d(sm.sfc[b], &tmSA, &sm.sff[b], c * 16 * SF_CH, (int32_t)m0);
+                tma_load_2d(sm.sfc[b] + SFC_A_BYTES, &tmSB, &sm.sff[b], c * 16 * SF_CH, (int32_t)n0);
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------------------------------------------------- MMA issuer (leader)
+        if (leader && elect_one()) {
+            const uint32_t idesc = idesc_mxf4nvf4(256, 256);
+            bool ok = true;
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % PSTAGES;
+                const uint32_t ph = (uint32_t)(kt / PSTAGES) & 1u;
+                const int c = kt / SF_CH, t = kt - c * SF_CH, b = c % SF_BUFS;
+                if (!wait_or_timeout(&sm.full[s], ph, err) ||
+                    (t == 0 && !wait_or_timeout(&sm.sfr[b], (uint32_t)(c / SF_BUFS) & 1u, err))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t col_a = tmem + P_SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
+                const uint32_t col_b = col_a + SFA_COLS;
+                const uint8_t* at = sm.sfc[b] + t * SF_TILE_ATOM_BYTES;
+#pragma unroll
+                for (int j = 0; j < MMAS_PER_TILE; ++j) {
+                    tmem_cp_32x128b_warpx4_pair(col_a + 4 * j,
+                                                smem_desc(smem_u32(at + j * ATOM_BYTES), 0, 128, kLayoutNone));
+                    tmem_cp_32x128b_warpx4_pair(
+                        col_b + 8 * j, smem_desc(smem_u32(at + SFA_BYTES + 2 * j * ATOM_BYTES), 0, 128, kLayoutNone));
+                    tmem_cp_32x128b_warpx4_pair(
+                        col_b + 8 * j + 4,
+                        smem_desc(smem_u32(at + SFA_BYTES + (2 * j + 1) * ATOM_BYTES), 0, 128, kLayoutNone));
+                }
+                const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
+#pragma unroll
+                for (int j = 0; j < MMAS_PER_TILE; ++j)
+                    mma_mxf4nvf4_pair(tmem, desc_kmajor_sw128(a_base + 32 * j), desc_kmajor_sw128(b_base + 32 * j),
+                                      idesc, col_a + 4 * j, col_b + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                mma_commit_pair_multicast(&sm.empty[s], 0x3);
+                if (t == SF_CH - 1 || kt == KT - 1) mma_commit_pair_multicast(&sm.sf_empty[b], 0x3);
+            }
+            if (ok) mma_commit_pair_multicast(&sm.tmem_full, 0x3);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------- scale loaders
+        // Warps 4-5 take the even chunks, 6-7 the odd ones; warp 4 + 2 g + t
+        // handles K tile t of its chunks: lane l reads the 16 scale bytes of A
+        // rows l + 32 i and B rows l + 32 i for that K tile; once both warps of
+        // the pair have read (the barrier reduction), each writes its K
+        // tile's atoms over the chunk.
+        const int g = (warp - 4) >> 1, t = (warp - 4) & 1;
+        const uint32_t leader_sfr0 = map_to_rank(smem_u32(&sm.sfr[0]), 0);
+        for (int c = g; c < NC; c += 2) {
+            const int b = c % SF_BUFS;
+            const uint32_t ph = (uint32_t)(c / SF_BUFS) & 1u;
+            const bool landed = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.sff[b], ph, err));
+            uint4 ca[4], cb[8];
+            const uint8_t* dense = sm.sfc[b];
+            if (landed) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    ca[i] = *reinterpret_cast<const uint4*>(dense + (lane + 32 * i) * (16 * SF_CH) + 16 * t);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    cb[i] = *reinterpret_cast<const uint4*>(dense + SFC_A_BYTES + (lane + 32 * i) * (16 * SF_CH) +
+                                                            16 * t);
+            }
+            if (!bar_red_and(1 + g, 2 * 32, landed)) break;
+            uint8_t* at = sm.sfc[b] + t * SF_TILE_ATOM_BYTES;
+            write_atoms(at, at + SFA_BYTES, ca, cb, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_sfr0 + 8u * (uint32_t)b);
+        }
+    }
+
+    // -------------------------------------------------------------- epilogue
+    // As in the single-CTA kernel, on this CTA's 128 accumulator rows.
+    __syncwarp();
+    {
+        const int q = warp & 3, half = warp >> 2;
+        const int64_t row0 = m0 + 32 * q, col0 = n0 + 128 * half;
+        const bool ok = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.tmem_full, 0, err));
+        if (ok && row0 < M && col0 < N) {
+            tc_fence_after();
+            const float gab = __fmul_rn(__ldg(ga), __ldg(gb));
+            uint8_t* stage = &sm.a[0][0] + warp * EPI_WARP_BYTES;
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half + 32 * c), r[c]);
+            tmem_ld_wait();
+            stage_and_store(stage, r, gab, c_f32, lane, &tmC, col0, row0, N);
+        }
+    }
+
+    // both CTAs done: no MMA, copy, TMEM read or remote arrival outstanding
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+}
+
+int pair_smem_bytes() { return (int)sizeof(PairSmem) + 1024; }
 
 
 }  // namespace
@@ -365,12 +597,18 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(gemm_nvfp4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pair_smem_bytes());
+        if (e != cudaSuccess) return e;
         configured[dev] = 1;
     }
+    // CTA pairs (256 x 256 tiles) need the scale rows by TMA and pay off once
+    // M spans more than one 128-row tile.
+    const bool use_pair = tma_sf && m > BM;
     CUtensorMap ta, tb;
     e = make_tmap_u8_2d(&ta, aq, (uint64_t)m, (uint64_t)(k / 2), (uint64_t)(k / 2), BM, BKB);
     if (e != cudaSuccess) return e;
-    e = make_tmap_u8_2d(&tb, bq, (uint64_t)n, (uint64_t)(k / 2), (uint64_t)(k / 2), BN, BKB);
+    e = make_tmap_u8_2d(&tb, bq, (uint64_t)n, (uint64_t)(k / 2), (uint64_t)(k / 2), use_pair ? 128 : BN, BKB);
     if (e != cudaSuccess) return e;
     CUtensorMap tsa, tsb;
     std::memset(&tsa, 0, sizeof(tsa));
@@ -391,6 +629,17 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
         e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)n, (uint64_t)n * 2, 32, 64,
                          CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
+    if (use_pair) {
+        e = make_tmap_2d(&tsa, as, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)m, (uint64_t)(k / 16), (uint64_t)(k / 16),
+                         128, 16 * SF_CH, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (e != cudaSuccess) return e;
+        e = make_tmap_2d(&tsb, bs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n, (uint64_t)(k / 16), (uint64_t)(k / 16),
+                         256, 16 * SF_CH, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (e != cudaSuccess) return e;
+        const int64_t pairs = ((m + 255) / 256) * ((n + 255) / 256);
+        return launch_pdl(gemm_nvfp4_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS), pair_smem_bytes(),
+                          st, ta, tb, tsa, tsb, tc, ag, bg, m, n, k, c_f32, err);
+    }
     const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
     return launch_pdl(tma_sf ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>, dim3((unsigned)grid),
                       dim3(NUM_THREADS), smem_bytes(), st, ta, tb, tsa, tsb, tc, (const uint8_t*)as, ag,

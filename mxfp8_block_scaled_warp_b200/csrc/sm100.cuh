@@ -203,6 +203,38 @@ __device__ __forceinline__ void mma_commit_pair_multicast(uint64_t* bar, uint16_
                  :: "r"(smem_u32(bar)), "h"(cta_mask) : "memory");
 }
 
+// Block-scaled NVFP4 MMA issued by the leader for the pair (operand and
+// scale addresses are the same offsets in both CTAs).
+__device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Shared -> TMEM scale copy for the pair: each CTA's own shared memory at
+// `sdesc` into its own TMEM at `taddr` (32 rows x 128 bits, replicated into
+// the four lane quadrants).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Named-barrier AND-reduction over `nthreads` threads (whole warps) on
+// barrier `id`: every participant gets whether all passed `pred`.
+__device__ __forceinline__ bool bar_red_and(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred P, Q;\n\t"
+        "setp.ne.u32 P, %3, 0;\n\t"
+        "bar.red.and.pred Q, %1, %2, P;\n\t"
+        "selp.u32 %0, 1, 0, Q;\n\t}"
+        : "=r"(r) : "r"(id), "r"(nthreads), "r"((uint32_t)pred) : "memory");
+    return r != 0;
+}
+
 // ----------------------------------------------------------------- packed fp32x2
 
 __device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {

@@ -34,10 +34,12 @@ def pack(codes: np.ndarray) -> np.ndarray:
     return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
 
 
-# K a multiple of 256 takes the path whose scale rows arrive by TMA (rows of
-# K/16 bytes on 16-byte boundaries); other K read the scale rows directly.
+# K a multiple of 256 takes the paths whose scale rows arrive by TMA (rows of
+# K/16 bytes on 16-byte boundaries), with CTA pairs (256 x 256 tiles) once M
+# exceeds 128; other K read the scale rows directly.
 @pytest.mark.parametrize("m,n,k", [(128, 256, 256), (200, 272, 384), (1, 16, 128), (300, 512, 1024),
-                                   (257, 256, 640), (160, 256, 896), (384, 512, 1152)])
+                                   (257, 256, 640), (160, 256, 896), (384, 512, 1152), (129, 16, 256),
+                                   (520, 336, 512), (640, 1024, 2048)])
 def test_nvfp4_gemm_random(fpq, orc, m, n, k):
     a = rand((m, k), 700 + m, std=0.02, outliers=0.01)
     b = rand((n, k), 800 + n, std=0.02, outliers=0.01)
@@ -111,3 +113,22 @@ def test_nvfp4_gemm_full_size_sampled(fpq, orc):
     check(got, ref, orc, "nvfp4 full size", rms=float(np.sqrt(np.mean(ref ** 2))))
     assert fpq.fpq_get_device_error() == 0
 
+
+
+def test_nvfp4_gemm_repeatable(fpq):
+    """Repeated launches on the same inputs give bit-identical results (the
+    CTA-pair kernel hands scale atoms between CTAs through barriers; a
+    missing ordering would show up as run-to-run differences)."""
+    rng = np.random.default_rng(11)
+    m, n, k = 2048, 1024, 4096
+    aq = dev(rng.integers(0, 256, (m, k // 2), dtype=np.uint8))
+    bq = dev(rng.integers(0, 256, (n, k // 2), dtype=np.uint8))
+    # E4M3 scales in [2^-3, 2^3): exponent fields 4..9, random mantissas
+    sa = dev((rng.integers(4, 10, (m, k // 16)) << 3 | rng.integers(0, 8, (m, k // 16))).astype(np.uint8))
+    sb = dev((rng.integers(4, 10, (n, k // 16)) << 3 | rng.integers(0, 8, (n, k // 16))).astype(np.uint8))
+    one = dev(np.ones(1, np.float32))
+    first = fpq.scaled_gemm_nvfp4(aq, sa, one, bq, sb, one, out_dtype=torch.float32)
+    for _ in range(8):
+        again = fpq.scaled_gemm_nvfp4(aq, sa, one, bq, sb, one, out_dtype=torch.float32)
+        assert torch.equal(again, first)
+    assert fpq.fpq_get_device_error() == 0
