@@ -172,146 +172,62 @@ quant_fp8_1x128_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
 
 // ----------------------------------------------------------------- FP8 128x128
 
-// Persistent kernel: each CTA walks the 128x128 blocks b = blockIdx.x,
-// blockIdx.x + gridDim.x, ... through a QB_STAGES-deep shared-memory ring.
-// One thread issues a single 2-D TMA load per block (128 rows x 256 B, no
-// swizzle, no multicast) completing on the stage's mbarrier, so the next
-// blocks stream in while the CTA reduces and quantizes the current one.
-// 256 threads; thread t owns the 8 chunks (16 B) c = t + 256 i of the block:
-// row c / 16, columns 8 (c % 16).  Rows past the end of a batch item (a short
-// last block row) are loaded but excluded from the amax and not stored.
-constexpr int QB_STAGES = 2;
-constexpr int QB_BLOCK_BYTES = 128 * 128 * 2;
+// One CTA of QB_THREADS threads per 128x128 block (grid = all blocks of all
+// batch items).  Thread t owns the QB_CHUNKS 16-byte chunks c = t +
+// QB_THREADS i of the block (row c / 16, columns 8 (c % 16)) and issues all
+// their loads before using any.  Few chunks per thread keep many warps
+// resident, which hides the latency of the encoder's dependent steps.  One
+// barrier: each warp publishes its absmax, then every thread combines them
+// and derives the same scale.  Rows past the end of a batch item (a short
+// last block row) read as zero and are not stored.
+constexpr int QB_THREADS = 512;
+constexpr int QB_CHUNKS = 128 * 16 / QB_THREADS;
+constexpr int QB_WARPS = QB_THREADS / 32;
 
-__device__ __forceinline__ void tma_load_block(void* dst, const CUtensorMap* map, int32_t col, int32_t row,
-                                               uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];"
-        :: "r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(reinterpret_cast<uint64_t>(map)),
-           "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(col), "r"(row)
-        : "memory");
-}
-
-__device__ __forceinline__ void mbar_init_cta(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;"
-                 :: "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                 :: "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(bytes) : "memory");
-}
-
-// Wait for a phase; gives up (returns false) after ~4 s of wall time.
-__device__ __forceinline__ bool mbar_wait_phase(uint64_t* bar, uint32_t parity) {
-    const uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        uint32_t ok;
-        asm volatile("{\n\t.reg .pred P;\n\tmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
-                     "selp.b32 %0, 1, 0, P;\n\t}" : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
-        if (ok) return true;
-        uint64_t now;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
-        if (it == 0) t0 = now;
-        else if (now - t0 > 4000000000ull) return false;
-    }
-}
-
-struct QbBlock {
-    int64_t b, bi, bj, rmax;
-};
-
-__device__ __forceinline__ QbBlock qb_block(int64_t idx, int64_t rows, int64_t nbr, int64_t nbc) {
-    QbBlock k;
-    k.bj = idx % nbc;
-    const int64_t t = idx / nbc;
-    k.bi = t % nbr;
-    k.b = t / nbr;
-    k.rmax = min64(128, rows - k.bi * 128);
-    return k;
-}
-
-// Issue the load of block `idx` into stage buffer `dst` (one thread).
-__device__ __forceinline__ void qb_issue(const CUtensorMap* map, int64_t idx, int64_t rows, int64_t nbr, int64_t nbc,
-                                         uint8_t* dst, uint64_t* bar) {
-    const QbBlock k = qb_block(idx, rows, nbr, nbc);
-    mbar_expect_tx(bar, (uint32_t)QB_BLOCK_BYTES);
-    tma_load_block(dst, map, (int32_t)(k.bj * 128), (int32_t)(k.b * rows + k.bi * 128), bar);
-}
-
-__global__ void __launch_bounds__(256, 2)
-quant_fp8_128x128_kernel(const __grid_constant__ CUtensorMap tmX, uint8_t* __restrict__ q, float* __restrict__ s,
-                         int64_t batch, int64_t rows, int64_t cols, uint32_t* err) {
+__global__ void __launch_bounds__(QB_THREADS, 2048 / QB_THREADS)
+quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s,
+                         int64_t rows, int64_t cols) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
-    extern __shared__ __align__(128) uint8_t qb_smem[];
-    __shared__ __align__(8) uint64_t full[QB_STAGES];
-    __shared__ uint32_t red[8];
-    __shared__ float sc_sh;
+    __shared__ uint32_t red[QB_WARPS];
     const int64_t nbr = (rows + 127) / 128, nbc = cols / 128;
-    const int64_t nblocks = batch * nbr * nbc;
+    const int64_t idx = blockIdx.x;
+    const int64_t bj = idx % nbc, t2 = idx / nbc, bi = t2 % nbr, b = t2 / nbr;
+    const int rmax = (int)min64(128, rows - bi * 128);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < QB_STAGES; ++i) mbar_init_cta(&full[i], 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const int64_t row0 = b * rows + bi * 128;
+    const uint8_t* xb = x + (row0 * cols + bj * 128) * 2;
+    uint4 v[QB_CHUNKS];
+#pragma unroll
+    for (int i = 0; i < QB_CHUNKS; ++i) {
+        const int c = threadIdx.x + QB_THREADS * i, r = c >> 4;
+        v[i] = r < rmax ? ld_stream(xb + (int64_t)r * cols * 2 + (c & 15) * 16) : make_uint4(0, 0, 0, 0);
     }
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < QB_CHUNKS; ++i)
+        m = max2(m, max2(max2(abs2(v[i].x), abs2(v[i].y)), max2(abs2(v[i].z), abs2(v[i].w))));
+    m = group_max<32>(hmax2(m));
+    if (lane == 0) red[warp] = m;
     __syncthreads();
-    if (threadIdx.x == 0)
-        for (int i = 0; i < QB_STAGES; ++i) {
-            const int64_t idx = blockIdx.x + (int64_t)i * gridDim.x;
-            if (idx < nblocks) qb_issue(&tmX, idx, rows, nbr, nbc, qb_smem + i * QB_BLOCK_BYTES, &full[i]);
-        }
-    int it = 0;
-    for (int64_t idx = blockIdx.x; idx < nblocks; idx += gridDim.x, ++it) {
-        const int st = it % QB_STAGES;
-        const uint32_t parity = (uint32_t)(it / QB_STAGES) & 1u;
-        const uint8_t* buf = qb_smem + st * QB_BLOCK_BYTES;
-        const QbBlock k = qb_block(idx, rows, nbr, nbc);
-        if (!mbar_wait_phase(&full[st], parity)) {
-            if (threadIdx.x == 0) raise_device_error(err, FPQ_ERR_DEVICE_TIMEOUT);
-            return;    // every thread of the CTA times out on the same phase
-        }
-        uint4 v[8];
-        uint32_t m = 0;
+    uint32_t a = red[0];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int c = threadIdx.x + 256 * i, r = c >> 4;
-            v[i] = r < k.rmax ? *reinterpret_cast<const uint4*>(buf + r * 256 + (c & 15) * 16) : make_uint4(0, 0, 0, 0);
-            m = max2(m, max2(max2(abs2(v[i].x), abs2(v[i].y)), max2(abs2(v[i].z), abs2(v[i].w))));
-        }
-        // every thread has its data in registers: the stage can be refilled
-        __syncthreads();
-        if (threadIdx.x == 0 && idx + (int64_t)QB_STAGES * gridDim.x < nblocks)
-            qb_issue(&tmX, idx + (int64_t)QB_STAGES * gridDim.x, rows, nbr, nbc, qb_smem + st * QB_BLOCK_BYTES,
-                     &full[st]);
-        m = group_max<32>(hmax2(m));
-        if (lane == 0) red[warp] = m;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t a = red[0];
-            for (int w = 1; w < 8; ++w) a = max(a, red[w]);
-            const float sc = fp32_scale(a);
-            sc_sh = sc;
-            s[(k.b * nbr + k.bi) * nbc + k.bj] = sc;
-        }
-        __syncthreads();
-        const float sc = sc_sh;
-        const bool fast = reciprocal_ok(sc);
-        const QuotientBracket br = quotient_bracket(fast ? sc : 1.0f);
-        uint8_t* qb = q + (k.b * rows + k.bi * 128) * cols + k.bj * 128;
+    for (int w = 1; w < QB_WARPS; ++w) a = max(a, red[w]);
+    const float sc = fp32_scale(a);
+    if (threadIdx.x == 0) s[idx] = sc;
+    const bool fast = reciprocal_ok(sc);
+    const QuotientBracket br = quotient_bracket(fast ? sc : 1.0f);
+    uint8_t* qb = q + row0 * cols + bj * 128;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int c = threadIdx.x + 256 * i, r = c >> 4, c8 = (c & 15) * 8;
-            if (r < k.rmax) {
-                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-                uint32_t e[4];
+    for (int i = 0; i < QB_CHUNKS; ++i) {
+        const int c = threadIdx.x + QB_THREADS * i, r = c >> 4, c8 = (c & 15) * 8;
+        if (r < rmax) {
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            uint32_t e[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    e[j] = fast ? e4m3x2_of_quotients(bf16_lo(w[j]), bf16_hi(w[j]), br)
-                                : f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[j]), sc), __fdiv_rn(bf16_hi(w[j]), sc));
-                st_v2(qb + r * cols + c8, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
-            }
+            for (int j = 0; j < 4; ++j)
+                e[j] = fast ? e4m3x2_of_quotients(bf16_lo(w[j]), bf16_hi(w[j]), br)
+                            : f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[j]), sc), __fdiv_rn(bf16_hi(w[j]), sc));
+            st_v2(qb + (int64_t)r * cols + c8, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
         }
     }
 }
@@ -611,15 +527,8 @@ cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows,
         break;
     case FPQ_FP8_128x128: {
         const int64_t nblocks = batch * ((rows + 127) / 128) * (cols / 128);
-        const int smem = QB_STAGES * QB_BLOCK_BYTES;
-        cudaError_t e = cudaFuncSetAttribute(quant_fp8_128x128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        CUtensorMap map;
-        e = make_tmap_2d(&map, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)(batch * rows), (uint64_t)cols,
-                         (uint64_t)cols * 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
-        if (e != cudaSuccess) return e;
-        const int grid = (int)min64(nblocks, (int64_t)sms * 2);
-        quant_fp8_128x128_kernel<<<grid, 256, smem, st>>>(map, (uint8_t*)q, (float*)scales, batch, rows, cols, err);
+        quant_fp8_128x128_kernel<<<(unsigned)nblocks, QB_THREADS, 0, st>>>((const uint8_t*)x, (uint8_t*)q,
+                                                                          (float*)scales, rows, cols);
         break;
     }
     case FPQ_NVFP4: {
