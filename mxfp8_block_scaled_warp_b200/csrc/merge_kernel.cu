@@ -13,15 +13,19 @@ namespace fpq {
 namespace {
 
 constexpr int kMaxRank = 64;
+constexpr int RPT = 8;                          // rows of the block per thread
+constexpr int MT = 16 * (128 / RPT);            // threads per CTA
+constexpr int MERGE_MIN_BLOCKS = 2;
 
-// One CTA per 128x128 block of W, 256 threads as a 16 x 16 grid: thread
-// (ty, tx) owns rows 8 ty .. 8 ty + 7 and columns 8 tx .. 8 tx + 7 of the
-// block, so each rank step j costs it two 32-byte shared loads (B column j of
-// its rows, A row j of its columns) for 64 fused multiply-adds.  The delta is
+// One CTA per 128x128 block of W, MT threads as a (128 / RPT) x 16 grid:
+// thread (ty, tx) owns rows RPT ty .. RPT ty + RPT - 1 and columns 8 tx ..
+// 8 tx + 7 of the block, so each rank step j costs it RPT / 4 + 2 16-byte
+// shared loads (B column j of its rows, A row j of its columns) for 8 RPT
+// fused multiply-adds; few rows per thread keep many warps resident.  The delta is
 // accumulated in fp32 with j ascending from zero, exactly as the definition
 // states, then merged into W and rounded to bf16; the block's amax, scale and
 // E4M3 codes follow, and optionally the fake-quantized bf16 copy.
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(MT, MERGE_MIN_BLOCKS)
 lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict__ a,
                      const uint16_t* __restrict__ b, int64_t n, int64_t k, int r, float alpha_over_r,
                      uint8_t* __restrict__ wq, float* __restrict__ ws, uint16_t* __restrict__ w_fq) {
@@ -34,22 +38,22 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     const int rmax = (int)min64(128, n - row0);
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 
-    // this thread's 8 rows x 8 columns of W (one 16-byte load per row), issued
-    // first so the HBM latency overlaps the staging and the rank-r product
-    uint4 wv[8];
+    // this thread's RPT rows x 8 columns of W (one 16-byte load per row),
+    // issued first so the HBM latency overlaps the staging and the product
+    uint4 wv[RPT];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rr = 8 * ty + i;
+    for (int i = 0; i < RPT; ++i) {
+        const int rr = RPT * ty + i;
         wv[i] = rr < rmax ? ld_stream(w + (row0 + rr) * k + col0 + 8 * tx) : make_uint4(0, 0, 0, 0);
     }
     // stage the block's B rows ([128, r] contiguous) transposed, and A's r rows
     // of 128 columns, as fp32; every 16-byte load is issued before any store
-    constexpr int kMaxChunks = 128 * kMaxRank * 2 / 16 / 256;         // 4 per operand at r = 64
+    constexpr int kMaxChunks = (128 * kMaxRank * 2 / 16 + MT - 1) / MT;   // per operand at r = 64
     const int chunks = 128 * r * 2 / 16;                               // 16-byte chunks per operand
     uint4 bc[kMaxChunks], ac[kMaxChunks];
 #pragma unroll
     for (int i = 0; i < kMaxChunks; ++i) {
-        const int c = threadIdx.x + 256 * i;
+        const int c = threadIdx.x + MT * i;
         if (c < chunks) {
             // B elements e .. e+7 of the block (row (e+h) / r, rank (e+h) % r);
             // only the block's first rmax * r elements exist
@@ -69,7 +73,7 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     }
 #pragma unroll
     for (int i = 0; i < kMaxChunks; ++i) {
-        const int c = threadIdx.x + 256 * i;
+        const int c = threadIdx.x + MT * i;
         if (c < chunks) {
             const uint32_t bw[4] = {bc[i].x, bc[i].y, bc[i].z, bc[i].w};
             const int e = 8 * c;
@@ -86,30 +90,36 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     }
     __syncthreads();
 
-    float d[8][8];
+    float d[RPT][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < RPT; ++i)
 #pragma unroll
         for (int e = 0; e < 8; ++e) d[i][e] = 0.0f;
 #pragma unroll 2
     for (int j = 0; j < r; ++j) {
-        const float4 b0 = *reinterpret_cast<const float4*>(sBt + j * 128 + 8 * ty);
-        const float4 b1 = *reinterpret_cast<const float4*>(sBt + j * 128 + 8 * ty + 4);
+        float bv[RPT];
+#pragma unroll
+        for (int i = 0; i < RPT; i += 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(sBt + j * 128 + RPT * ty + i);
+            bv[i] = b4.x;
+            if (i + 1 < RPT) bv[i + 1] = b4.y;
+            if (i + 2 < RPT) bv[i + 2] = b4.z;
+            if (i + 3 < RPT) bv[i + 3] = b4.w;
+        }
         const float4 a0 = *reinterpret_cast<const float4*>(sA + j * 128 + 8 * tx);
         const float4 a1 = *reinterpret_cast<const float4*>(sA + j * 128 + 8 * tx + 4);
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
         const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < RPT; ++i)
 #pragma unroll
             for (int e = 0; e < 8; ++e) d[i][e] = __fmaf_rn(bv[i], av[e], d[i][e]);
     }
 
     // merge, round to bf16, block amax
-    uint32_t v[8][4];
+    uint32_t v[RPT][4];
     uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < RPT; ++i) {
         const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -117,32 +127,27 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
             const float hi = __fmaf_rn(alpha_over_r, d[i][2 * e + 1], bf16_hi(ww[e]));
             v[i][e] = f32x2_to_bf16x2(lo, hi);
         }
-        if (8 * ty + i < rmax)
+        if (RPT * ty + i < rmax)
 #pragma unroll
             for (int e = 0; e < 4; ++e) m = max2(m, abs2(v[i][e]));
     }
     m = hmax2(m);
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __shared__ uint32_t red[8];
-    __shared__ float sc_sh;
+    __shared__ uint32_t red[MT / 32];
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t am = red[0];
-        for (int i = 1; i < 8; ++i) am = max(am, red[i]);
-        const float sc = am == 0 ? 1.0f : __fdiv_rn(__uint_as_float(am << 16), 448.0f);
-        sc_sh = sc;
-        ws[bi * (k / 128) + bj] = sc;
-    }
-    __syncthreads();
-    const float sc = sc_sh;
+    uint32_t am = red[0];
+#pragma unroll
+    for (int i = 1; i < MT / 32; ++i) am = max(am, red[i]);
+    const float sc = am == 0 ? 1.0f : __fdiv_rn(__uint_as_float(am << 16), 448.0f);
+    if (threadIdx.x == 0) ws[bi * (k / 128) + bj] = sc;
     const bool fast = reciprocal_ok(sc);
     const QuotientBracket br = quotient_bracket(fast ? sc : 1.0f);
 
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rr = 8 * ty + i;
+    for (int i = 0; i < RPT; ++i) {
+        const int rr = RPT * ty + i;
         if (rr < rmax) {
             uint32_t e[4];
 #pragma unroll
@@ -177,7 +182,7 @@ cudaError_t launch_lora_merge_fakequant(const void* w, const void* a, const void
         if (e != cudaSuccess) return e;
     }
     dim3 grid((unsigned)(k / 128), (unsigned)((n + 127) / 128));
-    lora_merge_fq_kernel<<<grid, 256, smem, st>>>((const uint16_t*)w, (const uint16_t*)a, (const uint16_t*)b,
+    lora_merge_fq_kernel<<<grid, MT, smem, st>>>((const uint16_t*)w, (const uint16_t*)a, (const uint16_t*)b,
                                                   n, k, r, alpha_over_r, (uint8_t*)wq, ws, (uint16_t*)w_fq);
     return cudaGetLastError();
 }

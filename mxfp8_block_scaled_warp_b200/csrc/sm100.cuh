@@ -105,13 +105,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
-// 2-D tile prefetch global -> L2 (no shared-memory destination, no
-// completion to wait for).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
-}
-
 // 2-D tile store shared -> global (bulk-group completion).  Parts of the box
 // outside the tensor are not written.  The writing threads must have made
 // their shared-memory stores visible to the async proxy first
