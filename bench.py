@@ -110,6 +110,7 @@ class Step:
     dominant = ""
     unit = "TFLOP/s"           # the rate `value` is reported in: flops (GEMM steps) or bytes
     dtype = "e4m3xe4m3->f32 (bf16 in/out)"
+    tensor_ratio = 2.0         # the GEMM's dense tensor peak / the measured bf16 peak (nominal 4.5 / 2.25)
 
     @property
     def work(self) -> float:
@@ -361,8 +362,67 @@ class MoePrequant(Step):
         return hb, db
 
 
+class Nvfp4Gemm(Step):
+    """The fine-grained GEMM shape in NVFP4: both operands quantized on the
+    GPU (packed E2M1, E4M3 scale per 16, fp32 tensor scale) and multiplied
+    on the tensor cores (kind::mxf4nvf4, CTA pairs)."""
+    name = "nvfp4_gemm"
+    dominant = "gemm_nvfp4"
+    dtype = "e2m1xe2m1->f32 (bf16 in/out)"
+    tensor_ratio = 4.0         # dense fp4 / bf16, nominal 9 / 2.25
+
+    def __init__(self, fpq, dev, m=4096, n=2048, k=7168):
+        self.f = fpq
+        self.m, self.n, self.k = m, n, k
+        wl = workloads.ds_fp8_gemm(m, n, k)
+        self.a_host, self.b_host = wl["a"].pin_memory(), wl["b"].pin_memory()
+        self.a, self.b = self.a_host.to(dev), self.b_host.to(dev)
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.qa, self.sa = torch.empty((m, k // 2), **u8), torch.empty((m, k // 16), **u8)
+        self.qb, self.sb = torch.empty((n, k // 2), **u8), torch.empty((n, k // 16), **u8)
+        self.ga = torch.empty((1,), dtype=torch.float32, device=dev)
+        self.gb = torch.empty((1,), dtype=torch.float32, device=dev)
+        wsb = (max(1, fpq.fpq_quantize_workspace_bytes(fpq.NVFP4, 1)) + 15) // 16 * 16
+        self.wsa, self.wsb = torch.empty((wsb,), **u8), torch.empty((wsb,), **u8)
+        self.c = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        self.c_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
+        self.flops = 2.0 * m * n * k
+        # algorithmic bytes: bf16 read once, codes and scales written once
+        self.qa_bytes = m * k * (2 + 0.5 + 1 / 16) + 4
+        self.qb_bytes = n * k * (2 + 0.5 + 1 / 16) + 4
+        self.quant_bytes = self.qa_bytes + self.qb_bytes
+        self.launches = 3      # two quantize kernels (each after a workspace memset) and the GEMM
+        self.config = {"workload": "nvfp4_gemm: A bf16 4096x7168 N(0,1) and B bf16 2048x7168 N(0,0.02) -> packed "
+                                   "E2M1 with E4M3 scale per 16 and fp32 tensor scale; C = gA gB A B^T fp32 "
+                                   "accumulate, bf16 out",
+                       "m": m, "n": n, "k": k, "l2": "flushed before every step (256 MiB write)"}
+
+    def kernels(self):
+        f = self.f
+        return [
+            ("quant_nvfp4_a", lambda: f.fpq_quantize_block(f.NVFP4, self.a, 1, self.m, self.k, self.qa, self.sa,
+                                                           self.ga, self.wsa)),
+            ("quant_nvfp4_b", lambda: f.fpq_quantize_block(f.NVFP4, self.b, 1, self.n, self.k, self.qb, self.sb,
+                                                           self.gb, self.wsb)),
+            ("gemm_nvfp4", lambda: f.fpq_scaled_gemm_nvfp4(self.qa, self.sa, self.ga, self.qb, self.sb, self.gb,
+                                                           self.m, self.n, self.k, self.c, f.OUT_BF16)),
+        ]
+
+    def kernel_work(self):
+        return {"quant_nvfp4_a": ("GB/s", self.qa_bytes), "quant_nvfp4_b": ("GB/s", self.qb_bytes),
+                "gemm_nvfp4": ("TFLOP/s", self.flops)}
+
+    def e2e_step(self, stream):
+        self.a.copy_(self.a_host, non_blocking=True)
+        self.b.copy_(self.b_host, non_blocking=True)
+        for _, fn in self.kernels():
+            fn()
+        self.c_host.copy_(self.c, non_blocking=True)
+        return self.a_host.numel() * 2 + self.b_host.numel() * 2, self.c.numel() * 2
+
+
 STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": QatForward,
-         "moe_prequant": MoePrequant}
+         "moe_prequant": MoePrequant, "nvfp4_gemm": Nvfp4Gemm}
 
 
 # ------------------------------------------------------------------ traffic from committed ncu summaries
@@ -370,7 +430,8 @@ STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": Qat
 def _source_hash(kernel: str) -> str | None:
     src = {"gemm_fp8_f32scale": "gemm_fp8_f32scale.cu", "gemm_grouped_mxfp8": "gemm_mxfp8.cu",
            "gemm_mxfp8": "gemm_mxfp8.cu", "quant_fp8_1x128": "quant_kernels.cu",
-           "quant_mxfp8": "quant_kernels.cu", "lora_merge_fq": "merge_kernel.cu"}.get(kernel)
+           "quant_mxfp8": "quant_kernels.cu", "lora_merge_fq": "merge_kernel.cu",
+           "gemm_nvfp4": "gemm_nvfp4.cu"}.get(kernel)
     if not src:
         return None
     with open(os.path.join(ROOT, "mxfp8_block_scaled_warp_b200", "csrc", src), "rb") as f:
@@ -401,6 +462,8 @@ def cpu_baseline(workload: str, budget_s: float = 12.0):
     oracle.build()
     if workload == "moe_prequant":
         return _cpu_baseline_prequant(oracle, budget_s)
+    if workload == "nvfp4_gemm":
+        return _cpu_baseline_nvfp4_gemm(oracle, budget_s)
     if workload != "ds_fp8_gemm":
         return None
     m, n, k = 4096, 2048, 7168
@@ -433,6 +496,36 @@ def cpu_baseline(workload: str, budget_s: float = 12.0):
             "sample": f"1x128 quantize of {rows_a} rows and 128x128 quantize of 256 rows of the 7168-wide "
                       f"operands, {count} fp64 GEMM entries (K=7168); extrapolated to the full 4096x2048x7168 "
                       f"step ({step_s:.1f} s per step on one core)"}
+
+
+def _cpu_baseline_nvfp4_gemm(oracle, budget_s: float):
+    """The oracle's NVFP4 quantizer on leading rows of both operands and its
+    fp64 GEMM entries (K = 7168), extrapolated to the whole 4096x2048x7168
+    step (both quantizes and every entry)."""
+    m, n, k = 4096, 2048, 7168
+    wl = workloads.ds_fp8_gemm(m, n, k)
+    a, b = workloads.as_u16(wl["a"]), workloads.as_u16(wl["b"])
+    rows = 64
+    t0 = time.perf_counter()
+    qa, sa, ga = oracle.quant_nvfp4(a[:rows])
+    qb, sb, gb = oracle.quant_nvfp4(b[:rows])
+    t_q = (time.perf_counter() - t0) / (2 * rows * k)
+    probe = 64
+    rr, cc = np.arange(probe) % rows, (np.arange(probe) * 7) % rows
+    t0 = time.perf_counter()
+    oracle.gemm_entries(3, qa, sa, 3, qb, sb, rr, cc, ag=ga, bg=gb)
+    per = (time.perf_counter() - t0) / probe
+    count = int(max(probe, min(200000, (budget_s - t_q * 2 * rows * k) / max(per, 1e-9))))
+    rng = np.random.default_rng(0)
+    rr, cc = rng.integers(0, rows, count), rng.integers(0, rows, count)
+    t0 = time.perf_counter()
+    oracle.gemm_entries(3, qa, sa, 3, qb, sb, rr, cc, ag=ga, bg=gb)
+    per = (time.perf_counter() - t0) / count
+    step_s = t_q * (m + n) * k + per * m * n
+    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "work": 2.0 * m * n * k, "cores": 1,
+            "kind": "oracle",
+            "sample": f"NVFP4 quantize of {rows} rows of each 7168-wide operand, {count} fp64 GEMM entries "
+                      f"(K=7168); extrapolated to the full 4096x2048x7168 step ({step_s:.1f} s per step on one core)"}
 
 
 def _cpu_baseline_prequant(oracle, budget_s: float):
@@ -640,12 +733,13 @@ def main():
 
     peaks = _peaks()
     fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
+    tensor_peak = step.tensor_ratio * peaks["bf16_tflops"]
     kernels_out = {}
     for n in names:
         unit, work = step.kernel_work()[n]
         ms = statistics.mean(per_kernel[n])
         ach = work / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
-        pk = peaks["hbm_gbs"] if unit == "GB/s" else fp8_peak_burst
+        pk = peaks["hbm_gbs"] if unit == "GB/s" else tensor_peak
         kernels_out[n] = {"ms": ms, "achieved": ach, "unit": unit, "frac_of_peak": ach / pk}
     dom = kernels_out[step.dominant]
     traffic = _traffic(step.dominant, step.name)
@@ -654,9 +748,11 @@ def main():
                     "unit": "GB/s", "frac": dom["achieved"] / peaks["hbm_gbs"], "traffic": traffic,
                     "peak_note": f"{peaks['source']} HBM copy bandwidth"}
     else:
-        roofline = {"kernel": step.dominant, "bound": "tensor", "achieved": dom["achieved"], "peak": fp8_peak_burst,
-                    "unit": "TFLOP/s", "frac": dom["achieved"] / fp8_peak_burst, "traffic": traffic,
-                    "peak_note": f"fp8 = 2 x {peaks['source']} cuBLAS bf16 burst ({peaks['bf16_tflops']} TFLOP/s)"}
+        kind = "fp4" if step.tensor_ratio == 4.0 else "fp8"
+        roofline = {"kernel": step.dominant, "bound": "tensor", "achieved": dom["achieved"], "peak": tensor_peak,
+                    "unit": "TFLOP/s", "frac": dom["achieved"] / tensor_peak, "traffic": traffic,
+                    "peak_note": f"{kind} = {step.tensor_ratio:g} x {peaks['source']} cuBLAS bf16 burst "
+                                 f"({peaks['bf16_tflops']} TFLOP/s; nominal dense ratio)"}
     quant_ms = sum(statistics.mean(per_kernel[n]) for n in names if not n.startswith("gemm"))
     quant_gbs = step.quant_bytes / (quant_ms * 1e-3) / 1e9
 
@@ -687,7 +783,8 @@ def main():
             "config": dict(step.config, launch="CUDA graph of the step replayed per timed step; per-kernel times from a second graph with events around each kernel"), "quantize_gbs": quant_gbs, "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"],
             "kernels": kernels_out, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.launches * args.steps, "clocks": clk.summary(),
-            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp8_tflops": fp8_peak_burst, "source": peaks["source"]}}
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp8_tflops": fp8_peak_burst, "tensor_tflops": tensor_peak,
+                      "source": peaks["source"]}}
     if rank == 0:
         print(json.dumps(line))
     if pg:

@@ -112,7 +112,9 @@ def test_mxfp8_gemm_extreme_scales(fpq, orc):
 
 # ------------------------------------------------------------------ fp32-scale (1x128 x 128x128)
 
-@pytest.mark.parametrize("m,n,k", [(128, 128, 128), (200, 144, 384), (333, 400, 1024), (1, 16, 256)])
+# ragged M and N, one and several 128 x 256 tiles
+@pytest.mark.parametrize("m,n,k", [(128, 128, 128), (200, 144, 384), (333, 400, 1024), (1, 16, 256),
+                                   (129, 16, 128), (520, 272, 768), (640, 1024, 2048)])
 def test_fp8_blockscale_gemm_random(fpq, orc, m, n, k):
     a = rand((m, k), 300 + m)
     b = rand((n, k), 400 + n, std=0.02)
@@ -150,6 +152,23 @@ def test_fp8_blockscale_gemm_one_hot_scales(fpq, orc):
     ref = orc.gemm_full(F1x128, aq, as_, F128, bq, bs)
     c = fpq.scaled_gemm(fpq.FP8_1x128, dev(aq), dev(as_), fpq.FP8_128x128, dev(bq), dev(bs), out_dtype=torch.float32)
     assert np.array_equal(c.cpu().numpy().astype(np.float64), ref)
+
+
+def test_fp8_blockscale_gemm_repeatable(fpq):
+    """Repeated launches give bit-identical C: the promotion warps and the MMA
+    thread hand the two TMEM buffers back and forth through barriers, and a
+    missing ordering would show up as run-to-run differences."""
+    rng = np.random.default_rng(12)
+    m, n, k = 2048, 1024, 4096
+    aq = dev(rng.integers(0, 0x7F, (m, k), dtype=np.uint8) | (rng.integers(0, 2, (m, k), dtype=np.uint8) << 7))
+    bq = dev(rng.integers(0, 0x7F, (n, k), dtype=np.uint8) | (rng.integers(0, 2, (n, k), dtype=np.uint8) << 7))
+    as_ = dev(rng.uniform(0.5, 2.0, (m, k // 128)).astype(np.float32))
+    bs = dev(rng.uniform(0.5, 2.0, (n // 128, k // 128)).astype(np.float32))
+    first = fpq.scaled_gemm(fpq.FP8_1x128, aq, as_, fpq.FP8_128x128, bq, bs, out_dtype=torch.float32)
+    for _ in range(8):
+        assert torch.equal(fpq.scaled_gemm(fpq.FP8_1x128, aq, as_, fpq.FP8_128x128, bq, bs, out_dtype=torch.float32),
+                           first)
+    assert fpq.fpq_get_device_error() == 0
 
 
 def _sampled_dense_check(orc, c_gpu, aq, as_, fa, bq, bs, fb, rows, cols, what):
