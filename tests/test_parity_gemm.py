@@ -154,12 +154,36 @@ def test_fp8_blockscale_gemm_one_hot_scales(fpq, orc):
     assert np.array_equal(c.cpu().numpy().astype(np.float64), ref)
 
 
+# More tiles than SMs (a second, partial wave; a ragged last row of tiles):
+# 12 entries of every 128 x 256 tile and the ragged edges against the oracle.
+@pytest.mark.parametrize("m,n,k", [(2560, 2048, 256), (3968 + 50, 2048, 384)])
+def test_fp8_blockscale_gemm_many_tiles(fpq, orc, m, n, k):
+    a = rand((m, k), 500 + m)
+    b = rand((n, k), 600 + n, std=0.02)
+    aq, as_ = orc.quant_fp8_1x128(a)
+    bq, bs = orc.quant_fp8_128x128(b)
+    c = fpq.scaled_gemm(fpq.FP8_1x128, dev(aq), dev(as_), fpq.FP8_128x128, dev(bq), dev(bs), out_dtype=torch.float32)
+    assert fpq.fpq_get_device_error() == 0
+    rng = np.random.default_rng(m)
+    rows, cols = [], []
+    for mt in range((m + 127) // 128):
+        for nt in range((n + 255) // 256):
+            rows += list(rng.integers(128 * mt, min(m, 128 * mt + 128), 12))
+            cols += list(rng.integers(256 * nt, min(n, 256 * nt + 256), 12))
+    rows += [m - 1] * 4 + list(rng.integers(0, m, 4))
+    cols += list(rng.integers(0, n, 4)) + [n - 1] * 4
+    rows, cols = np.array(rows), np.array(cols)
+    ref = orc.gemm_entries(F1x128, aq, as_, F128, bq, bs, rows, cols)
+    got = c[torch.from_numpy(rows).cuda(), torch.from_numpy(cols).cuda()]
+    check(got, ref, orc, f"fp8 blockscale {m}x{n}x{k}", rms=float(np.sqrt(np.mean(ref ** 2))))
+
+
 def test_fp8_blockscale_gemm_repeatable(fpq):
     """Repeated launches give bit-identical C: the promotion warps and the MMA
     thread hand the two TMEM buffers back and forth through barriers, and a
     missing ordering would show up as run-to-run differences."""
     rng = np.random.default_rng(12)
-    m, n, k = 2048, 1024, 4096
+    m, n, k = 4096, 1280, 4096          # 160 tiles: more than one wave
     aq = dev(rng.integers(0, 0x7F, (m, k), dtype=np.uint8) | (rng.integers(0, 2, (m, k), dtype=np.uint8) << 7))
     bq = dev(rng.integers(0, 0x7F, (n, k), dtype=np.uint8) | (rng.integers(0, 2, (n, k), dtype=np.uint8) << 7))
     as_ = dev(rng.uniform(0.5, 2.0, (m, k // 128)).astype(np.float32))
