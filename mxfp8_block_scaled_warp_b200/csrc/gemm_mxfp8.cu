@@ -101,6 +101,59 @@ __device__ __forceinline__ uint4 load_sf_group(const uint8_t* sf, int64_t row, i
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+struct TileMap {
+    int valid, g, mt, nt;
+    int32_t rb, re;     // A rows owned by the tile's group
+};
+
+// Tile t -> (group, m tile, n tile) for row tiles of bm rows, run by one warp
+// (all lanes return the same map).  Grouped (off = the offsets staged in
+// shared memory): the groups are scanned 32 at a time (tile counts,
+// inclusive prefix sum over the warp, ballot for the group holding tile t),
+// and every group is validated: offsets must rise from 0 to M.
+__device__ TileMap map_tile(int t, int bm, const int32_t* off, bool grouped, int groups, int64_t M, int n_tiles,
+                            int lane, uint32_t* err) {
+    TileMap r{0, 0, 0, 0, 0, (int32_t)M};
+    if (!grouped) {
+        r.mt = t / n_tiles;
+        r.nt = t - r.mt * n_tiles;
+        r.valid = (int64_t)r.mt * bm < M;
+        return r;
+    }
+    bool bad = off[0] != 0 || off[groups] != (int32_t)M;
+    int before = 0;                          // tiles of the groups in earlier chunks
+    for (int c0 = 0; c0 < groups; c0 += 32) {
+        const int e = c0 + lane;
+        const int32_t b0 = e < groups ? off[e] : 0, b1 = e < groups ? off[e + 1] : 0;
+        if (b1 < b0) bad = true;
+        const int tiles = b1 > b0 ? ((b1 - b0 + bm - 1) / bm) * n_tiles : 0;
+        int incl = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int lo = before + incl - tiles;
+        const unsigned hit = __ballot_sync(0xFFFFFFFFu, tiles > 0 && t >= lo && t < lo + tiles);
+        if (hit) {
+            const int src = __ffs(hit) - 1;
+            const int tt = t - __shfl_sync(0xFFFFFFFFu, lo, src);
+            r.g = c0 + src;
+            r.rb = __shfl_sync(0xFFFFFFFFu, b0, src);
+            r.re = __shfl_sync(0xFFFFFFFFu, b1, src);
+            r.mt = tt / n_tiles;
+            r.nt = tt - r.mt * n_tiles;
+            r.valid = 1;
+        }
+        before += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (__any_sync(0xFFFFFFFFu, bad)) {
+        if (blockIdx.x == 0 && lane == 0) raise_device_error(err, FPQ_ERR_DEVICE_BAD_INPUT);
+        r.valid = 0;
+    }
+    return r;
+}
+
 // grouped: offsets != nullptr.  For the dense product groups = 1 and the
 // single group spans rows [0, M).
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -134,53 +187,14 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
     __syncthreads();
     if (warp == 0) {
-        int valid = 0, g = 0, mt = 0, nt = 0;
-        int32_t rb = 0, re = (int32_t)M;
-        const int t = blockIdx.x;
-        if (offsets == nullptr) {
-            mt = t / n_tiles;
-            nt = t - mt * n_tiles;
-            valid = (int64_t)mt * BM < M;
-        } else {
-            bool bad = sm.off[0] != 0 || sm.off[groups] != (int32_t)M;
-            int before = 0;                          // tiles of the groups in earlier chunks
-            for (int c0 = 0; c0 < groups; c0 += 32) {
-                const int e = c0 + lane;
-                const int32_t b0 = e < groups ? sm.off[e] : 0, b1 = e < groups ? sm.off[e + 1] : 0;
-                if (b1 < b0) bad = true;
-                const int tiles = b1 > b0 ? ((b1 - b0 + BM - 1) / BM) * n_tiles : 0;
-                int incl = tiles;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                const int lo = before + incl - tiles;
-                const unsigned hit = __ballot_sync(0xFFFFFFFFu, tiles > 0 && t >= lo && t < lo + tiles);
-                if (hit) {
-                    const int src = __ffs(hit) - 1;
-                    const int tt = t - __shfl_sync(0xFFFFFFFFu, lo, src);
-                    g = c0 + src;
-                    rb = __shfl_sync(0xFFFFFFFFu, b0, src);
-                    re = __shfl_sync(0xFFFFFFFFu, b1, src);
-                    mt = tt / n_tiles;
-                    nt = tt - mt * n_tiles;
-                    valid = 1;
-                }
-                before += __shfl_sync(0xFFFFFFFFu, incl, 31);
-            }
-            if (__any_sync(0xFFFFFFFFu, bad)) {
-                if (blockIdx.x == 0 && lane == 0) raise_device_error(err, FPQ_ERR_DEVICE_BAD_INPUT);
-                valid = 0;
-            }
-        }
+        const TileMap tm = map_tile(blockIdx.x, BM, sm.off, offsets != nullptr, groups, M, n_tiles, lane, err);
         if (lane == 0) {
-            sm.tile_valid = valid;
-            sm.group = g;
-            sm.m_tile = mt;
-            sm.n_tile = nt;
-            sm.row_begin = rb;
-            sm.row_end = re;
+            sm.tile_valid = tm.valid;
+            sm.group = tm.g;
+            sm.m_tile = tm.mt;
+            sm.n_tile = tm.nt;
+            sm.row_begin = tm.rb;
+            sm.row_end = tm.re;
         }
     }
     __syncthreads();
@@ -350,6 +364,305 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
 int smem_bytes() { return (int)sizeof(Smem) + 1024; }
 
+// ============================================================== CTA pair
+// A cluster of two CTAs computes one 256 x 256 tile with tcgen05 cta_group::2
+// (grouped: 256 rows of one group).  CTA r stages A rows a_row0 = row_begin +
+// 256 mt + 128 r and B rows n0 + 128 r of each 128-wide K tile in its own
+// shared memory and receives its 128 accumulator rows in its own TMEM; per SM
+// a K tile is 16 + 16 KB of codes instead of 16 + 32 KB, which is what bounds
+// the one-CTA kernel (the TMA feed from L2).  The leader issues the MMAs
+// (M = 256, N = 256, 4 x K = 32 per K tile, scale byte selected per MMA) and
+// the scale copies, and commits to the barriers of both CTAs.
+//
+// Scales: chunks of P_SF_CH K tiles, one TMA box of (4 P_SF_CH)-byte scale
+// rows for this CTA's 128 A rows and one for the tile's 256 B rows (every
+// output column meets this CTA's rows), two chunks in flight; loader warps
+// 4-7 rearrange a landed chunk in place into the TMEM-copy atoms of its K
+// tiles (warp 4 + i: K tiles 2i, 2i + 1) and arrive on the leader's sfr.
+//
+// Warp roles in both CTAs: warp 0 code-tile TMA producer; warp 1 scale-chunk
+// TMA producer; warp 2 TMEM allocator (leader: MMA issuer); warps 4-7 scale
+// loaders; then all eight warps run the epilogue: whole 32-row blocks inside
+// the group by TMA stores, a block crossing the group's end by masked stores.
+constexpr int P_STAGES = 6;
+constexpr int P_A_TILE = 128 * BK, P_B_TILE = 128 * BK;
+constexpr int P_SF_CH = 8;                                   // K tiles per scale chunk
+constexpr int P_SFC_A = 128 * 4 * P_SF_CH;                   // dense: A row r at r * 32
+constexpr int P_SFC_BYTES = P_SFC_A + 256 * 4 * P_SF_CH;     // + 256 B rows
+constexpr int P_TILE_ATOMS = SFA_BYTES + SFB_BYTES;          // a K tile's atoms: A, B rows 0-127, B rows 128-255
+static_assert(P_SF_CH * P_TILE_ATOMS == P_SFC_BYTES, "in-place rearrangement");
+static_assert(P_SF_CH == 8, "loader warp 4 + i takes K tiles 2i and 2i + 1 of a chunk");
+constexpr uint32_t P_SF_COL0 = 256;
+static_assert(P_SF_COL0 + P_STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM columns (pair)");
+constexpr int P_EPI_WARP_BYTES = 32 * 128 * 4;               // a warp's 32 x 128 block of C, fp32
+
+struct __align__(1024) PairSmem {
+    uint8_t a[P_STAGES][P_A_TILE];
+    uint8_t b[P_STAGES][P_B_TILE];
+    uint8_t sfc[2][P_SFC_BYTES];
+    uint64_t full[P_STAGES];    // leader's copy used: code tiles of both CTAs
+    uint64_t empty[P_STAGES];   // both CTAs: the leader's commit after the stage's MMAs
+    uint64_t sff[2];            // this CTA's scale chunk has landed
+    uint64_t sfr[2];            // leader's copy used: atoms of both CTAs written (8 warps)
+    uint64_t sf_empty[2];       // both CTAs: the leader's commit after a chunk's last MMAs
+    uint64_t tmem_full;         // both CTAs: the leader's commit after the last MMA
+    uint32_t tmem_base;
+    int32_t tile_valid;
+    int32_t group;
+    int32_t row_begin, row_end;
+    int32_t m_tile, n_tile;
+    int32_t off[kMaxGroups + 1];
+};
+static_assert(8 * P_EPI_WARP_BYTES <= P_STAGES * (P_A_TILE + P_B_TILE), "epilogue staging exceeds the ring");
+
+// Byte offset of 16-byte chunk j (0-7) of row r in a box of 128-byte rows
+// stored with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t box_off(int r, int j) { return (uint32_t)(r * 128 + 16 * (j ^ (r & 7))); }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                       const __grid_constant__ CUtensorMap tmC, const int32_t* __restrict__ offsets, int groups,
+                       int64_t M, int64_t N, int64_t K, void* __restrict__ C, int c_f32, uint32_t* err,
+                       uint64_t timeout_ns, uint32_t extra_tx) {
+    extern __shared__ uint8_t smem_raw[];
+    PairSmem& sm = *reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int n_tiles = (int)((N + BN - 1) / BN);
+    const int KT = (int)(K / BK);
+    const int NC = (KT + P_SF_CH - 1) / P_SF_CH;
+
+    if (offsets != nullptr) {
+        pdl_wait();    // the group offsets may come from the preceding grid
+        for (int i = threadIdx.x; i <= groups; i += NUM_THREADS) sm.off[i] = offsets[i];
+    }
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.sff[b], 1);
+            mbar_init(&sm.sfr[b], 8);
+            mbar_init(&sm.sf_empty[b], 1);
+        }
+        mbar_init(&sm.tmem_full, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // both CTAs of the pair map the same pair tile
+        const TileMap tm = map_tile((int)(blockIdx.x >> 1), 2 * BM, sm.off, offsets != nullptr, groups, M, n_tiles,
+                                    lane, err);
+        if (lane == 0) {
+            sm.tile_valid = tm.valid;
+            sm.group = tm.g;
+            sm.m_tile = tm.mt;
+            sm.n_tile = tm.nt;
+            sm.row_begin = tm.rb;
+            sm.row_end = tm.re;
+        }
+    }
+    __syncthreads();
+    if (!sm.tile_valid) return;      // the same decision in both CTAs
+
+    if (warp == 2) {
+        tmem_alloc_pair(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    pdl_wait();
+
+    const int64_t a_row0 = (int64_t)sm.row_begin + (int64_t)sm.m_tile * 2 * BM + 128 * (int64_t)rank;
+    const int64_t a_rows_end = sm.row_end;
+    const int64_t n0 = (int64_t)sm.n_tile * BN;
+    const int64_t bt_row0 = (int64_t)sm.group * N + n0;       // the tile's first B row (flattened)
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- code-tile TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmC);
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % P_STAGES;
+                const uint32_t ph = (uint32_t)(kt / P_STAGES) & 1u;
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err, timeout_ns)) break;
+                if (leader) mbar_arrive_expect_tx(&sm.full[s], 2 * (P_A_TILE + P_B_TILE) + extra_tx);
+                tma_load_2d_pair(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)a_row0);
+                tma_load_2d_pair(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)(bt_row0 + 128 * rank));
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- scale-chunk TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmSA);
+            tma_prefetch_desc(&tmSB);
+            for (int c = 0; c < NC; ++c) {
+                const int b = c & 1;
+                const uint32_t ph = (uint32_t)(c >> 1) & 1u;
+                if (!wait_or_timeout(&sm.sf_empty[b], ph ^ 1u, err, timeout_ns)) break;
+                mbar_arrive_expect_tx(&sm.sff[b], P_SFC_BYTES);
+                tma_load_2d(sm.sfc[b], &tmSA, &sm.sff[b], c * 4 * P_SF_CH, (int32_t)a_row0);
+                tma_load_2d(sm.sfc[b] + P_SFC_A, &tmSB, &sm.sff[b], c * 4 * P_SF_CH, (int32_t)bt_row0);
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------------------------------------------------- MMA issuer (leader)
+        if (leader && elect_one()) {
+            bool ok = true;
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % P_STAGES;
+                const uint32_t ph = (uint32_t)(kt / P_STAGES) & 1u;
+                const int c = kt / P_SF_CH, t = kt - c * P_SF_CH, b = c & 1;
+                if (!wait_or_timeout(&sm.full[s], ph, err, timeout_ns) ||
+                    (t == 0 && !wait_or_timeout(&sm.sfr[b], (uint32_t)(c >> 1) & 1u, err, timeout_ns))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sf_col = tmem + P_SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
+                const uint8_t* at = sm.sfc[b] + t * P_TILE_ATOMS;
+                tmem_cp_32x128b_warpx4_pair(sf_col + 0, smem_desc(smem_u32(at), 0, 128, kLayoutNone));
+                tmem_cp_32x128b_warpx4_pair(sf_col + 4, smem_desc(smem_u32(at + SFA_BYTES), 0, 128, kLayoutNone));
+                tmem_cp_32x128b_warpx4_pair(sf_col + 8, smem_desc(smem_u32(at + SFA_BYTES + 512), 0, 128, kLayoutNone));
+                const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
+#pragma unroll
+                for (int k = 0; k < BK / 32; ++k) {
+                    const uint32_t idesc = idesc_mxf8f6f4(2 * BM, BN, (uint32_t)k, (uint32_t)k);
+                    mma_mxf8f6f4_pair(tmem, desc_kmajor_sw128(a_base + 32 * k), desc_kmajor_sw128(b_base + 32 * k),
+                                      idesc, (sf_col + 0) | ((uint32_t)k << 30), (sf_col + 4) | ((uint32_t)k << 30),
+                                      (kt > 0 || k > 0) ? 1u : 0u);
+                }
+                mma_commit_pair_multicast(&sm.empty[s], 0x3);
+                if (t == P_SF_CH - 1 || kt == KT - 1) mma_commit_pair_multicast(&sm.sf_empty[b], 0x3);
+            }
+            if (ok) mma_commit_pair_multicast(&sm.tmem_full, 0x3);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------- scale loaders
+        // Lane l reads, for K tiles 2i and 2i + 1 of the chunk (i = warp - 4),
+        // the 8 scale bytes of A rows l + 32 q (q < 4) and B rows l + 32 q
+        // (q < 8); once all four warps have read (the barrier reduction) each
+        // writes its two K tiles' atoms: word q of lane l = row l + 32 q.
+        const int i2 = 2 * (warp - 4);
+        const uint32_t leader_sfr0 = map_to_rank(smem_u32(&sm.sfr[0]), 0);
+        for (int c = 0; c < NC; ++c) {
+            const int b = c & 1;
+            const uint32_t ph = (uint32_t)(c >> 1) & 1u;
+            const bool landed = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.sff[b], ph, err, timeout_ns));
+            uint2 ra[4], rb[8];
+            const uint8_t* dense = sm.sfc[b];
+            if (landed) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    ra[q] = *reinterpret_cast<const uint2*>(dense + (lane + 32 * q) * (4 * P_SF_CH) + 4 * i2);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    rb[q] = *reinterpret_cast<const uint2*>(dense + P_SFC_A + (lane + 32 * q) * (4 * P_SF_CH) + 4 * i2);
+            }
+            if (!bar_red_and(1, 4 * 32, landed)) break;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint8_t* at = sm.sfc[b] + (i2 + h) * P_TILE_ATOMS;
+                auto w = [&](const uint2& v) { return h ? v.y : v.x; };
+                *reinterpret_cast<uint4*>(at + lane * 16) = make_uint4(w(ra[0]), w(ra[1]), w(ra[2]), w(ra[3]));
+                *reinterpret_cast<uint4*>(at + SFA_BYTES + lane * 16) =
+                    make_uint4(w(rb[0]), w(rb[1]), w(rb[2]), w(rb[3]));
+                *reinterpret_cast<uint4*>(at + SFA_BYTES + 512 + lane * 16) =
+                    make_uint4(w(rb[4]), w(rb[5]), w(rb[6]), w(rb[7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_sfr0 + 8u * (uint32_t)b);
+        }
+    }
+
+    // -------------------------------------------------------------- epilogue
+    // All eight warps once the last MMA has completed (the operand ring is
+    // then free): warp w reads TMEM lanes 32 (w & 3) .. + 31 (this CTA's
+    // accumulator rows) and columns 128 (w >> 2) .. + 127, stages the 32 x 128
+    // block in 128-byte-swizzled boxes, then writes it with TMA stores (the
+    // unit clips rows past M and columns past N) when all 32 rows belong to
+    // the group, else row by row, skipping rows outside the group.
+    __syncwarp();
+    {
+        const int q = warp & 3, half = warp >> 2;
+        const int64_t row0 = a_row0 + 32 * q, col0 = n0 + 128 * half;
+        const bool ok = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.tmem_full, 0, err, timeout_ns));
+        if (ok && row0 < a_rows_end && col0 < N) {
+            tc_fence_after();
+            uint8_t* stage = &sm.a[0][0] + warp * P_EPI_WARP_BYTES;
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half + 32 * c), r[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (c_f32) {     // columns 32c .. 32c + 31 = box c
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(stage + c * 4096 + box_off(lane, j)) =
+                            make_uint4(r[c][4 * j], r[c][4 * j + 1], r[c][4 * j + 2], r[c][4 * j + 3]);
+                } else {         // columns 32c .. 32c + 31 = box c / 2, chunks 4 (c % 2) .. + 3
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t h[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            h[e] = f32x2_to_bf16x2(__uint_as_float(r[c][8 * j + 2 * e]),
+                                                   __uint_as_float(r[c][8 * j + 2 * e + 1]));
+                        *reinterpret_cast<uint4*>(stage + (c / 2) * 4096 + box_off(lane, 4 * (c % 2) + j)) =
+                            make_uint4(h[0], h[1], h[2], h[3]);
+                    }
+                }
+            }
+            const int boxes = c_f32 ? 4 : 2, box_cols = c_f32 ? 32 : 64;
+            if (row0 + 32 <= a_rows_end) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    for (int x = 0; x < boxes; ++x)
+                        if (col0 + x * box_cols < N)
+                            tma_store_2d(&tmC, stage + x * 4096, (int32_t)(col0 + x * box_cols), (int32_t)row0);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();     // the staging must stay valid until read
+                }
+            } else {
+                __syncwarp();
+                // a row is 16 (bf16) or 32 (fp32) 16-byte chunks: lanes take
+                // chunk lane % chunks of row rr + lane / chunks
+                const int chunks = c_f32 ? 32 : 16, rows_per = 32 / chunks, esz = c_f32 ? 4 : 2;
+                const int ch = lane % chunks, box = ch / 8, j = ch % 8;
+                for (int rr = lane / chunks; rr < 32; rr += rows_per) {
+                    const int64_t row = row0 + rr;
+                    const int64_t col = col0 + (int64_t)ch * (16 / esz);
+                    if (row < a_rows_end && col < N)
+                        st_v4(reinterpret_cast<uint8_t*>(C) + (row * N + col) * esz,
+                              *reinterpret_cast<const uint4*>(stage + box * 4096 + box_off(rr, j)));
+                }
+            }
+            __syncwarp();
+        }
+    }
+
+    // both CTAs done: no MMA, copy, TMEM read or remote arrival outstanding
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+}
+
+int pair_smem_bytes() { return (int)sizeof(PairSmem) + 1024; }
+
 // Wait limit and the stall switch for the timeout test (see the file header).
 uint64_t wait_timeout_ns() {
     const char* v = std::getenv("FPQ_WAIT_TIMEOUT_MS");
@@ -361,20 +674,47 @@ uint32_t debug_extra_tx() {
     return (v && v[0] == '1') ? 16u : 0u;
 }
 
+// CTA pairs need the scale rows on 16-byte boundaries (K a multiple of 512)
+// and pay off once M spans more than one 128-row tile.
+bool use_pair(int64_t M, int64_t K) { return K % 512 == 0 && M > BM; }
+
 cudaError_t launch(const void* aq, const void* as, const void* bq, const void* bs, const int32_t* offsets,
                    int groups, int64_t M, int64_t N, int64_t K, void* c, int c_f32, uint32_t* err,
-                   int64_t grid, cudaStream_t st) {
+                   int64_t tiles, int64_t pair_tiles, cudaStream_t st) {
+    const bool pair = use_pair(M, K);
     CUtensorMap ta, tb;
     cudaError_t e = make_tmap_u8_2d(&ta, aq, (uint64_t)M, (uint64_t)K, (uint64_t)K, BM, BK);
     if (e != cudaSuccess) return e;
-    e = make_tmap_u8_2d(&tb, bq, (uint64_t)(groups * N), (uint64_t)K, (uint64_t)K, BN, BK);
+    e = make_tmap_u8_2d(&tb, bq, (uint64_t)(groups * N), (uint64_t)K, (uint64_t)K, pair ? 128 : BN, BK);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemm_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+    if (!pair) {
+        e = cudaFuncSetAttribute(gemm_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e != cudaSuccess) return e;
+        if (tiles < 1) return cudaSuccess;
+        return launch_pdl(gemm_mxfp8_kernel, dim3((unsigned)tiles), dim3(NUM_THREADS), smem_bytes(), st, ta, tb,
+                          (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err,
+                          wait_timeout_ns(), debug_extra_tx());
+    }
+    CUtensorMap tsa, tsb, tc;
+    e = make_tmap_2d(&tsa, as, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)M, (uint64_t)(K / 32), (uint64_t)(K / 32),
+                     128, 4 * P_SF_CH, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess) return e;
-    if (grid < 1) return cudaSuccess;
-    return launch_pdl(gemm_mxfp8_kernel, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta, tb,
-                      (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err,
-                      wait_timeout_ns(), debug_extra_tx());
+    e = make_tmap_2d(&tsb, bs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(groups * N), (uint64_t)(K / 32),
+                     (uint64_t)(K / 32), 256, 4 * P_SF_CH, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    if (c_f32)
+        e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)M, (uint64_t)N, (uint64_t)N * 4, 32, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)M, (uint64_t)N, (uint64_t)N * 2, 32, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemm_mxfp8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pair_smem_bytes());
+    if (e != cudaSuccess) return e;
+    if (pair_tiles < 1) return cudaSuccess;
+    return launch_pdl(gemm_mxfp8_pair_kernel, dim3((unsigned)(2 * pair_tiles)), dim3(NUM_THREADS), pair_smem_bytes(),
+                      st, ta, tb, tsa, tsb, tc, offsets, groups, M, N, K, c, c_f32, err, wait_timeout_ns(),
+                      debug_extra_tx());
 }
 
 }  // namespace
@@ -382,18 +722,21 @@ cudaError_t launch(const void* aq, const void* as, const void* bq, const void* b
 cudaError_t launch_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs, int64_t m,
                               int64_t n, int64_t k, void* c, int c_f32, uint32_t* err, int sms, cudaStream_t st) {
     (void)sms;
-    const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
-    return launch(aq, as, bq, bs, nullptr, 1, m, n, k, c, c_f32, err, grid, st);
+    const int64_t n_tiles = (n + BN - 1) / BN;
+    return launch(aq, as, bq, bs, nullptr, 1, m, n, k, c, c_f32, err, ((m + BM - 1) / BM) * n_tiles,
+                  ((m + 2 * BM - 1) / (2 * BM)) * n_tiles, st);
 }
 
 cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs,
                                       const int32_t* offsets, int groups, int64_t total_m, int64_t n, int64_t k,
                                       void* c, int c_f32, uint32_t* err, int sms, cudaStream_t st) {
     (void)sms;
-    // Upper bound on the tile count without reading the device-side offsets:
-    // every group adds at most one partial row tile.
-    const int64_t grid = ((total_m + BM - 1) / BM + groups) * ((n + BN - 1) / BN);
-    return launch(aq, as, bq, bs, offsets, groups, total_m, n, k, c, c_f32, err, grid, st);
+    // Upper bounds on the tile counts without reading the device-side
+    // offsets: every group adds at most one partial row tile.
+    const int64_t n_tiles = (n + BN - 1) / BN;
+    return launch(aq, as, bq, bs, offsets, groups, total_m, n, k, c, c_f32, err,
+                  ((total_m + BM - 1) / BM + groups) * n_tiles, ((total_m + 2 * BM - 1) / (2 * BM) + groups) * n_tiles,
+                  st);
 }
 
 }  // namespace fpq

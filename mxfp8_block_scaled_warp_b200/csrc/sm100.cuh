@@ -215,6 +215,18 @@ __device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t a_de
         : "memory");
 }
 
+// Block-scaled MXFP8 MMA issued by the leader for the pair (E8M0 scale byte
+// per 32 K-elements selected by the sf ids in idesc).
+__device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
 // Shared -> TMEM scale copy for the pair: each CTA's own shared memory at
 // `sdesc` into its own TMEM at `taddr` (32 rows x 128 bits, replicated into
 // the four lane quadrants).

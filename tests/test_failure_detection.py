@@ -21,15 +21,19 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 
-def _mx_operands(fpq):
+def _mx_operands(fpq, m):
     wl = workloads.mxfp8_256x512()
-    qa, sa = fpq.quantize(wl["a"].cuda(), fpq.MXFP8)
+    a = wl["a"] if m == wl["a"].shape[0] else workloads.normal_bf16((m, 512), 0.02, 7)
+    qa, sa = fpq.quantize(a.cuda(), fpq.MXFP8)
     qb, sb = fpq.quantize(wl["b"].cuda(), fpq.MXFP8)
     return qa, sa, qb, sb
 
 
-def test_gemm_wait_timeout_is_reported_and_context_survives(fpq, orc):
-    qa, sa, qb, sb = _mx_operands(fpq)
+# m = 64: one-CTA kernel; m = 256: CTA pair (the leader's stage barrier
+# never completes; the peer, the scale loaders and the epilogue time out too)
+@pytest.mark.parametrize("m", [64, 256])
+def test_gemm_wait_timeout_is_reported_and_context_survives(fpq, orc, m):
+    qa, sa, qb, sb = _mx_operands(fpq, m)
     torch.cuda.synchronize()
     assert fpq.fpq_get_device_error() == 0
     good = fpq.scaled_gemm(fpq.MXFP8, qa, sa, fpq.MXFP8, qb, sb, out_dtype=torch.float32)
@@ -40,7 +44,7 @@ def test_gemm_wait_timeout_is_reported_and_context_survives(fpq, orc):
     try:
         t0 = time.time()
         stalled = torch.full_like(good, -7.0)
-        fpq.fpq_scaled_gemm(fpq.MXFP8, qa, sa, fpq.MXFP8, qb, sb, 64, 256, 512, stalled, fpq.OUT_F32)
+        fpq.fpq_scaled_gemm(fpq.MXFP8, qa, sa, fpq.MXFP8, qb, sb, m, 256, 512, stalled, fpq.OUT_F32)
         code = fpq.fpq_get_device_error()
         elapsed = time.time() - t0
     finally:

@@ -40,8 +40,10 @@ def rand_codes(rng, shape, lo=0x00, hi=0x7E):
 
 # ------------------------------------------------------------------ MXFP8 dense
 
+# M above 128 with K a multiple of 512 runs on CTA pairs (256 x 256 tiles,
+# scale rows by TMA); the other shapes on one-CTA 128 x 256 tiles
 @pytest.mark.parametrize("m,n,k", [(64, 256, 512), (300, 272, 640), (128, 256, 128), (1, 16, 128),
-                                   (257, 512, 1024)])
+                                   (257, 512, 1024), (300, 272, 1024), (520, 512, 2048), (129, 16, 512)])
 def test_mxfp8_gemm_random(fpq, orc, m, n, k):
     a = rand((m, k), 100 + m, std=0.02, outliers=0.01)
     b = rand((n, k), 200 + n, std=0.02, outliers=0.01)
@@ -255,6 +257,46 @@ def test_grouped_small_all_entries(fpq, orc):
     for dt in (torch.float32, torch.bfloat16):
         c = fpq.grouped_scaled_gemm(fpq.MXFP8, dev(aq), dev(as_), dev(bq), dev(bs), dev(offsets), out_dtype=dt)
         check(c, ref, orc, f"grouped small {dt}")
+    assert fpq.fpq_get_device_error() == 0
+
+
+@pytest.mark.parametrize("n", [256, 272])
+def test_grouped_pair_all_entries(fpq, orc, n):
+    """Grouped GEMM on CTA pairs (K a multiple of 512): an empty expert, one
+    of 7 rows, a pair tile ending inside an expert (293 = 256 + 37 rows), one
+    just over a pair tile (257) and a single row; with N = 272 the last
+    column tile reaches into the next expert's weight rows, whose output
+    columns must not be written."""
+    groups, k = 5, 512
+    offsets = np.array([0, 7, 7, 300, 557, 558], np.int32)
+    total = int(offsets[-1])
+    a = rand((total, k), 510, std=1.0)
+    w = rand((groups * n, k), 511 + n, std=0.02).reshape(groups, n, k)
+    aq, as_ = orc.quant_mxfp8(a)
+    bq, bs = orc.quant_mxfp8(w)
+    rows, cols = np.meshgrid(np.arange(total), np.arange(n), indexing="ij")
+    ref = orc.grouped_gemm_entries(FMX, aq, as_, bq, bs, offsets, rows.ravel(), cols.ravel()).reshape(total, n)
+    for dt in (torch.float32, torch.bfloat16):
+        c = fpq.grouped_scaled_gemm(fpq.MXFP8, dev(aq), dev(as_), dev(bq), dev(bs), dev(offsets), out_dtype=dt)
+        check(c, ref, orc, f"grouped pair n={n} {dt}")
+    assert fpq.fpq_get_device_error() == 0
+
+
+def test_grouped_pair_repeatable(fpq):
+    """Repeated grouped launches on CTA pairs give bit-identical C (the scale
+    atoms are handed between the CTAs of a pair through barriers)."""
+    rng = np.random.default_rng(13)
+    groups, n, k = 8, 512, 2048
+    offsets = np.array([0, 300, 300, 1100, 1357, 2000, 2001, 2600, 3072], np.int32)
+    total = int(offsets[-1])
+    aq = dev(rand_codes(rng, (total, k)))
+    bq = dev(rand_codes(rng, (groups, n, k)))
+    as_ = dev(rng.integers(120, 134, (total, k // 32)).astype(np.uint8))
+    bs = dev(rng.integers(120, 134, (groups, n, k // 32)).astype(np.uint8))
+    off = dev(offsets)
+    first = fpq.grouped_scaled_gemm(fpq.MXFP8, aq, as_, bq, bs, off, out_dtype=torch.float32)
+    for _ in range(6):
+        assert torch.equal(fpq.grouped_scaled_gemm(fpq.MXFP8, aq, as_, bq, bs, off, out_dtype=torch.float32), first)
     assert fpq.fpq_get_device_error() == 0
 
 
