@@ -32,6 +32,11 @@ __device__ __forceinline__ Unit load_unit(const uint4* x, int64_t u) {
     return Unit{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
 }
 
+__device__ __forceinline__ Unit load_unit_hint(const uint4* x, int64_t u, uint64_t pol) {
+    uint4 a = ld_stream_hint(x + 2 * u, pol), b = ld_stream_hint(x + 2 * u + 1, pol);
+    return Unit{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
+}
+
 __device__ __forceinline__ uint32_t unit_absmax(const Unit& v) {
     uint32_t m = abs2(v.w[0]);
 #pragma unroll
@@ -383,15 +388,18 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
         const int n = (int)min64(NV_TILE_UNITS, upm - w.t * NV_TILE_UNITS);
         const uint4* xi = x + 2 * base;
         const int u0 = threadIdx.x;
+        // The amax pass keeps its lines in L2 (evict-last) for the encode pass,
+        // which reads them a matrix later and lets them go (evict-first).
         if (w.is_a) {
+            const uint64_t keep = l2_policy_evict_last();
             uint32_t m = 0;
             Unit cur;
-            if (u0 < n) cur = load_unit(xi, u0);
+            if (u0 < n) cur = load_unit_hint(xi, u0, keep);
 #pragma unroll
             for (int i = 0; i < NV_UNITS_PER_THREAD; ++i) {
                 const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit(xi, u + kThreads);
+                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, keep);
                 if (u < n) m = max(m, unit_absmax(cur));
                 cur = nxt;
             }
@@ -407,8 +415,9 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
                 atomicAdd(done + w.b, 1u);
             }
         } else {
+            const uint64_t drop = l2_policy_evict_first();
             Unit cur;
-            if (u0 < n) cur = load_unit(xi, u0);    // the input is ready; only g must wait
+            if (u0 < n) cur = load_unit_hint(xi, u0, drop);    // the input is ready; only g must wait
             if (threadIdx.x == 0) s_ok = wait_count(done + w.b, (uint32_t)nT, err) ? 1 : 0;
             __syncthreads();
             if (!s_ok) return;
@@ -423,7 +432,7 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
             for (int i = 0; i < NV_UNITS_PER_THREAD; ++i) {
                 const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit(xi, u + kThreads);
+                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, drop);
                 if (u < n) nvfp4_encode_unit(cur, g, g_ok, gb, rg, tab6, s_dec, s_inv, qi + u, si + u);
                 cur = nxt;
             }
