@@ -214,6 +214,54 @@ FPQ_API fpq_status fpq_scaled_gemm_nvfp4(const void* aq, const void* as, const f
                                          void* c, int32_t c_dtype, void* stream);
 
 /*
+ * fpq_gemm_bf16 -- C = alpha * (P * Q^T) on bf16 operands with fp32
+ * accumulation on the tensor cores (the products of the QAT backward below).
+ *
+ *   p    bf16 [m, k] row-major (K contiguous)
+ *   q    bf16 [n, k] row-major (K contiguous)
+ *   c    bf16 [m, n] (round-to-nearest-even of fp32(alpha * fp32 sum))
+ *
+ * Requires m >= 1, n and k positive multiples of 8, 16-byte aligned
+ * pointers.  Errors: FPQ_ERR_INVALID_ARG, FPQ_ERR_ALIGNMENT, FPQ_ERR_CUDA;
+ * device-side wait timeouts go to the device error word.
+ */
+FPQ_API fpq_status fpq_gemm_bf16(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha,
+                                 void* c, void* stream);
+
+/*
+ * fpq_qat_backward -- backward of the QAT linear layer with the
+ * straight-through estimator ["DeepSeek R1 and V3 get quantization-aware
+ * fine-tuning on Fireworks", Synopsis and Interpretation: LoRA adapters
+ * trained through the FP8-quantized forward, the base weight frozen].  The
+ * forward is y = fq(x) fq(W_eff)^T with W_eff = W + (alpha/r) B A
+ * (fpq_lora_merge_fakequant + the 1x128 fake-quant of x + fpq_scaled_gemm);
+ * the fake-quantizers pass gradients unchanged, so for the output gradient
+ * dy:
+ *   dx = dy Wfq,   dw = dy^T Xfq,   da = (alpha/r) B^T dw,   db = (alpha/r) dw A^T
+ * each with fp32 accumulation and rounded to bf16; da and db use the bf16 dw.
+ *
+ *   dy      bf16 [m, n]      gradient of the layer output
+ *   x_fq    bf16 [m, k]      fake-quantized activations (dequantized 1x128 codes)
+ *   w_fq    bf16 [n, k]      fake-quantized merged weight (w_fq output of
+ *                            fpq_lora_merge_fakequant)
+ *   lora_a  bf16 [r, k], lora_b bf16 [n, r]
+ *   dx      bf16 [m, k];  dw bf16 [n, k] (gradient of W_eff);
+ *   da      bf16 [r, k];  db bf16 [n, r]
+ *   workspace   16-byte aligned, fpq_qat_backward_workspace_bytes(m, n, k, r)
+ *               bytes (transposed operands), caller-owned
+ *
+ * Requires m, n, k positive multiples of 8 and r a multiple of 8 in [8, 256];
+ * every pointer 16-byte aligned.  Errors: FPQ_ERR_INVALID_ARG,
+ * FPQ_ERR_ALIGNMENT, FPQ_ERR_WORKSPACE, FPQ_ERR_CUDA; device-side wait
+ * timeouts go to the device error word.
+ */
+FPQ_API size_t fpq_qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);
+FPQ_API fpq_status fpq_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
+                                    const void* lora_b, int64_t m, int64_t n, int64_t k, int32_t r,
+                                    float alpha_over_r, void* dx, void* dw, void* da, void* db, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
  * fpq_grouped_scaled_gemm -- per-expert product over a token-permuted
  * activation matrix (MoE routed experts) [FP "Quick start": routed MoE
  * expert projections; DS "Как FP8 связан с MoE-архитектурой DeepSeek V3"]:

@@ -25,10 +25,10 @@ __all__ = [
     "FP8_1x128", "FP8_128x128", "MXFP8", "NVFP4", "OUT_BF16", "OUT_F32", "FpqError", "lib_path", "load",
     "fpq_version", "fpq_quantize_workspace_bytes", "fpq_quantize_block", "fpq_dequantize",
     "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_scaled_gemm_nvfp4", "fpq_grouped_scaled_gemm",
-    "fpq_get_device_error",
+    "fpq_get_device_error", "fpq_gemm_bf16", "fpq_qat_backward_workspace_bytes", "fpq_qat_backward",
     "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
     "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "scaled_gemm_nvfp4", "grouped_scaled_gemm",
-    "scale_shape", "code_shape",
+    "scale_shape", "code_shape", "gemm_bf16", "qat_backward",
 ]
 
 FP8_1x128, FP8_128x128, MXFP8, NVFP4 = 0, 1, 2, 3
@@ -75,6 +75,9 @@ def _load() -> ctypes.CDLL:
         "fpq_scaled_gemm_nvfp4": (I32, [P, P, P, P, P, P, I64, I64, I64, P, I32, P]),
         "fpq_grouped_scaled_gemm": (I32, [I32, P, P, P, P, P, I32, I64, I64, I64, P, I32, P]),
         "fpq_get_device_error": (I32, [P, ctypes.POINTER(I32)]),
+        "fpq_gemm_bf16": (I32, [P, P, I64, I64, I64, F, P, P]),
+        "fpq_qat_backward_workspace_bytes": (SZ, [I64, I64, I64, I32]),
+        "fpq_qat_backward": (I32, [P, P, P, P, P, I64, I64, I64, I32, F, P, P, P, P, P, SZ, P]),
         "fpq_quantize_nvfp4_noalloc": (I32, [P, I64, I64, I64, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -139,6 +142,22 @@ def fpq_scaled_gemm(fmt_a, aq, as_, fmt_b, bq, bs, m, n, k, c, c_dtype, stream=N
 def fpq_scaled_gemm_nvfp4(aq, as_, ag, bq, bs, bg, m, n, k, c, c_dtype, stream=None):
     _check(load().fpq_scaled_gemm_nvfp4(_ptr(aq), _ptr(as_), _ptr(ag), _ptr(bq), _ptr(bs), _ptr(bg), m, n, k,
                                       _ptr(c), c_dtype, _stream(stream)), "fpq_scaled_gemm_nvfp4")
+
+
+def fpq_gemm_bf16(p, q, m, n, k, alpha, c, stream=None):
+    _check(load().fpq_gemm_bf16(_ptr(p), _ptr(q), m, n, k, float(alpha), _ptr(c), _stream(stream)), "fpq_gemm_bf16")
+
+
+def fpq_qat_backward_workspace_bytes(m: int, n: int, k: int, r: int) -> int:
+    return load().fpq_qat_backward_workspace_bytes(m, n, k, r)
+
+
+def fpq_qat_backward(dy, x_fq, w_fq, lora_a, lora_b, m, n, k, r, alpha_over_r, dx, dw, da, db, workspace,
+                     stream=None):
+    wsb = workspace.numel() * workspace.element_size()
+    _check(load().fpq_qat_backward(_ptr(dy), _ptr(x_fq), _ptr(w_fq), _ptr(lora_a), _ptr(lora_b), m, n, k, r,
+                                   float(alpha_over_r), _ptr(dx), _ptr(dw), _ptr(da), _ptr(db), _ptr(workspace),
+                                   wsb, _stream(stream)), "fpq_qat_backward")
 
 
 def fpq_grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, groups, total_m, n, k, c, c_dtype, stream=None):
@@ -250,6 +269,32 @@ def scaled_gemm_nvfp4(aq, as_, ag, bq, bs, bg, out_dtype=torch.bfloat16, stream=
     fpq_scaled_gemm_nvfp4(aq, as_, ag, bq, bs, bg, m, n, k, c, OUT_F32 if out_dtype == torch.float32 else OUT_BF16,
                           stream)
     return c
+
+
+def gemm_bf16(p, q, alpha: float = 1.0, stream=None):
+    """C = alpha (P Q^T) for bf16 P [m, k] and Q [n, k]; C bf16 [m, n]."""
+    m, k = p.shape
+    n = q.shape[0]
+    c = torch.empty((m, n), dtype=torch.bfloat16, device=p.device)
+    fpq_gemm_bf16(p, q, m, n, k, alpha, c, stream)
+    return c
+
+
+def qat_backward(dy, x_fq, w_fq, lora_a, lora_b, alpha_over_r: float, stream=None):
+    """Gradients of the QAT linear layer (straight-through estimator) for the
+    output gradient dy [m, n]: returns (dx [m, k], dw [n, k], da [r, k],
+    db [n, r]), all bf16."""
+    m, n = dy.shape
+    k = x_fq.shape[1]
+    r = lora_a.shape[0]
+    dev = dy.device
+    dx = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((n, k), dtype=torch.bfloat16, device=dev)
+    da = torch.empty((r, k), dtype=torch.bfloat16, device=dev)
+    db = torch.empty((n, r), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((fpq_qat_backward_workspace_bytes(m, n, k, r) + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    fpq_qat_backward(dy, x_fq, w_fq, lora_a, lora_b, m, n, k, r, alpha_over_r, dx, dw, da, db, ws, stream)
+    return dx, dw, da, db
 
 
 def grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, out_dtype=torch.bfloat16, stream=None):

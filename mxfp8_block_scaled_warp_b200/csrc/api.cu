@@ -234,6 +234,48 @@ fpq_status fpq_scaled_gemm_nvfp4(const void* aq, const void* as, const float* ag
                                             (cudaStream_t)stream), "nvfp4 gemm launch");
 }
 
+fpq_status fpq_gemm_bf16(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha, void* c,
+                         void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (m < 1 || n < 8 || n % 8 || k < 8 || k % 8 || m > (1 << 30) || n > (1 << 30) || k > (1 << 30)) {
+        set_detail("need m >= 1, n and k positive multiples of 8");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if ((st = check_ptrs({p, q, c})) != FPQ_OK) return st;
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_gemm_bf16(p, q, m, n, k, alpha, c, d->err, (cudaStream_t)stream), "bf16 gemm launch");
+}
+
+size_t fpq_qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) {
+    if (m < 1 || n < 1 || k < 1 || r < 1) return 0;
+    return fpq::qat_backward_workspace_bytes(m, n, k, r);
+}
+
+fpq_status fpq_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
+                            const void* lora_b, int64_t m, int64_t n, int64_t k, int32_t r, float alpha_over_r,
+                            void* dx, void* dw, void* da, void* db, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (m < 8 || m % 8 || n < 8 || n % 8 || k < 8 || k % 8 || r < 8 || r % 8 || r > 256 || m > (1 << 30) ||
+        n > (1 << 30) || k > (1 << 30)) {
+        set_detail("need m, n, k positive multiples of 8 and r a multiple of 8 in [8, 256]");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if ((st = check_ptrs({dy, x_fq, w_fq, lora_a, lora_b, dx, dw, da, db})) != FPQ_OK) return st;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < fpq::qat_backward_workspace_bytes(m, n, k, r)) {
+        set_detail("need a 16-byte aligned workspace of fpq_qat_backward_workspace_bytes() bytes");
+        return FPQ_ERR_WORKSPACE;
+    }
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_qat_backward(dy, x_fq, w_fq, lora_a, lora_b, m, n, k, r, alpha_over_r, dx, dw, da,
+                                              db, workspace, d->err, (cudaStream_t)stream),
+                     "qat backward launch");
+}
+
 fpq_status fpq_grouped_scaled_gemm(fpq_format fmt, const void* aq, const void* as, const void* bq,
                                    const void* bs, const int32_t* group_offsets, int32_t groups,
                                    int64_t total_m, int64_t n, int64_t k, void* c, int32_t c_dtype,

@@ -1,0 +1,226 @@
+// gemm_bf16.cu -- bf16 GEMM on the 5th-generation tensor cores for the
+// backward of the QAT step: C = alpha * (P * Q^T), P [M, K] and Q [N, K]
+// bf16, K-major, fp32 accumulation in TMEM, bf16 output (round to nearest
+// even).  With the straight-through estimator the fake-quantizers pass
+// gradients unchanged, so the backward of y = fq(x) fq(W_eff)^T is plain
+// bf16 products of the gradient with the fake-quantized operands
+// ("DeepSeek R1 and V3 get quantization-aware fine-tuning on Fireworks",
+// Synopsis: the LoRA adapters are trained through the quantized forward).
+//
+// One 128 x 256 output tile per CTA; the K loop runs over 64-wide K tiles
+// (128 bytes per row, 128-byte swizzle) through a 4-stage TMA ring; four
+// tcgen05.mma kind::f16 (bf16 x bf16 -> fp32, K = 16 each) per K tile.
+// Warp roles: warp 0 TMA producer, warp 2 TMEM allocator and MMA issuer
+// (one elected thread); then all eight warps run the epilogue: TMEM lanes
+// 32 (w & 3) .. + 31 and columns 128 (w >> 2) .. + 127 of the accumulator,
+// times alpha, to bf16, staged in 128-byte-swizzled boxes and written by
+// TMA stores (which clip rows past M and columns past N).
+// Every wait on an mbarrier is bounded by wall time (4 s); on expiry the
+// kernel records FPQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace fpq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 64;           // BK in bf16 elements (128 bytes)
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BK * 2, B_TILE = BN * BK * 2;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int NUM_THREADS = 256;
+constexpr int EPI_WARP_BYTES = 32 * 128 * 2;        // a warp's 32 x 128 block of C, bf16
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+
+struct __align__(1024) Smem {
+    uint8_t a[STAGES][A_TILE];
+    uint8_t b[STAGES][B_TILE];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tmem_full;
+    uint32_t tmem_base;
+};
+static_assert(8 * EPI_WARP_BYTES <= STAGES * (A_TILE + B_TILE), "epilogue staging exceeds the ring");
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
+// (bits 7-9 and 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > kTimeoutNs) {
+            raise_device_error(err, FPQ_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmC, int64_t M, int64_t N, int64_t K, float alpha,
+                 uint32_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = (int)((N + BN - 1) / BN);
+    const int mt = blockIdx.x / n_tiles, nt = blockIdx.x - mt * n_tiles;
+    const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
+    const int KT = (int)((K + BK - 1) / BK);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.tmem_full, 1);
+        fence_barrier_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    pdl_wait();
+
+    if (warp == 0) {
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmC);
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
+                mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE);
+                tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)m0);
+                tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)n0);
+            }
+        }
+    } else if (warp == 2) {
+        if (elect_one()) {
+            const uint32_t idesc = idesc_bf16(BM, BN);
+            bool ok = true;
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
+                if (!wait_or_timeout(&sm.full[s], ph, err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    mma_bf16(tmem, desc_kmajor_sw128(a_base + 32 * k), desc_kmajor_sw128(b_base + 32 * k), idesc,
+                             (kt > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.empty[s]);
+            }
+            if (ok) mma_commit(&sm.tmem_full);
+        }
+    }
+
+    __syncwarp();     // the role warps' other lanes wait here for the elected lane, without polling
+    {
+        const int q = warp & 3, half = warp >> 2;
+        const int64_t row0 = m0 + 32 * q, col0 = n0 + 128 * half;
+        const bool ok = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.tmem_full, 0, err));
+        if (ok && row0 < M && col0 < N) {
+            tc_fence_after();
+            uint8_t* stage = &sm.a[0][0] + warp * EPI_WARP_BYTES;
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half + 32 * c), r[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {     // columns 32c + 8j .. + 7 = box c / 2, chunk 4 (c % 2) + j
+                    uint32_t h[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        h[e] = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(r[c][8 * j + 2 * e]), alpha),
+                                               __fmul_rn(__uint_as_float(r[c][8 * j + 2 * e + 1]), alpha));
+                    *reinterpret_cast<uint4*>(stage + (c / 2) * 4096 + sw128_offset(lane, 4 * (c % 2) + j)) =
+                        make_uint4(h[0], h[1], h[2], h[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                for (int x = 0; x < 2; ++x)
+                    if (col0 + x * 64 < N) tma_store_2d(&tmC, stage + x * 4096, (int32_t)(col0 + x * 64), (int32_t)row0);
+                bulk_commit_group();
+                bulk_wait_group_read0();     // the staging must stay valid until read
+            }
+            __syncwarp();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+int smem_bytes() { return (int)sizeof(Smem) + 1024; }
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha, void* c,
+                             uint32_t* err, cudaStream_t st) {
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        if (e != cudaSuccess) return e;
+        configured[dev] = 1;
+    }
+    CUtensorMap ta, tb, tc;
+    e = make_tmap_2d(&ta, p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)k, (uint64_t)k * 2, BM, BK,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d(&tb, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)n, (uint64_t)k, (uint64_t)k * 2, BN, BK,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)n, (uint64_t)n * 2, 32, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
+    return launch_pdl(gemm_bf16_kernel, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta, tb, tc, m, n,
+                      k, alpha, err);
+}
+
+}  // namespace fpq

@@ -39,6 +39,17 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
                               const float* bg, int64_t m, int64_t n, int64_t k, void* c, int c_f32, uint32_t* err,
                               cudaStream_t st);
 
+// C = alpha P Q^T, P [m, k] and Q [n, k] bf16 K-major, C [m, n] bf16.
+cudaError_t launch_gemm_bf16(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha, void* c,
+                             uint32_t* err, cudaStream_t st);
+
+// QAT backward (straight-through estimator); workspace of
+// qat_backward_workspace_bytes bytes.
+size_t qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t r);
+cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
+                                const void* lora_b, int64_t m, int64_t n, int64_t k, int64_t r, float alpha_over_r,
+                                void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, cudaStream_t st);
+
 cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void* bq,
                                       const void* bs, const int32_t* offsets, int groups,
                                       int64_t total_m, int64_t n, int64_t k, void* c, int c_f32,

@@ -1,0 +1,106 @@
+// qat_backward.cu -- the backward of the QAT step's linear layer with the
+// straight-through estimator ("DeepSeek R1 and V3 get quantization-aware
+// fine-tuning on Fireworks", Synopsis and Interpretation: LoRA adapters
+// trained through the FP8-quantized forward, then merged).  The forward is
+// y = fq(x) fq(W_eff)^T with W_eff = W + (alpha / r) B A; the fake-quantizers
+// pass gradients unchanged, W is frozen, so for the output gradient dY:
+//   dX     = dY Wfq                  [M, K]
+//   dW_eff = dY^T Xfq                [N, K]   (bf16, also an output)
+//   dA     = (alpha / r) B^T dW_eff  [r, K]
+//   dB     = (alpha / r) dW_eff A^T  [N, r]
+// with Xfq = fq(x), Wfq = fq(W_eff) in bf16 and fp32 accumulation, all
+// results rounded to bf16.  Every product runs on the bf16 tensor-core GEMM
+// (C = alpha P Q^T with both operands K-major); the operands that are not
+// K-major for their product are transposed first into the caller's
+// workspace by a tiled transpose kernel.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace fpq {
+
+namespace {
+
+// bf16 [R, C] -> [C, R].  One CTA of 256 threads per 64 x 64 tile: 16-byte
+// row loads into shared memory (rows padded by 8 elements), then each thread
+// gathers 8 consecutive elements of an output row (a column of the tile)
+// and writes them as one 16-byte store.  R and C are multiples of 8.
+constexpr int TT = 64;
+
+__global__ void __launch_bounds__(256)
+transpose_bf16_kernel(const uint16_t* __restrict__ in, uint16_t* __restrict__ out, int64_t R, int64_t C) {
+    pdl_trigger();
+    __shared__ uint16_t tile[TT][TT + 8];
+    const int64_t r0 = (int64_t)blockIdx.y * TT, c0 = (int64_t)blockIdx.x * TT;
+    pdl_wait();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int v = threadIdx.x + 256 * i;          // 512 chunks of 8 elements
+        const int r = v >> 3, c = (v & 7) * 8;
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (r0 + r < R && c0 + c < C) x = *reinterpret_cast<const uint4*>(in + (r0 + r) * C + c0 + c);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            tile[r][c + 2 * j] = (uint16_t)(w[j] & 0xFFFFu);
+            tile[r][c + 2 * j + 1] = (uint16_t)(w[j] >> 16);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int v = threadIdx.x + 256 * i;
+        const int oc = v >> 3, orr = (v & 7) * 8;     // output row c0 + oc, columns r0 + orr .. + 7
+        if (c0 + oc < C && r0 + orr < R) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                w[j] = (uint32_t)tile[orr + 2 * j][oc] | ((uint32_t)tile[orr + 2 * j + 1][oc] << 16);
+            *reinterpret_cast<uint4*>(out + (c0 + oc) * R + r0 + orr) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+cudaError_t transpose(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
+    const dim3 grid((unsigned)((C + TT - 1) / TT), (unsigned)((R + TT - 1) / TT));
+    return launch_pdl(transpose_bf16_kernel, grid, dim3(256), 0, st, (const uint16_t*)in, (uint16_t*)out, R, C);
+}
+
+inline size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+// Workspace: Wfq^T [K, N], dY^T [N, M], Xfq^T [K, M], dW^T [K, N], B^T [r, N],
+// bf16, each region 256-byte aligned.
+size_t qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t r) {
+    return round_up(2 * (size_t)(k * n)) + round_up(2 * (size_t)(n * m)) + round_up(2 * (size_t)(k * m)) +
+           round_up(2 * (size_t)(k * n)) + round_up(2 * (size_t)(r * n));
+}
+
+cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
+                                const void* lora_b, int64_t m, int64_t n, int64_t k, int64_t r, float alpha_over_r,
+                                void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, cudaStream_t st) {
+    uint8_t* p = static_cast<uint8_t*>(ws);
+    void* wt = p;  p += round_up(2 * (size_t)(k * n));
+    void* dyt = p; p += round_up(2 * (size_t)(n * m));
+    void* xt = p;  p += round_up(2 * (size_t)(k * m));
+    void* dwt = p; p += round_up(2 * (size_t)(k * n));
+    void* bt = p;
+    cudaError_t e;
+    // dX = dY Wfq: contraction over N; Q = Wfq^T [K, N]
+    if ((e = transpose(w_fq, wt, n, k, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm_bf16(dy, wt, m, k, n, 1.0f, dx, err, st)) != cudaSuccess) return e;
+    // dW = dY^T Xfq: contraction over M; P = dY^T [N, M], Q = Xfq^T [K, M]
+    if ((e = transpose(dy, dyt, m, n, st)) != cudaSuccess) return e;
+    if ((e = transpose(x_fq, xt, m, k, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm_bf16(dyt, xt, n, k, m, 1.0f, dw, err, st)) != cudaSuccess) return e;
+    // dA = (alpha / r) B^T dW: contraction over N; P = B^T [r, N], Q = dW^T [K, N]
+    if ((e = transpose(dw, dwt, n, k, st)) != cudaSuccess) return e;
+    if ((e = transpose(lora_b, bt, n, r, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm_bf16(bt, dwt, r, k, n, alpha_over_r, da, err, st)) != cudaSuccess) return e;
+    // dB = (alpha / r) dW A^T: contraction over K; P = dW [N, K], Q = A [r, K]
+    return launch_gemm_bf16(dw, lora_a, n, r, k, alpha_over_r, db, err, st);
+}
+
+}  // namespace fpq

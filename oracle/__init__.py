@@ -84,6 +84,10 @@ def lib() -> ctypes.CDLL:
             "orc_gemm_entries": (None, [I, P, P, P, I, P, P, P, I64, I64, I64, P, P, I64, P]),
             "orc_gemm_full": (None, [I, P, P, P, I, P, P, P, I64, I64, I64, P]),
             "orc_grouped_gemm_entries": (None, [I, P, P, P, P, P, I32, I64, I64, I64, P, P, I64, P]),
+            "orc_gemm_bf16_entries": (None, [P, P, I64, D, P, P, I64, P]),
+            "orc_gemm_bf16_full": (None, [P, P, I64, I64, I64, D, P]),
+            "orc_bf16_encode_f64": (U16, [D]),
+            "orc_bf16_encode_f64_array": (None, [P, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -314,3 +318,50 @@ def gemm_tolerance_ok(got: np.ndarray, ref: np.ndarray, rms_ref: float | None = 
     err = np.abs(got - ref)
     ratio = float(np.max(err / np.maximum(bound, 1e-300))) if err.size else 0.0
     return bool(np.all(err <= bound)), ratio
+
+
+# ---------------------------------------------------------------- QAT backward (oracle.c, "QAT backward")
+
+def gemm_bf16_full(p: np.ndarray, q: np.ndarray, alpha: float = 1.0) -> np.ndarray:
+    """fp64 C = alpha * P Q^T, P [m, k], Q [n, k] bf16 (uint16)."""
+    p, q = _bf16(p), _bf16(q)
+    m, k = p.shape
+    n = q.shape[0]
+    assert q.shape[1] == k
+    out = np.empty((m, n), np.float64)
+    lib().orc_gemm_bf16_full(_p(p), _p(q), m, n, k, float(alpha), _p(out))
+    return out
+
+
+def gemm_bf16_entries(p: np.ndarray, q: np.ndarray, rows, cols, alpha: float = 1.0) -> np.ndarray:
+    """fp64 entries alpha * (P Q^T)[rows[i], cols[i]]."""
+    p, q = _bf16(p), _bf16(q)
+    k = p.shape[1]
+    assert q.shape[1] == k
+    rows = np.ascontiguousarray(rows, np.int64)
+    cols = np.ascontiguousarray(cols, np.int64)
+    out = np.empty(rows.shape[0], np.float64)
+    lib().orc_gemm_bf16_entries(_p(p), _p(q), k, float(alpha), _p(rows), _p(cols), rows.shape[0], _p(out))
+    return out
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Nearest bf16 (ties to even) of fp64 values, as uint16 patterns."""
+    x = np.ascontiguousarray(x, np.float64)
+    out = np.empty(x.shape, np.uint16)
+    lib().orc_bf16_encode_f64_array(_p(x), x.size, _p(out))
+    return out
+
+
+def qat_backward(dy, x_fq, w_fq, lora_a, lora_b, alpha_over_r: float):
+    """(dx, dw, da, db) in fp64 for the straight-through-estimator backward:
+    dx = dy Wfq, dw = dy^T Xfq, da = (alpha/r) B^T bf16(dw),
+    db = (alpha/r) bf16(dw) A^T.  Inputs bf16 as uint16; the transposes here
+    only move data."""
+    dy, x_fq, w_fq, lora_a, lora_b = (_bf16(t) for t in (dy, x_fq, w_fq, lora_a, lora_b))
+    dx = gemm_bf16_full(dy, np.ascontiguousarray(w_fq.T))
+    dw = gemm_bf16_full(np.ascontiguousarray(dy.T), np.ascontiguousarray(x_fq.T))
+    dw16 = bf16_round(dw)
+    da = gemm_bf16_full(np.ascontiguousarray(lora_b.T), np.ascontiguousarray(dw16.T), alpha_over_r)
+    db = gemm_bf16_full(dw16, lora_a, alpha_over_r)
+    return dx, dw, da, db

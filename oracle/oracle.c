@@ -507,3 +507,66 @@ ORC_API void orc_grouped_gemm_entries(int fmt, const uint8_t* aq, const void* as
         out[i] = orc_gemm_entry(fmt, aq, as, 0, fmt, be, bse, 0, total_m, n, k, row, col_idx[i]);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* QAT backward with the straight-through estimator ("DeepSeek R1 and V3 get */
+/* quantization-aware fine-tuning on Fireworks", Synopsis and Interpretation: */
+/* LoRA adapters trained through the FP8-quantized forward, base weight      */
+/* frozen).  For y = fq(x) fq(W_eff)^T, W_eff = W + (alpha/r) B A, the        */
+/* fake-quantizers pass gradients unchanged:                                  */
+/*   dx = dy Wfq, dw = dy^T Xfq, da = (alpha/r) B^T bf16(dw),                 */
+/*   db = (alpha/r) bf16(dw) A^T.                                             */
+/* The building block is one product entry of bf16 operands, C[i][j] =       */
+/* alpha * sum_t P[i][t] Q[j][t] (both operands row-major with the summed    */
+/* index last), summed in fp64 with t ascending (every product of two bf16   */
+/* values is exact in fp64).                                                  */
+/* ------------------------------------------------------------------------ */
+
+static double bf16_dot(const uint16_t* p, const uint16_t* q, int64_t k)
+{
+    double s = 0.0;
+    for (int64_t t = 0; t < k; ++t) s += orc_bf16_decode(p[t]) * orc_bf16_decode(q[t]);
+    return s;
+}
+
+ORC_API void orc_gemm_bf16_entries(const uint16_t* p, const uint16_t* q, int64_t k, double alpha,
+                                   const int64_t* row_idx, const int64_t* col_idx, int64_t count, double* out)
+{
+    for (int64_t i = 0; i < count; ++i)
+        out[i] = alpha * bf16_dot(p + row_idx[i] * k, q + col_idx[i] * k, k);
+}
+
+ORC_API void orc_gemm_bf16_full(const uint16_t* p, const uint16_t* q, int64_t m, int64_t n, int64_t k,
+                                double alpha, double* out)
+{
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < n; ++j) out[i * n + j] = alpha * bf16_dot(p + i * k, q + j * k, k);
+}
+
+/* bf16 rounding (nearest, ties to even) of an fp64 value: the fp32 step is
+ * exact for every value the products above can produce only up to fp32
+ * precision, so the rounding is done from the two bf16 neighbours of the
+ * fp64 value directly. */
+ORC_API uint16_t orc_bf16_encode_f64(double v)
+{
+    if (isnan(v)) return 0x7FC0u;
+    float f = (float)v;                                /* nearest fp32 */
+    uint16_t c = orc_bf16_encode(f);
+    if ((double)f == v || isinf(f)) return c;
+    /* the fp32 rounding may have moved v onto a bf16 midpoint: decide the
+     * two bf16 candidates around v in fp64 */
+    uint32_t u = bits_from_f32(f);
+    uint16_t lo = (uint16_t)(u >> 16), hi = (uint16_t)(lo + 1);
+    double a = fabs(v), vlo = fabs(orc_bf16_decode(lo));
+    if (vlo > a) { hi = lo; lo = (uint16_t)(lo - 1); vlo = fabs(orc_bf16_decode(lo)); }
+    double vhi = ((hi & 0x7F80u) == 0x7F80u) ? ldexp(1.0, 128) : fabs(orc_bf16_decode(hi));
+    double dlo = a - vlo, dhi = vhi - a;
+    if (dlo < dhi) return lo;
+    if (dhi < dlo) return hi;
+    return (lo & 1u) ? hi : lo;
+}
+
+ORC_API void orc_bf16_encode_f64_array(const double* x, int64_t count, uint16_t* out)
+{
+    for (int64_t i = 0; i < count; ++i) out[i] = orc_bf16_encode_f64(x[i]);
+}

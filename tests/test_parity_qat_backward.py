@@ -1,0 +1,115 @@
+"""GPU parity of the bf16 tensor-core GEMM and the QAT backward
+(straight-through estimator; "DeepSeek R1 and V3 get quantization-aware
+fine-tuning on Fireworks", Synopsis and Interpretation) against the oracle's
+fp64 sums: |gpu - ref| <= 8e-3 |ref| + 1e-2 rms(ref) per element, the same
+acceptance as the other GEMMs; bit-exact where every product and partial sum
+is exact in fp32 and the result is a bf16 value."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def dev(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda() if a.dtype == np.uint16 else \
+        torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def rand(shape, seed, std=1.0):
+    return workloads.as_u16(workloads.normal_bf16(shape, std, seed))
+
+
+def check(got: torch.Tensor, ref: np.ndarray, orc, what: str, rms=None):
+    g = got.float().cpu().numpy().astype(np.float64)
+    ok, ratio = orc.gemm_tolerance_ok(g, ref, rms)
+    assert ok, f"{what}: worst |err|/bound = {ratio:.3f}"
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 256, 64), (200, 272, 136), (1, 8, 8), (300, 512, 1000), (16, 7168, 2048),
+                                   (2048, 16, 7168)])
+def test_gemm_bf16_random(fpq, orc, m, n, k):
+    p, q = rand((m, k), 900 + m), rand((n, k), 901 + n, std=0.05)
+    for alpha in (1.0, 2.0):
+        ref = orc.gemm_bf16_full(p, q, alpha)
+        c = fpq.gemm_bf16(dev(p), dev(q), alpha)
+        check(c, ref, orc, f"bf16 gemm {m}x{n}x{k} alpha={alpha}")
+    assert fpq.fpq_get_device_error() == 0
+
+
+def test_gemm_bf16_integer_exact(fpq, orc):
+    """Entries in {-1, 0, 1}: every product and partial sum is exact in fp32,
+    and alpha = 0.25 times a sum of at most 64 terms is a multiple of 0.25
+    below 16, which bf16 holds exactly: C must match bit for bit."""
+    rng = np.random.default_rng(30)
+    m, n, k = 256, 512, 64
+    ip, iq = rng.integers(-1, 2, (m, k)), rng.integers(-1, 2, (n, k))
+    p = workloads.as_u16(torch.from_numpy(ip.astype(np.float32)).to(torch.bfloat16))
+    q = workloads.as_u16(torch.from_numpy(iq.astype(np.float32)).to(torch.bfloat16))
+    c = fpq.gemm_bf16(dev(p), dev(q), 0.25)
+    ref = 0.25 * (ip @ iq.T).astype(np.float64)
+    assert np.array_equal(c.float().cpu().numpy().astype(np.float64), ref)
+
+
+def _qat_inputs(m, n, k, r, seed):
+    dy = rand((m, n), seed, std=1.0)
+    x_fq = rand((m, k), seed + 1, std=1.0)
+    w_fq = rand((n, k), seed + 2, std=0.02)
+    a = rand((r, k), seed + 3, std=0.01)
+    b = rand((n, r), seed + 4, std=0.01)
+    return dy, x_fq, w_fq, a, b
+
+
+@pytest.mark.parametrize("m,n,k,r", [(256, 272, 384, 16), (136, 64, 520, 8)])
+def test_qat_backward_small(fpq, orc, m, n, k, r):
+    dy, x_fq, w_fq, a, b = _qat_inputs(m, n, k, r, 950 + m)
+    dx, dw, da, db = fpq.qat_backward(dev(dy), dev(x_fq), dev(w_fq), dev(a), dev(b), 2.0)
+    rdx, rdw, rda, rdb = orc.qat_backward(dy, x_fq, w_fq, a, b, 2.0)
+    check(dx, rdx, orc, "dx")
+    check(dw, rdw, orc, "dw")
+    check(da, rda, orc, "da")
+    check(db, rdb, orc, "db")
+    assert fpq.fpq_get_device_error() == 0
+
+
+def test_qat_backward_full_size_sampled(fpq, orc):
+    """The QAT layer of the fine-grained workload's shape (x 8192 x 7168,
+    W 2048 x 7168, r = 16): sampled entries of dx and dw, and whole columns
+    of da and rows of db (those need whole columns / rows of the oracle's
+    bf16 dw)."""
+    m, n, k, r = 8192, 2048, 7168, 16
+    dy, x_fq, w_fq, a, b = _qat_inputs(m, n, k, r, 970)
+    dx, dw, da, db = fpq.qat_backward(dev(dy), dev(x_fq), dev(w_fq), dev(a), dev(b), 2.0)
+    assert fpq.fpq_get_device_error() == 0
+    rng = np.random.default_rng(31)
+    rows, cols = rng.integers(0, m, 256), rng.integers(0, k, 256)
+    ref = orc.gemm_bf16_entries(dy, np.ascontiguousarray(w_fq.T), rows, cols)
+    check(dx[torch.from_numpy(rows).cuda(), torch.from_numpy(cols).cuda()], ref, orc, "dx sampled",
+          rms=float(np.sqrt(np.mean(ref ** 2))))
+    dyt, xt = np.ascontiguousarray(dy.T), np.ascontiguousarray(x_fq.T)
+    rows, cols = rng.integers(0, n, 256), rng.integers(0, k, 256)
+    ref = orc.gemm_bf16_entries(dyt, xt, rows, cols)
+    check(dw[torch.from_numpy(rows).cuda(), torch.from_numpy(cols).cuda()], ref, orc, "dw sampled",
+          rms=float(np.sqrt(np.mean(ref ** 2))))
+    # da[:, kc] needs dw16[:, kc]; db[nr, :] needs dw16[nr, :]
+    kc = rng.integers(0, k, 3)
+    nn, kk = np.meshgrid(np.arange(n), kc, indexing="ij")
+    dw_cols = orc.bf16_round(orc.gemm_bf16_entries(dyt, xt, nn.ravel(), kk.ravel()).reshape(n, len(kc)))
+    ref = orc.gemm_bf16_full(np.ascontiguousarray(b.T), np.ascontiguousarray(dw_cols.T), 2.0)     # [r, 3]
+    check(da[:, torch.from_numpy(kc).cuda()], ref, orc, "da columns")
+    nr = rng.integers(0, n, 2)
+    rr, kk = np.meshgrid(nr, np.arange(k), indexing="ij")
+    dw_rows = orc.bf16_round(orc.gemm_bf16_entries(dyt, xt, rr.ravel(), kk.ravel()).reshape(len(nr), k))
+    ref = orc.gemm_bf16_full(dw_rows, a, 2.0)                                                       # [2, r]
+    check(db[torch.from_numpy(nr).cuda()], ref, orc, "db rows")
+
+
+def test_qat_backward_rejects_bad_args(fpq):
+    t = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fpq.FpqError):       # r not a multiple of 8
+        fpq.fpq_qat_backward(t, t, t, t, t, 64, 64, 64, 12, 1.0, t, t, t, t, ws)
+    with pytest.raises(fpq.FpqError):       # workspace too small
+        fpq.fpq_qat_backward(t, t, t, t, t, 64, 64, 64, 8, 1.0, t, t, t, t, ws[:16])
