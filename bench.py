@@ -362,6 +362,76 @@ class MoePrequant(Step):
         return hb, db
 
 
+class QatBackward(Step):
+    """The backward of the QAT linear layer (straight-through estimator) at
+    the QAT workload's shape: x 8192x7168, W 2048x7168, LoRA r = 16, alpha/r
+    = 2; dx, dW_eff, dA, dB in bf16 on the bf16 tensor-core GEMM, each
+    operand read in its stored layout.  The same four launches as
+    fpq_qat_backward, issued through the C ABI one by one so that each is
+    timed."""
+    name = "qat_backward"
+    dominant = "gemm_bf16_dx"
+    dtype = "bf16xbf16->f32 (bf16 out)"
+    tensor_ratio = 1.0
+
+    def __init__(self, fpq, dev, m=8192, n=2048, k=7168):
+        self.f = fpq
+        wl = workloads.qat_forward(m=m, n=n, k=k)
+        r = wl["lora_a"].shape[0]
+        self.m, self.n, self.k, self.r = m, n, k, r
+        self.aor = wl["alpha_over_r"]
+        x, w = wl["x"].to(dev), wl["w"].to(dev)
+        self.a, self.b = wl["lora_a"].to(dev), wl["lora_b"].to(dev)
+        # the forward's fake-quantized operands, made by the library
+        xq, xs = fpq.quantize(x, fpq.FP8_1x128)
+        self.x_fq = fpq.dequantize(fpq.FP8_1x128, xq, xs)
+        self.w_fq = fpq.lora_merge_fakequant(w, self.a, self.b, self.aor, want_fq=True)[2]
+        del x, w, xq, xs
+        self.dy_host = workloads.normal_bf16((m, n), 1.0, seed=3005).pin_memory()
+        self.dy = self.dy_host.to(dev)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        self.dx, self.dw = torch.empty((m, k), **bf), torch.empty((n, k), **bf)
+        self.da, self.db = torch.empty((r, k), **bf), torch.empty((n, r), **bf)
+        wsb = fpq.fpq_qat_backward_workspace_bytes(m, n, k, r)
+        self.ws = torch.empty(((wsb + 15) // 16 * 16,), dtype=torch.uint8, device=dev) if wsb else None
+        self.dx_host = torch.empty((m, k), dtype=torch.bfloat16).pin_memory()
+        self.da_host = torch.empty((r, k), dtype=torch.bfloat16).pin_memory()
+        self.db_host = torch.empty((n, r), dtype=torch.bfloat16).pin_memory()
+        self.flops = 2.0 * (2 * m * n * k + 2 * r * n * k)
+        self.quant_bytes = 0.0          # no quantize kernel in this step
+        self.launches = 4
+        self.config = {"workload": "qat_backward: dy 8192x2048 N(0,1); x_fq = 1x128 fake-quant of x 8192x7168 "
+                                   "N(0,1); w_fq = 128x128 fake-quant of W + 2 B A (W 2048x7168 N(0,0.02), r = 16); "
+                                   "dx = dy w_fq, dW = dy^T x_fq, dA = 2 B^T dW, dB = 2 dW A^T, bf16",
+                       "m": m, "n": n, "k": k, "r": r, "l2": "flushed before every step (256 MiB write)"}
+
+    def kernels(self):
+        f, m, n, k, r, aor = self.f, self.m, self.n, self.k, self.r, self.aor
+        return [
+            ("gemm_bf16_dx", lambda: f.fpq_gemm_bf16_layout(self.dy, 0, self.w_fq, 1, m, k, n, 1.0, self.dx)),
+            ("gemm_bf16_dw", lambda: f.fpq_gemm_bf16_layout(self.dy, 1, self.x_fq, 1, n, k, m, 1.0, self.dw)),
+            ("gemm_bf16_da", lambda: f.fpq_gemm_bf16_layout(self.b, 1, self.dw, 1, r, k, n, aor, self.da)),
+            ("gemm_bf16_db", lambda: f.fpq_gemm_bf16_layout(self.dw, 0, self.a, 0, n, r, k, aor, self.db)),
+        ]
+
+    def kernel_work(self):
+        m, n, k, r = self.m, self.n, self.k, self.r
+        return {"gemm_bf16_dx": ("TFLOP/s", 2.0 * m * n * k), "gemm_bf16_dw": ("TFLOP/s", 2.0 * m * n * k),
+                "gemm_bf16_da": ("TFLOP/s", 2.0 * r * n * k), "gemm_bf16_db": ("TFLOP/s", 2.0 * r * n * k)}
+
+    def e2e_step(self, stream):
+        """dy from pinned host memory, the public fpq_qat_backward call, dx,
+        dA and dB back to pinned host memory (dW_eff stays on the device)."""
+        f = self.f
+        self.dy.copy_(self.dy_host, non_blocking=True)
+        f.fpq_qat_backward(self.dy, self.x_fq, self.w_fq, self.a, self.b, self.m, self.n, self.k, self.r, self.aor,
+                           self.dx, self.dw, self.da, self.db, self.ws)
+        self.dx_host.copy_(self.dx, non_blocking=True)
+        self.da_host.copy_(self.da, non_blocking=True)
+        self.db_host.copy_(self.db, non_blocking=True)
+        return self.dy.numel() * 2, (self.dx.numel() + self.da.numel() + self.db.numel()) * 2
+
+
 class Nvfp4Gemm(Step):
     """The fine-grained GEMM shape in NVFP4: both operands quantized on the
     GPU (packed E2M1, E4M3 scale per 16, fp32 tensor scale) and multiplied
@@ -422,7 +492,7 @@ class Nvfp4Gemm(Step):
 
 
 STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": QatForward,
-         "moe_prequant": MoePrequant, "nvfp4_gemm": Nvfp4Gemm}
+         "moe_prequant": MoePrequant, "nvfp4_gemm": Nvfp4Gemm, "qat_backward": QatBackward}
 
 
 # ------------------------------------------------------------------ traffic from committed ncu summaries
@@ -431,7 +501,7 @@ def _source_hash(kernel: str) -> str | None:
     src = {"gemm_fp8_f32scale": "gemm_fp8_f32scale.cu", "gemm_grouped_mxfp8": "gemm_mxfp8.cu",
            "gemm_mxfp8": "gemm_mxfp8.cu", "quant_fp8_1x128": "quant_kernels.cu",
            "quant_mxfp8": "quant_kernels.cu", "lora_merge_fq": "merge_kernel.cu",
-           "gemm_nvfp4": "gemm_nvfp4.cu"}.get(kernel)
+           "gemm_nvfp4": "gemm_nvfp4.cu", "gemm_bf16_dx": "gemm_bf16.cu"}.get(kernel)
     if not src:
         return None
     with open(os.path.join(ROOT, "mxfp8_block_scaled_warp_b200", "csrc", src), "rb") as f:
@@ -759,7 +829,7 @@ def main():
                     "unit": "GB/s", "frac": dom["achieved"] / peaks["hbm_gbs"], "traffic": traffic,
                     "peak_note": f"{peaks['source']} HBM copy bandwidth"}
     else:
-        kind = "fp4" if step.tensor_ratio == 4.0 else "fp8"
+        kind = {4.0: "fp4", 2.0: "fp8", 1.0: "bf16"}[step.tensor_ratio]
         which = "sustained" if sustained else "burst"
         roofline = {"kernel": step.dominant, "bound": "tensor", "achieved": dom["achieved"], "peak": tensor_peak,
                     "unit": "TFLOP/s", "frac": dom["achieved"] / tensor_peak, "traffic": traffic,
@@ -768,7 +838,7 @@ def main():
                                  f"({bf16_peak} TFLOP/s; nominal dense ratio); {which} because the kernel-timing "
                                  f"loop's clock record {'shows' if sustained else 'does not show'} the power cap"}
     quant_ms = sum(statistics.mean(per_kernel[n]) for n in names if not n.startswith("gemm"))
-    quant_gbs = step.quant_bytes / (quant_ms * 1e-3) / 1e9
+    quant_gbs = step.quant_bytes / (quant_ms * 1e-3) / 1e9 if quant_ms > 0 else None
 
     # end to end: host buffers through the public API, copies inside the timed region
     e2e = None
@@ -794,7 +864,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": step.unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": step.dtype, "data": "synthetic",
-            "config": dict(step.config, launch="CUDA graph of the step replayed per timed step; per-kernel times from a second graph with events around each kernel"), "quantize_gbs": quant_gbs, "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"],
+            "config": dict(step.config, launch="CUDA graph of the step replayed per timed step; per-kernel times from a second graph with events around each kernel"), "quantize_gbs": quant_gbs,
+            "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"] if quant_gbs is not None else None,
             "kernels": kernels_out, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.launches * args.steps, "clocks": clk.summary(), "clocks_kernel_timing": ck,
             "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp8_tflops": fp8_peak_burst, "tensor_tflops": tensor_peak,

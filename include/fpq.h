@@ -229,6 +229,25 @@ FPQ_API fpq_status fpq_gemm_bf16(const void* p, const void* q, int64_t m, int64_
                                  void* c, void* stream);
 
 /*
+ * fpq_gemm_bf16_layout -- as fpq_gemm_bf16 with each operand in either
+ * layout: p_mn = 0: P stored [m, k] (K contiguous); p_mn = 1: P stored
+ * [k, m] (m contiguous, i.e. the product uses its transpose); likewise q_mn
+ * for Q ([n, k] or [k, n]).  Requires additionally m a multiple of 8 when
+ * p_mn = 1.
+ */
+FPQ_API fpq_status fpq_gemm_bf16_layout(const void* p, int32_t p_mn, const void* q, int32_t q_mn, int64_t m,
+                                        int64_t n, int64_t k, float alpha, void* c, void* stream);
+
+/*
+ * fpq_transpose_bf16 -- out[c, r] = in[r, c] for bf16 [rows, cols] (the data
+ * movement of the QAT backward below, exposed for callers that schedule its
+ * products themselves).  Requires rows and cols positive multiples of 8,
+ * 16-byte aligned pointers, in and out not overlapping.  Errors:
+ * FPQ_ERR_INVALID_ARG, FPQ_ERR_ALIGNMENT, FPQ_ERR_CUDA.
+ */
+FPQ_API fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, int64_t cols, void* stream);
+
+/*
  * fpq_qat_backward -- backward of the QAT linear layer with the
  * straight-through estimator ["DeepSeek R1 and V3 get quantization-aware
  * fine-tuning on Fireworks", Synopsis and Interpretation: LoRA adapters
@@ -247,8 +266,9 @@ FPQ_API fpq_status fpq_gemm_bf16(const void* p, const void* q, int64_t m, int64_
  *   lora_a  bf16 [r, k], lora_b bf16 [n, r]
  *   dx      bf16 [m, k];  dw bf16 [n, k] (gradient of W_eff);
  *   da      bf16 [r, k];  db bf16 [n, r]
- *   workspace   16-byte aligned, fpq_qat_backward_workspace_bytes(m, n, k, r)
- *               bytes (transposed operands), caller-owned
+ *   workspace   fpq_qat_backward_workspace_bytes(m, n, k, r) bytes, 16-byte
+ *               aligned, caller-owned; currently 0 (the products read every
+ *               operand in its stored layout) and the pointer may be NULL
  *
  * Requires m, n, k positive multiples of 8 and r a multiple of 8 in [8, 256];
  * every pointer 16-byte aligned.  Errors: FPQ_ERR_INVALID_ARG,

@@ -25,7 +25,9 @@ __all__ = [
     "FP8_1x128", "FP8_128x128", "MXFP8", "NVFP4", "OUT_BF16", "OUT_F32", "FpqError", "lib_path", "load",
     "fpq_version", "fpq_quantize_workspace_bytes", "fpq_quantize_block", "fpq_dequantize",
     "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_scaled_gemm_nvfp4", "fpq_grouped_scaled_gemm",
-    "fpq_get_device_error", "fpq_gemm_bf16", "fpq_qat_backward_workspace_bytes", "fpq_qat_backward",
+    "fpq_get_device_error", "fpq_gemm_bf16", "fpq_gemm_bf16_layout", "fpq_transpose_bf16",
+    "fpq_qat_backward_workspace_bytes",
+    "fpq_qat_backward",
     "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
     "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "scaled_gemm_nvfp4", "grouped_scaled_gemm",
     "scale_shape", "code_shape", "gemm_bf16", "qat_backward",
@@ -76,6 +78,8 @@ def _load() -> ctypes.CDLL:
         "fpq_grouped_scaled_gemm": (I32, [I32, P, P, P, P, P, I32, I64, I64, I64, P, I32, P]),
         "fpq_get_device_error": (I32, [P, ctypes.POINTER(I32)]),
         "fpq_gemm_bf16": (I32, [P, P, I64, I64, I64, F, P, P]),
+        "fpq_transpose_bf16": (I32, [P, P, I64, I64, P]),
+        "fpq_gemm_bf16_layout": (I32, [P, I32, P, I32, I64, I64, I64, F, P, P]),
         "fpq_qat_backward_workspace_bytes": (SZ, [I64, I64, I64, I32]),
         "fpq_qat_backward": (I32, [P, P, P, P, P, I64, I64, I64, I32, F, P, P, P, P, P, SZ, P]),
         "fpq_quantize_nvfp4_noalloc": (I32, [P, I64, I64, I64, P, P, P, P]),
@@ -148,16 +152,26 @@ def fpq_gemm_bf16(p, q, m, n, k, alpha, c, stream=None):
     _check(load().fpq_gemm_bf16(_ptr(p), _ptr(q), m, n, k, float(alpha), _ptr(c), _stream(stream)), "fpq_gemm_bf16")
 
 
+def fpq_gemm_bf16_layout(p, p_mn, q, q_mn, m, n, k, alpha, c, stream=None):
+    _check(load().fpq_gemm_bf16_layout(_ptr(p), int(p_mn), _ptr(q), int(q_mn), m, n, k, float(alpha), _ptr(c),
+                                       _stream(stream)), "fpq_gemm_bf16_layout")
+
+
+def fpq_transpose_bf16(x, out, rows, cols, stream=None):
+    _check(load().fpq_transpose_bf16(_ptr(x), _ptr(out), rows, cols, _stream(stream)), "fpq_transpose_bf16")
+
+
 def fpq_qat_backward_workspace_bytes(m: int, n: int, k: int, r: int) -> int:
     return load().fpq_qat_backward_workspace_bytes(m, n, k, r)
 
 
 def fpq_qat_backward(dy, x_fq, w_fq, lora_a, lora_b, m, n, k, r, alpha_over_r, dx, dw, da, db, workspace,
                      stream=None):
-    wsb = workspace.numel() * workspace.element_size()
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load().fpq_qat_backward(_ptr(dy), _ptr(x_fq), _ptr(w_fq), _ptr(lora_a), _ptr(lora_b), m, n, k, r,
-                                   float(alpha_over_r), _ptr(dx), _ptr(dw), _ptr(da), _ptr(db), _ptr(workspace),
-                                   wsb, _stream(stream)), "fpq_qat_backward")
+                                   float(alpha_over_r), _ptr(dx), _ptr(dw), _ptr(da), _ptr(db),
+                                   _ptr(workspace) if workspace is not None else None, wsb, _stream(stream)),
+           "fpq_qat_backward")
 
 
 def fpq_grouped_scaled_gemm(fmt, aq, as_, bq, bs, group_offsets, groups, total_m, n, k, c, c_dtype, stream=None):
@@ -292,7 +306,8 @@ def qat_backward(dy, x_fq, w_fq, lora_a, lora_b, alpha_over_r: float, stream=Non
     dw = torch.empty((n, k), dtype=torch.bfloat16, device=dev)
     da = torch.empty((r, k), dtype=torch.bfloat16, device=dev)
     db = torch.empty((n, r), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty((fpq_qat_backward_workspace_bytes(m, n, k, r) + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    wsb = fpq_qat_backward_workspace_bytes(m, n, k, r)
+    ws = torch.empty((wsb + 15) // 16 * 16, dtype=torch.uint8, device=dev) if wsb else None
     fpq_qat_backward(dy, x_fq, w_fq, lora_a, lora_b, m, n, k, r, alpha_over_r, dx, dw, da, db, ws, stream)
     return dx, dw, da, db
 

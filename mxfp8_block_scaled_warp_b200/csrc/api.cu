@@ -245,7 +245,38 @@ fpq_status fpq_gemm_bf16(const void* p, const void* q, int64_t m, int64_t n, int
     if ((st = check_ptrs({p, q, c})) != FPQ_OK) return st;
     const DeviceState* d = device_state(&st);
     if (!d) return st;
-    return from_cuda(fpq::launch_gemm_bf16(p, q, m, n, k, alpha, c, d->err, (cudaStream_t)stream), "bf16 gemm launch");
+    return from_cuda(fpq::launch_gemm_bf16(p, false, q, false, m, n, k, alpha, c, d->err, (cudaStream_t)stream),
+                     "bf16 gemm launch");
+}
+
+fpq_status fpq_gemm_bf16_layout(const void* p, int32_t p_mn, const void* q, int32_t q_mn, int64_t m, int64_t n,
+                                int64_t k, float alpha, void* c, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (m < 1 || n < 8 || n % 8 || k < 8 || k % 8 || (p_mn && m % 8) || m > (1 << 30) || n > (1 << 30) ||
+        k > (1 << 30) || (p_mn != 0 && p_mn != 1) || (q_mn != 0 && q_mn != 1)) {
+        set_detail("need n, k positive multiples of 8, m >= 1 (a multiple of 8 when P is MN-major), flags 0|1");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if ((st = check_ptrs({p, q, c})) != FPQ_OK) return st;
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_gemm_bf16(p, p_mn != 0, q, q_mn != 0, m, n, k, alpha, c, d->err,
+                                           (cudaStream_t)stream),
+                     "bf16 gemm launch");
+}
+
+fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, int64_t cols, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (rows < 8 || rows % 8 || cols < 8 || cols % 8 || rows > (1 << 30) || cols > (1 << 30)) {
+        set_detail("need rows and cols positive multiples of 8");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if ((st = check_ptrs({in, out})) != FPQ_OK) return st;
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_transpose_bf16(in, out, rows, cols, (cudaStream_t)stream), "transpose launch");
 }
 
 size_t fpq_qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) {
@@ -265,7 +296,8 @@ fpq_status fpq_qat_backward(const void* dy, const void* x_fq, const void* w_fq, 
         return FPQ_ERR_INVALID_ARG;
     }
     if ((st = check_ptrs({dy, x_fq, w_fq, lora_a, lora_b, dx, dw, da, db})) != FPQ_OK) return st;
-    if (!workspace || !aligned16(workspace) || workspace_bytes < fpq::qat_backward_workspace_bytes(m, n, k, r)) {
+    const size_t need = fpq::qat_backward_workspace_bytes(m, n, k, r);
+    if (need > 0 && (!workspace || !aligned16(workspace) || workspace_bytes < need)) {
         set_detail("need a 16-byte aligned workspace of fpq_qat_backward_workspace_bytes() bytes");
         return FPQ_ERR_WORKSPACE;
     }

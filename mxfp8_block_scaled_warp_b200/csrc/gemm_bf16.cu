@@ -8,8 +8,14 @@
 // Synopsis: the LoRA adapters are trained through the quantized forward).
 //
 // One 128 x 256 output tile per CTA; the K loop runs over 64-wide K tiles
-// (128 bytes per row, 128-byte swizzle) through a 4-stage TMA ring; four
-// tcgen05.mma kind::f16 (bf16 x bf16 -> fp32, K = 16 each) per K tile.
+// through a 4-stage TMA ring; four tcgen05.mma kind::f16 (bf16 x bf16 ->
+// fp32, K = 16 each) per K tile.  Either operand may be K-major (stored
+// [rows, K], a K tile = one TMA box of 128-byte rows) or MN-major (stored
+// [K, rows]: its K tile = boxes of 64 rows-of-the-product x 64 K, each K row
+// 128 bytes, 128-byte swizzle; the MMA reads it through an MN-major shared
+// memory descriptor: 8 K rows of 128 bytes per 1 KB swizzle atom, atoms
+// 1 KB apart along K (SBO), 64-element blocks 8 KB apart along M or N (LBO)),
+// so the backward products need no transposed copies.
 // Warp roles: warp 0 TMA producer, warp 2 TMEM allocator and MMA issuer
 // (one elected thread); then all eight warps run the epilogue: TMEM lanes
 // 32 (w & 3) .. + 31 and columns 128 (w >> 2) .. + 127 of the accumulator,
@@ -38,9 +44,11 @@ constexpr int NUM_THREADS = 256;
 constexpr int EPI_WARP_BYTES = 32 * 128 * 2;        // a warp's 32 x 128 block of C, bf16
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
+constexpr int MN_BOX = 64 * BK * 2;                 // one MN-major box: 64 rows-of-the-product x 64 K
 struct __align__(1024) Smem {
     uint8_t a[STAGES][A_TILE];
     uint8_t b[STAGES][B_TILE];
+    uint8_t guard[32768];      // keeps any descriptor-addressed read of the last stage inside the allocation
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tmem_full;
@@ -49,9 +57,18 @@ struct __align__(1024) Smem {
 static_assert(8 * EPI_WARP_BYTES <= STAGES * (A_TILE + B_TILE), "epilogue staging exceeds the ring");
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
-// (bits 7-9 and 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+// (bits 7-9 and 10-12 = 1), A / B MN-major (bits 15 / 16), N >> 3 at bit
+// 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// Shared-memory descriptor of K step kk (16 K) of an operand tile.
+template <bool MN>
+__device__ __forceinline__ uint64_t op_desc(uint32_t base, int kk) {
+    return MN ? smem_desc(base + 2048u * (uint32_t)kk, 8192, 1024, kLayoutSw128)
+              : desc_kmajor_sw128(base + 32u * (uint32_t)kk);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -82,6 +99,7 @@ __device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
     }
 }
 
+template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmC, int64_t M, int64_t N, int64_t K, float alpha,
@@ -122,13 +140,25 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
                 if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
                 mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE);
-                tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)m0);
-                tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)n0);
+                if (A_MN) {
+#pragma unroll
+                    for (int j = 0; j < BM / 64; ++j)
+                        tma_load_2d(sm.a[s] + j * MN_BOX, &tmA, &sm.full[s], (int32_t)(m0 + 64 * j), kt * BK);
+                } else {
+                    tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)m0);
+                }
+                if (B_MN) {
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j)
+                        tma_load_2d(sm.b[s] + j * MN_BOX, &tmB, &sm.full[s], (int32_t)(n0 + 64 * j), kt * BK);
+                } else {
+                    tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)n0);
+                }
             }
         }
     } else if (warp == 2) {
         if (elect_one()) {
-            const uint32_t idesc = idesc_bf16(BM, BN);
+            const uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
             bool ok = true;
             for (int kt = 0; kt < KT; ++kt) {
                 const int s = kt % STAGES;
@@ -138,7 +168,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
 #pragma unroll
                 for (int k = 0; k < BK / 16; ++k)
-                    mma_bf16(tmem, desc_kmajor_sw128(a_base + 32 * k), desc_kmajor_sw128(b_base + 32 * k), idesc,
+                    mma_bf16(tmem, op_desc<A_MN>(a_base, k), op_desc<B_MN>(b_base, k), idesc,
                              (kt > 0 || k > 0) ? 1u : 0u);
                 mma_commit(&sm.empty[s]);
             }
@@ -194,33 +224,48 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
 int smem_bytes() { return (int)sizeof(Smem) + 1024; }
 
-}  // namespace
-
-cudaError_t launch_gemm_bf16(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha, void* c,
-                             uint32_t* err, cudaStream_t st) {
+template <bool A_MN, bool B_MN>
+cudaError_t launch_t(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha, void* c,
+                     uint32_t* err, cudaStream_t st) {
     static int configured[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        e = cudaFuncSetAttribute(gemm_bf16_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem_bytes());
         if (e != cudaSuccess) return e;
         configured[dev] = 1;
     }
     CUtensorMap ta, tb, tc;
-    e = make_tmap_2d(&ta, p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)k, (uint64_t)k * 2, BM, BK,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
+    // K-major [rows, k], box 128 or 256 rows x 64 K; MN-major [k, rows], box 64 K x 64 rows
+    e = A_MN ? make_tmap_2d(&ta, p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)k, (uint64_t)m, (uint64_t)m * 2,
+                            BK, 64, CU_TENSOR_MAP_SWIZZLE_128B)
+             : make_tmap_2d(&ta, p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)k, (uint64_t)k * 2,
+                            BM, BK, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    e = make_tmap_2d(&tb, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)n, (uint64_t)k, (uint64_t)k * 2, BN, BK,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
+    e = B_MN ? make_tmap_2d(&tb, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)k, (uint64_t)n, (uint64_t)n * 2,
+                            BK, 64, CU_TENSOR_MAP_SWIZZLE_128B)
+             : make_tmap_2d(&tb, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)n, (uint64_t)k, (uint64_t)k * 2,
+                            BN, BK, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)n, (uint64_t)n * 2, 32, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
-    return launch_pdl(gemm_bf16_kernel, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta, tb, tc, m, n,
-                      k, alpha, err);
+    return launch_pdl(gemm_bf16_kernel<A_MN, B_MN>, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta,
+                      tb, tc, m, n, k, alpha, err);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n, int64_t k,
+                             float alpha, void* c, uint32_t* err, cudaStream_t st) {
+    if (p_mn) return q_mn ? launch_t<true, true>(p, q, m, n, k, alpha, c, err, st)
+                          : launch_t<true, false>(p, q, m, n, k, alpha, c, err, st);
+    return q_mn ? launch_t<false, true>(p, q, m, n, k, alpha, c, err, st)
+                : launch_t<false, false>(p, q, m, n, k, alpha, c, err, st);
 }
 
 }  // namespace fpq

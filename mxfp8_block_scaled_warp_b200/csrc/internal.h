@@ -39,9 +39,13 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
                               const float* bg, int64_t m, int64_t n, int64_t k, void* c, int c_f32, uint32_t* err,
                               cudaStream_t st);
 
-// C = alpha P Q^T, P [m, k] and Q [n, k] bf16 K-major, C [m, n] bf16.
-cudaError_t launch_gemm_bf16(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha, void* c,
-                             uint32_t* err, cudaStream_t st);
+// C = alpha P Q^T, C [m, n] bf16.  P is [m, k] (K-major) or, with p_mn,
+// stored as [k, m] (MN-major); likewise Q [n, k] or, with q_mn, [k, n].
+cudaError_t launch_gemm_bf16(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n, int64_t k,
+                             float alpha, void* c, uint32_t* err, cudaStream_t st);
+
+// bf16 [R, C] -> [C, R] (R, C multiples of 8).
+cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st);
 
 // QAT backward (straight-through estimator); workspace of
 // qat_backward_workspace_bytes bytes.

@@ -10,9 +10,9 @@
 //   dB     = (alpha / r) dW_eff A^T  [N, r]
 // with Xfq = fq(x), Wfq = fq(W_eff) in bf16 and fp32 accumulation, all
 // results rounded to bf16.  Every product runs on the bf16 tensor-core GEMM
-// (C = alpha P Q^T with both operands K-major); the operands that are not
-// K-major for their product are transposed first into the caller's
-// workspace by a tiled transpose kernel.
+// (C = alpha P Q^T), which reads each operand in the layout it is stored in
+// (K-major or MN-major).  The tiled bf16 transpose below is exported as a
+// utility.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -62,45 +62,31 @@ transpose_bf16_kernel(const uint16_t* __restrict__ in, uint16_t* __restrict__ ou
     }
 }
 
-cudaError_t transpose(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
-    const dim3 grid((unsigned)((C + TT - 1) / TT), (unsigned)((R + TT - 1) / TT));
-    return launch_pdl(transpose_bf16_kernel, grid, dim3(256), 0, st, (const uint16_t*)in, (uint16_t*)out, R, C);
-}
-
 inline size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
-// Workspace: Wfq^T [K, N], dY^T [N, M], Xfq^T [K, M], dW^T [K, N], B^T [r, N],
-// bf16, each region 256-byte aligned.
-size_t qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t r) {
-    return round_up(2 * (size_t)(k * n)) + round_up(2 * (size_t)(n * m)) + round_up(2 * (size_t)(k * m)) +
-           round_up(2 * (size_t)(k * n)) + round_up(2 * (size_t)(r * n));
+cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
+    const dim3 grid((unsigned)((C + TT - 1) / TT), (unsigned)((R + TT - 1) / TT));
+    return launch_pdl(transpose_bf16_kernel, grid, dim3(256), 0, st, (const uint16_t*)in, (uint16_t*)out, R, C);
 }
+
+// No workspace: every operand is read in the layout it is stored in (the
+// GEMM takes K-major or MN-major operands).
+size_t qat_backward_workspace_bytes(int64_t, int64_t, int64_t, int64_t) { return 0; }
 
 cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
                                 const void* lora_b, int64_t m, int64_t n, int64_t k, int64_t r, float alpha_over_r,
-                                void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, cudaStream_t st) {
-    uint8_t* p = static_cast<uint8_t*>(ws);
-    void* wt = p;  p += round_up(2 * (size_t)(k * n));
-    void* dyt = p; p += round_up(2 * (size_t)(n * m));
-    void* xt = p;  p += round_up(2 * (size_t)(k * m));
-    void* dwt = p; p += round_up(2 * (size_t)(k * n));
-    void* bt = p;
+                                void* dx, void* dw, void* da, void* db, void*, uint32_t* err, cudaStream_t st) {
     cudaError_t e;
-    // dX = dY Wfq: contraction over N; Q = Wfq^T [K, N]
-    if ((e = transpose(w_fq, wt, n, k, st)) != cudaSuccess) return e;
-    if ((e = launch_gemm_bf16(dy, wt, m, k, n, 1.0f, dx, err, st)) != cudaSuccess) return e;
-    // dW = dY^T Xfq: contraction over M; P = dY^T [N, M], Q = Xfq^T [K, M]
-    if ((e = transpose(dy, dyt, m, n, st)) != cudaSuccess) return e;
-    if ((e = transpose(x_fq, xt, m, k, st)) != cudaSuccess) return e;
-    if ((e = launch_gemm_bf16(dyt, xt, n, k, m, 1.0f, dw, err, st)) != cudaSuccess) return e;
-    // dA = (alpha / r) B^T dW: contraction over N; P = B^T [r, N], Q = dW^T [K, N]
-    if ((e = transpose(dw, dwt, n, k, st)) != cudaSuccess) return e;
-    if ((e = transpose(lora_b, bt, n, r, st)) != cudaSuccess) return e;
-    if ((e = launch_gemm_bf16(bt, dwt, r, k, n, alpha_over_r, da, err, st)) != cudaSuccess) return e;
-    // dB = (alpha / r) dW A^T: contraction over K; P = dW [N, K], Q = A [r, K]
-    return launch_gemm_bf16(dw, lora_a, n, r, k, alpha_over_r, db, err, st);
+    // dX [m, k] = dY Wfq: contraction over n; dY [m, n] K-major, Wfq [n, k] MN-major
+    if ((e = launch_gemm_bf16(dy, false, w_fq, true, m, k, n, 1.0f, dx, err, st)) != cudaSuccess) return e;
+    // dW [n, k] = dY^T Xfq: contraction over m; dY [m, n] and Xfq [m, k] MN-major
+    if ((e = launch_gemm_bf16(dy, true, x_fq, true, n, k, m, 1.0f, dw, err, st)) != cudaSuccess) return e;
+    // dA [r, k] = (alpha / r) B^T dW: contraction over n; B [n, r] and dW [n, k] MN-major
+    if ((e = launch_gemm_bf16(lora_b, true, dw, true, r, k, n, alpha_over_r, da, err, st)) != cudaSuccess) return e;
+    // dB [n, r] = (alpha / r) dW A^T: contraction over k; dW [n, k] and A [r, k] K-major
+    return launch_gemm_bf16(dw, false, lora_a, false, n, r, k, alpha_over_r, db, err, st);
 }
 
 }  // namespace fpq

@@ -39,6 +39,28 @@ def test_gemm_bf16_random(fpq, orc, m, n, k):
     assert fpq.fpq_get_device_error() == 0
 
 
+@pytest.mark.parametrize("p_mn,q_mn", [(False, True), (True, False), (True, True)])
+@pytest.mark.parametrize("m,n,k", [(128, 256, 64), (200, 272, 136), (16, 7168, 2048), (520, 16, 1000)])
+def test_gemm_bf16_mn_major(fpq, orc, p_mn, q_mn, m, n, k):
+    """Operands stored with the product's row index contiguous ([k, m] and
+    [k, n]) are read through MN-major descriptors, not transposed."""
+    p, q = rand((m, k), 920 + m), rand((n, k), 921 + n, std=0.05)
+    ref = orc.gemm_bf16_full(p, q, 0.5)
+    ps = np.ascontiguousarray(p.T) if p_mn else p
+    qs = np.ascontiguousarray(q.T) if q_mn else q
+    c = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    fpq.fpq_gemm_bf16_layout(dev(ps), p_mn, dev(qs), q_mn, m, n, k, 0.5, c)
+    check(c, ref, orc, f"bf16 gemm mn {p_mn}{q_mn} {m}x{n}x{k}")
+    assert fpq.fpq_get_device_error() == 0
+
+
+def test_transpose_bf16_exact(fpq):
+    x = rand((200, 136), 930)
+    out = torch.empty((136, 200), dtype=torch.bfloat16, device="cuda")
+    fpq.fpq_transpose_bf16(dev(x), out, 200, 136)
+    assert np.array_equal(workloads.as_u16(out), np.ascontiguousarray(x.T))
+
+
 def test_gemm_bf16_integer_exact(fpq, orc):
     """Entries in {-1, 0, 1}: every product and partial sum is exact in fp32,
     and alpha = 0.25 times a sum of at most 64 terms is a multiple of 0.25
@@ -108,8 +130,10 @@ def test_qat_backward_full_size_sampled(fpq, orc):
 
 def test_qat_backward_rejects_bad_args(fpq):
     t = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
     with pytest.raises(fpq.FpqError):       # r not a multiple of 8
-        fpq.fpq_qat_backward(t, t, t, t, t, 64, 64, 64, 12, 1.0, t, t, t, t, ws)
-    with pytest.raises(fpq.FpqError):       # workspace too small
-        fpq.fpq_qat_backward(t, t, t, t, t, 64, 64, 64, 8, 1.0, t, t, t, t, ws[:16])
+        fpq.fpq_qat_backward(t, t, t, t, t, 64, 64, 64, 12, 1.0, t, t, t, t, None)
+    with pytest.raises(fpq.FpqError):       # m not a multiple of 8
+        fpq.fpq_qat_backward(t, t, t, t, t, 60, 64, 64, 8, 1.0, t, t, t, t, None)
+    big = torch.zeros(4096 + 8, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fpq.FpqError):       # misaligned operand
+        fpq.fpq_qat_backward(big[1:4097].view(64, 64), t, t, t, t, 64, 64, 64, 8, 1.0, t, t, t, t, None)
