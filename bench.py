@@ -366,9 +366,9 @@ class QatBackward(Step):
     """The backward of the QAT linear layer (straight-through estimator) at
     the QAT workload's shape: x 8192x7168, W 2048x7168, LoRA r = 16, alpha/r
     = 2; dx, dW_eff, dA, dB in bf16 on the bf16 tensor-core GEMM, each
-    operand read in its stored layout.  The same four launches as
-    fpq_qat_backward, issued through the C ABI one by one so that each is
-    timed."""
+    operand read in its stored layout, dA and dB split over the contraction.
+    The same launches as fpq_qat_backward, issued through the C ABI one by
+    one so that each product is timed (dA and dB with their reductions)."""
     name = "qat_backward"
     dominant = "gemm_bf16_dx"
     dtype = "bf16xbf16->f32 (bf16 out)"
@@ -394,12 +394,15 @@ class QatBackward(Step):
         self.da, self.db = torch.empty((r, k), **bf), torch.empty((n, r), **bf)
         wsb = fpq.fpq_qat_backward_workspace_bytes(m, n, k, r)
         self.ws = torch.empty(((wsb + 15) // 16 * 16,), dtype=torch.uint8, device=dev) if wsb else None
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.ws_a = torch.empty((fpq.fpq_gemm_bf16_splitk_workspace_bytes(r, k, n),), **u8)
+        self.ws_b = torch.empty((fpq.fpq_gemm_bf16_splitk_workspace_bytes(n, r, k),), **u8)
         self.dx_host = torch.empty((m, k), dtype=torch.bfloat16).pin_memory()
         self.da_host = torch.empty((r, k), dtype=torch.bfloat16).pin_memory()
         self.db_host = torch.empty((n, r), dtype=torch.bfloat16).pin_memory()
         self.flops = 2.0 * (2 * m * n * k + 2 * r * n * k)
         self.quant_bytes = 0.0          # no quantize kernel in this step
-        self.launches = 4
+        self.launches = 6                # dA and dB: split-K GEMM + slice reduction each
         self.config = {"workload": "qat_backward: dy 8192x2048 N(0,1); x_fq = 1x128 fake-quant of x 8192x7168 "
                                    "N(0,1); w_fq = 128x128 fake-quant of W + 2 B A (W 2048x7168 N(0,0.02), r = 16); "
                                    "dx = dy w_fq, dW = dy^T x_fq, dA = 2 B^T dW, dB = 2 dW A^T, bf16",
@@ -410,8 +413,8 @@ class QatBackward(Step):
         return [
             ("gemm_bf16_dx", lambda: f.fpq_gemm_bf16_layout(self.dy, 0, self.w_fq, 1, m, k, n, 1.0, self.dx)),
             ("gemm_bf16_dw", lambda: f.fpq_gemm_bf16_layout(self.dy, 1, self.x_fq, 1, n, k, m, 1.0, self.dw)),
-            ("gemm_bf16_da", lambda: f.fpq_gemm_bf16_layout(self.b, 1, self.dw, 1, r, k, n, aor, self.da)),
-            ("gemm_bf16_db", lambda: f.fpq_gemm_bf16_layout(self.dw, 0, self.a, 0, n, r, k, aor, self.db)),
+            ("gemm_bf16_da", lambda: f.fpq_gemm_bf16_splitk(self.b, 1, self.dw, 1, r, k, n, aor, self.da, self.ws_a)),
+            ("gemm_bf16_db", lambda: f.fpq_gemm_bf16_splitk(self.dw, 0, self.a, 0, n, r, k, aor, self.db, self.ws_b)),
         ]
 
     def kernel_work(self):

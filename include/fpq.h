@@ -239,6 +239,24 @@ FPQ_API fpq_status fpq_gemm_bf16_layout(const void* p, int32_t p_mn, const void*
                                         int64_t n, int64_t k, float alpha, void* c, void* stream);
 
 /*
+ * fpq_gemm_bf16_splitk -- as fpq_gemm_bf16_layout for products with few
+ * output tiles and a long contraction (m or n small, as for the LoRA
+ * gradients of the QAT backward): the contraction is cut into up to 16
+ * slices spread over the SMs, each slice's fp32 sums go to the workspace,
+ * and a second kernel adds the slices in order, multiplies by alpha and
+ * rounds to bf16 (so results are repeatable run to run).
+ *
+ *   workspace   fpq_gemm_bf16_splitk_workspace_bytes(m, n, k) bytes,
+ *               16-byte aligned, caller-owned, not read before written
+ *
+ * Requirements and errors: as fpq_gemm_bf16_layout, plus FPQ_ERR_WORKSPACE.
+ */
+FPQ_API size_t fpq_gemm_bf16_splitk_workspace_bytes(int64_t m, int64_t n, int64_t k);
+FPQ_API fpq_status fpq_gemm_bf16_splitk(const void* p, int32_t p_mn, const void* q, int32_t q_mn, int64_t m,
+                                        int64_t n, int64_t k, float alpha, void* c, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/*
  * fpq_transpose_bf16 -- out[c, r] = in[r, c] for bf16 [rows, cols] (the data
  * movement of the QAT backward below, exposed for callers that schedule its
  * products themselves).  Requires rows and cols positive multiples of 8,
@@ -267,8 +285,10 @@ FPQ_API fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, i
  *   dx      bf16 [m, k];  dw bf16 [n, k] (gradient of W_eff);
  *   da      bf16 [r, k];  db bf16 [n, r]
  *   workspace   fpq_qat_backward_workspace_bytes(m, n, k, r) bytes, 16-byte
- *               aligned, caller-owned; currently 0 (the products read every
- *               operand in its stored layout) and the pointer may be NULL
+ *               aligned, caller-owned, not read before written: fp32 partial
+ *               sums of da and db, whose few output tiles split their
+ *               contraction across the SMs (at most 16 slices each, added in
+ *               slice order by a second kernel, so results are repeatable)
  *
  * Requires m, n, k positive multiples of 8 and r a multiple of 8 in [8, 256];
  * every pointer 16-byte aligned.  Errors: FPQ_ERR_INVALID_ARG,

@@ -26,7 +26,7 @@ __all__ = [
     "fpq_version", "fpq_quantize_workspace_bytes", "fpq_quantize_block", "fpq_dequantize",
     "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_scaled_gemm_nvfp4", "fpq_grouped_scaled_gemm",
     "fpq_get_device_error", "fpq_gemm_bf16", "fpq_gemm_bf16_layout", "fpq_transpose_bf16",
-    "fpq_qat_backward_workspace_bytes",
+    "fpq_gemm_bf16_splitk_workspace_bytes", "fpq_gemm_bf16_splitk", "fpq_qat_backward_workspace_bytes",
     "fpq_qat_backward",
     "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
     "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "scaled_gemm_nvfp4", "grouped_scaled_gemm",
@@ -80,6 +80,8 @@ def _load() -> ctypes.CDLL:
         "fpq_gemm_bf16": (I32, [P, P, I64, I64, I64, F, P, P]),
         "fpq_transpose_bf16": (I32, [P, P, I64, I64, P]),
         "fpq_gemm_bf16_layout": (I32, [P, I32, P, I32, I64, I64, I64, F, P, P]),
+        "fpq_gemm_bf16_splitk_workspace_bytes": (SZ, [I64, I64, I64]),
+        "fpq_gemm_bf16_splitk": (I32, [P, I32, P, I32, I64, I64, I64, F, P, P, SZ, P]),
         "fpq_qat_backward_workspace_bytes": (SZ, [I64, I64, I64, I32]),
         "fpq_qat_backward": (I32, [P, P, P, P, P, I64, I64, I64, I32, F, P, P, P, P, P, SZ, P]),
         "fpq_quantize_nvfp4_noalloc": (I32, [P, I64, I64, I64, P, P, P, P]),
@@ -155,6 +157,17 @@ def fpq_gemm_bf16(p, q, m, n, k, alpha, c, stream=None):
 def fpq_gemm_bf16_layout(p, p_mn, q, q_mn, m, n, k, alpha, c, stream=None):
     _check(load().fpq_gemm_bf16_layout(_ptr(p), int(p_mn), _ptr(q), int(q_mn), m, n, k, float(alpha), _ptr(c),
                                        _stream(stream)), "fpq_gemm_bf16_layout")
+
+
+def fpq_gemm_bf16_splitk_workspace_bytes(m: int, n: int, k: int) -> int:
+    return load().fpq_gemm_bf16_splitk_workspace_bytes(m, n, k)
+
+
+def fpq_gemm_bf16_splitk(p, p_mn, q, q_mn, m, n, k, alpha, c, workspace, stream=None):
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().fpq_gemm_bf16_splitk(_ptr(p), int(p_mn), _ptr(q), int(q_mn), m, n, k, float(alpha), _ptr(c),
+                                       _ptr(workspace) if workspace is not None else None, wsb, _stream(stream)),
+           "fpq_gemm_bf16_splitk")
 
 
 def fpq_transpose_bf16(x, out, rows, cols, stream=None):

@@ -266,6 +266,35 @@ fpq_status fpq_gemm_bf16_layout(const void* p, int32_t p_mn, const void* q, int3
                      "bf16 gemm launch");
 }
 
+size_t fpq_gemm_bf16_splitk_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+    if (m < 1 || n < 1 || k < 1) return 0;
+    return (size_t)fpq::kMaxSplits * (size_t)m * (size_t)n * 4;
+}
+
+fpq_status fpq_gemm_bf16_splitk(const void* p, int32_t p_mn, const void* q, int32_t q_mn, int64_t m, int64_t n,
+                                int64_t k, float alpha, void* c, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (m < 1 || n < 8 || n % 8 || k < 8 || k % 8 || (p_mn && m % 8) || m > (1 << 30) || n > (1 << 30) ||
+        k > (1 << 30) || (p_mn != 0 && p_mn != 1) || (q_mn != 0 && q_mn != 1)) {
+        set_detail("need n, k positive multiples of 8, m >= 1 (a multiple of 8 when P is MN-major), flags 0|1");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if ((st = check_ptrs({p, q, c})) != FPQ_OK) return st;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < fpq_gemm_bf16_splitk_workspace_bytes(m, n, k)) {
+        set_detail("need a 16-byte aligned workspace of fpq_gemm_bf16_splitk_workspace_bytes() bytes");
+        return FPQ_ERR_WORKSPACE;
+    }
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_gemm_bf16_splitk(p, p_mn != 0, q, q_mn != 0, m, n, k, alpha, c,
+                                                  static_cast<float*>(workspace),
+                                                  fpq::bf16_split_count(m, n, k, d->sms), d->err,
+                                                  (cudaStream_t)stream),
+                     "bf16 split-k gemm launch");
+}
+
 fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, int64_t cols, void* stream) {
     t_detail[0] = 0;
     fpq_status st;
@@ -304,7 +333,7 @@ fpq_status fpq_qat_backward(const void* dy, const void* x_fq, const void* w_fq, 
     const DeviceState* d = device_state(&st);
     if (!d) return st;
     return from_cuda(fpq::launch_qat_backward(dy, x_fq, w_fq, lora_a, lora_b, m, n, k, r, alpha_over_r, dx, dw, da,
-                                              db, workspace, d->err, (cudaStream_t)stream),
+                                              db, workspace, d->err, d->sms, (cudaStream_t)stream),
                      "qat backward launch");
 }
 

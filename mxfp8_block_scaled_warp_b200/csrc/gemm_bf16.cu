@@ -25,6 +25,8 @@
 // kernel records FPQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
 #include <cuda.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -41,7 +43,7 @@ constexpr int STAGES = 4;
 constexpr int A_TILE = BM * BK * 2, B_TILE = BN * BK * 2;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr int NUM_THREADS = 256;
-constexpr int EPI_WARP_BYTES = 32 * 128 * 2;        // a warp's 32 x 128 block of C, bf16
+constexpr int EPI_WARP_BYTES = 32 * 128 * 4;        // a warp's 32 x 128 block of C (fp32 partials: 16 KB)
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 constexpr int MN_BOX = 64 * BK * 2;                 // one MN-major box: 64 rows-of-the-product x 64 K
@@ -99,18 +101,25 @@ __device__ bool wait_or_timeout(uint64_t* bar, uint32_t parity, uint32_t* err) {
     }
 }
 
+// Split-K (partial != nullptr): CTA b takes tile b / splits and the K tiles
+// [kts (b % splits), kts (b % splits + 1)) and writes its fp32 sums, without
+// alpha, to partial[b % splits][M][N] (rows past M and columns past N
+// skipped); reduce_partials_kernel adds the slices in order.
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmC, int64_t M, int64_t N, int64_t K, float alpha,
-                 uint32_t* err) {
+                 uint32_t* err, float* __restrict__ partial, int splits, int kts) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = (int)((N + BN - 1) / BN);
-    const int mt = blockIdx.x / n_tiles, nt = blockIdx.x - mt * n_tiles;
+    const int tile = (int)blockIdx.x / splits, split = (int)blockIdx.x - tile * splits;
+    const int mt = tile / n_tiles, nt = tile - mt * n_tiles;
     const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
-    const int KT = (int)((K + BK - 1) / BK);
+    const int KT_all = (int)((K + BK - 1) / BK);
+    const int kt0 = partial ? split * kts : 0;
+    const int KT = partial ? min(KT_all, kt0 + kts) - kt0 : KT_all;     // >= 1 by the launcher's choice
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -140,19 +149,20 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
                 if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err)) break;
                 mbar_arrive_expect_tx(&sm.full[s], A_TILE + B_TILE);
+                const int kk = (kt0 + kt) * BK;
                 if (A_MN) {
 #pragma unroll
                     for (int j = 0; j < BM / 64; ++j)
-                        tma_load_2d(sm.a[s] + j * MN_BOX, &tmA, &sm.full[s], (int32_t)(m0 + 64 * j), kt * BK);
+                        tma_load_2d(sm.a[s] + j * MN_BOX, &tmA, &sm.full[s], (int32_t)(m0 + 64 * j), kk);
                 } else {
-                    tma_load_2d(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)m0);
+                    tma_load_2d(sm.a[s], &tmA, &sm.full[s], kk, (int32_t)m0);
                 }
                 if (B_MN) {
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)
-                        tma_load_2d(sm.b[s] + j * MN_BOX, &tmB, &sm.full[s], (int32_t)(n0 + 64 * j), kt * BK);
+                        tma_load_2d(sm.b[s] + j * MN_BOX, &tmB, &sm.full[s], (int32_t)(n0 + 64 * j), kk);
                 } else {
-                    tma_load_2d(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)n0);
+                    tma_load_2d(sm.b[s], &tmB, &sm.full[s], kk, (int32_t)n0);
                 }
             }
         }
@@ -189,6 +199,24 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int c = 0; c < 4; ++c)
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half + 32 * c), r[c]);
             tmem_ld_wait();
+            if (partial) {
+                // fp32 sums staged row-major (512-byte rows, 16-byte chunk x of
+                // row l at position x ^ l), then written a row at a time
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(stage + lane * 512 + 16 * ((8 * c + j) ^ lane)) =
+                            make_uint4(r[c][4 * j], r[c][4 * j + 1], r[c][4 * j + 2], r[c][4 * j + 3]);
+                __syncwarp();
+                float* out = partial + (int64_t)split * M * N;
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int64_t row = row0 + rr, col = col0 + 4 * lane;
+                    if (row < M && col < N)
+                        st_v4(out + row * N + col, *reinterpret_cast<const uint4*>(stage + rr * 512 + 16 * (lane ^ rr)));
+                }
+                __syncwarp();
+            } else {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -211,6 +239,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 bulk_wait_group_read0();     // the staging must stay valid until read
             }
             __syncwarp();
+            }
         }
     }
 
@@ -224,9 +253,30 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
 int smem_bytes() { return (int)sizeof(Smem) + 1024; }
 
+// out[i] = bf16(alpha * sum_s part[s][i]), s ascending; four elements per
+// thread (count is a multiple of 4).
+__global__ void __launch_bounds__(256)
+reduce_partials_kernel(const float4* __restrict__ part, int splits, int64_t count4, float alpha,
+                       uint2* __restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < count4; i += (int64_t)gridDim.x * 256) {
+        float4 acc = __ldcg(part + i);
+        for (int s = 1; s < splits; ++s) {
+            const float4 v = __ldcg(part + s * count4 + i);
+            acc.x = __fadd_rn(acc.x, v.x);
+            acc.y = __fadd_rn(acc.y, v.y);
+            acc.z = __fadd_rn(acc.z, v.z);
+            acc.w = __fadd_rn(acc.w, v.w);
+        }
+        out[i] = make_uint2(f32x2_to_bf16x2(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha)),
+                            f32x2_to_bf16x2(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha)));
+    }
+}
+
 template <bool A_MN, bool B_MN>
 cudaError_t launch_t(const void* p, const void* q, int64_t m, int64_t n, int64_t k, float alpha, void* c,
-                     uint32_t* err, cudaStream_t st) {
+                     uint32_t* err, float* partial, int splits, int kts, cudaStream_t st) {
     static int configured[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -253,19 +303,48 @@ cudaError_t launch_t(const void* p, const void* q, int64_t m, int64_t n, int64_t
     e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)m, (uint64_t)n, (uint64_t)n * 2, 32, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
+    const int64_t grid = ((m + BM - 1) / BM) * ((n + BN - 1) / BN) * splits;
     return launch_pdl(gemm_bf16_kernel<A_MN, B_MN>, dim3((unsigned)grid), dim3(NUM_THREADS), smem_bytes(), st, ta,
-                      tb, tc, m, n, k, alpha, err);
+                      tb, tc, m, n, k, alpha, err, partial, splits, kts);
 }
 
 }  // namespace
 
+namespace {
+cudaError_t launch_any(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n, int64_t k,
+                       float alpha, void* c, uint32_t* err, float* partial, int splits, int kts, cudaStream_t st) {
+    if (p_mn) return q_mn ? launch_t<true, true>(p, q, m, n, k, alpha, c, err, partial, splits, kts, st)
+                          : launch_t<true, false>(p, q, m, n, k, alpha, c, err, partial, splits, kts, st);
+    return q_mn ? launch_t<false, true>(p, q, m, n, k, alpha, c, err, partial, splits, kts, st)
+                : launch_t<false, false>(p, q, m, n, k, alpha, c, err, partial, splits, kts, st);
+}
+}  // namespace
+
 cudaError_t launch_gemm_bf16(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n, int64_t k,
                              float alpha, void* c, uint32_t* err, cudaStream_t st) {
-    if (p_mn) return q_mn ? launch_t<true, true>(p, q, m, n, k, alpha, c, err, st)
-                          : launch_t<true, false>(p, q, m, n, k, alpha, c, err, st);
-    return q_mn ? launch_t<false, true>(p, q, m, n, k, alpha, c, err, st)
-                : launch_t<false, false>(p, q, m, n, k, alpha, c, err, st);
+    return launch_any(p, p_mn, q, q_mn, m, n, k, alpha, c, err, nullptr, 1, 0, st);
+}
+
+int bf16_split_count(int64_t m, int64_t n, int64_t k, int sms) {
+    const int64_t tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
+    const int64_t kt = (k + BK - 1) / BK;
+    int64_t splits = (int64_t)sms / tiles;                            // one wave (one CTA per SM)
+    splits = std::min<int64_t>(splits, std::min<int64_t>(kMaxSplits, kt / 2));   // at least two K tiles each
+    return (int)std::max<int64_t>(splits, 1);
+}
+
+cudaError_t launch_gemm_bf16_splitk(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n,
+                                    int64_t k, float alpha, void* c, float* partial, int splits, uint32_t* err,
+                                    cudaStream_t st) {
+    const int64_t kt = (k + BK - 1) / BK;
+    const int kts = (int)((kt + splits - 1) / splits);
+    splits = (int)((kt + kts - 1) / kts);                             // every slice non-empty
+    cudaError_t e = launch_any(p, p_mn, q, q_mn, m, n, k, alpha, c, err, partial, splits, kts, st);
+    if (e != cudaSuccess) return e;
+    const int64_t count4 = m * n / 4;
+    const int grid = (int)std::min<int64_t>((count4 + 255) / 256, 1184);
+    return launch_pdl(reduce_partials_kernel, dim3((unsigned)grid), dim3(256), 0, st, (const float4*)partial, splits,
+                      count4, alpha, (uint2*)c);
 }
 
 }  // namespace fpq

@@ -44,6 +44,15 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
 cudaError_t launch_gemm_bf16(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n, int64_t k,
                              float alpha, void* c, uint32_t* err, cudaStream_t st);
 
+// Split-K variant for products with few output tiles: fp32 partial sums of
+// `splits` K slices in `partial` ([splits, m, n] fp32), then a reduce kernel
+// writes bf16(alpha * sum) to c; m * n a multiple of 4.
+constexpr int kMaxSplits = 16;
+int bf16_split_count(int64_t m, int64_t n, int64_t k, int sms);
+cudaError_t launch_gemm_bf16_splitk(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n,
+                                    int64_t k, float alpha, void* c, float* partial, int splits, uint32_t* err,
+                                    cudaStream_t st);
+
 // bf16 [R, C] -> [C, R] (R, C multiples of 8).
 cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st);
 
@@ -52,7 +61,8 @@ cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t 
 size_t qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t r);
 cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
                                 const void* lora_b, int64_t m, int64_t n, int64_t k, int64_t r, float alpha_over_r,
-                                void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, cudaStream_t st);
+                                void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, int sms,
+                                cudaStream_t st);
 
 cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void* bq,
                                       const void* bs, const int32_t* offsets, int groups,

@@ -71,22 +71,33 @@ cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t 
     return launch_pdl(transpose_bf16_kernel, grid, dim3(256), 0, st, (const uint16_t*)in, (uint16_t*)out, R, C);
 }
 
-// No workspace: every operand is read in the layout it is stored in (the
-// GEMM takes K-major or MN-major operands).
-size_t qat_backward_workspace_bytes(int64_t, int64_t, int64_t, int64_t) { return 0; }
+// The skinny products dA [r, k] and dB [n, r] have few output tiles (r is
+// at most 256), so they split their contraction over the SMs and add fp32
+// partial sums in a second kernel; the workspace holds those partials (at
+// most kMaxSplits slices of each).  Every operand is read in the layout it
+// is stored in (the GEMM takes K-major or MN-major operands).
+size_t qat_backward_workspace_bytes(int64_t, int64_t n, int64_t k, int64_t r) {
+    return round_up((size_t)kMaxSplits * (size_t)(r * k) * 4) + round_up((size_t)kMaxSplits * (size_t)(n * r) * 4);
+}
 
 cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
                                 const void* lora_b, int64_t m, int64_t n, int64_t k, int64_t r, float alpha_over_r,
-                                void* dx, void* dw, void* da, void* db, void*, uint32_t* err, cudaStream_t st) {
+                                void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, int sms,
+                                cudaStream_t st) {
     cudaError_t e;
+    float* part_a = static_cast<float*>(ws);
+    float* part_b = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round_up((size_t)kMaxSplits * (size_t)(r * k) * 4));
     // dX [m, k] = dY Wfq: contraction over n; dY [m, n] K-major, Wfq [n, k] MN-major
     if ((e = launch_gemm_bf16(dy, false, w_fq, true, m, k, n, 1.0f, dx, err, st)) != cudaSuccess) return e;
     // dW [n, k] = dY^T Xfq: contraction over m; dY [m, n] and Xfq [m, k] MN-major
     if ((e = launch_gemm_bf16(dy, true, x_fq, true, n, k, m, 1.0f, dw, err, st)) != cudaSuccess) return e;
     // dA [r, k] = (alpha / r) B^T dW: contraction over n; B [n, r] and dW [n, k] MN-major
-    if ((e = launch_gemm_bf16(lora_b, true, dw, true, r, k, n, alpha_over_r, da, err, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm_bf16_splitk(lora_b, true, dw, true, r, k, n, alpha_over_r, da, part_a,
+                                     bf16_split_count(r, k, n, sms), err, st)) != cudaSuccess)
+        return e;
     // dB [n, r] = (alpha / r) dW A^T: contraction over k; dW [n, k] and A [r, k] K-major
-    return launch_gemm_bf16(dw, false, lora_a, false, n, r, k, alpha_over_r, db, err, st);
+    return launch_gemm_bf16_splitk(dw, false, lora_a, false, n, r, k, alpha_over_r, db, part_b,
+                                   bf16_split_count(n, r, k, sms), err, st);
 }
 
 }  // namespace fpq

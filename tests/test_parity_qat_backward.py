@@ -137,3 +137,61 @@ def test_qat_backward_rejects_bad_args(fpq):
     big = torch.zeros(4096 + 8, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(fpq.FpqError):       # misaligned operand
         fpq.fpq_qat_backward(big[1:4097].view(64, 64), t, t, t, t, 64, 64, 64, 8, 1.0, t, t, t, t, None)
+
+
+def _splitk(fpq, ps, p_mn, qs, q_mn, m, n, k, alpha):
+    c = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((fpq.fpq_gemm_bf16_splitk_workspace_bytes(m, n, k),), dtype=torch.uint8, device="cuda")
+    fpq.fpq_gemm_bf16_splitk(ps, p_mn, qs, q_mn, m, n, k, alpha, c, ws)
+    return c
+
+
+@pytest.mark.parametrize("p_mn,q_mn", [(False, False), (True, True), (False, True)])
+@pytest.mark.parametrize("m,n,k", [(16, 7168, 2048), (2048, 16, 7168), (8, 8, 8), (24, 520, 1000),
+                                   (200, 16, 1064), (16, 136, 8200)])
+def test_gemm_bf16_splitk(fpq, orc, p_mn, q_mn, m, n, k):
+    """Few output tiles, long contraction: the K slices' fp32 partial sums
+    are added by a second kernel; ragged K tails land in the last slice."""
+    if p_mn and m % 8:
+        pytest.skip("MN-major P needs m a multiple of 8")
+    p, q = rand((m, k), 940 + m), rand((n, k), 941 + n, std=0.05)
+    ref = orc.gemm_bf16_full(p, q, 2.0)
+    ps = np.ascontiguousarray(p.T) if p_mn else p
+    qs = np.ascontiguousarray(q.T) if q_mn else q
+    c = _splitk(fpq, dev(ps), p_mn, dev(qs), q_mn, m, n, k, 2.0)
+    check(c, ref, orc, f"bf16 split-k {p_mn}{q_mn} {m}x{n}x{k}")
+    assert fpq.fpq_get_device_error() == 0
+
+
+def test_gemm_bf16_splitk_integer_exact(fpq, orc):
+    """Entries in {-1, 0, 1} with K = 4096 (up to 16 slices of the
+    contraction): every partial sum is an integer below 2^24, so the fp32
+    slice sums and their total are exact, and C must be the round-to-
+    nearest-even bf16 of alpha times the exact integer sum; a slice lost or
+    added twice changes it."""
+    rng = np.random.default_rng(32)
+    m, n, k = 16, 512, 4096
+    ip, iq = rng.integers(-1, 2, (m, k)), rng.integers(-1, 2, (n, k))
+    p = workloads.as_u16(torch.from_numpy(ip.astype(np.float32)).to(torch.bfloat16))
+    q = workloads.as_u16(torch.from_numpy(iq.astype(np.float32)).to(torch.bfloat16))
+    c = _splitk(fpq, dev(p), False, dev(q), False, m, n, k, 0.25)
+    ref = orc.bf16_round(0.25 * (ip @ iq.T).astype(np.float64))       # bf16 bit patterns
+    assert np.array_equal(workloads.as_u16(c), ref)
+
+
+def test_gemm_bf16_splitk_repeatable(fpq):
+    """The slices are added in a fixed order: two runs agree bit for bit."""
+    m, n, k = 16, 7168, 2048
+    p, q = dev(rand((k, m), 960)), dev(rand((k, n), 961, std=0.05))
+    c1 = _splitk(fpq, p, True, q, True, m, n, k, 2.0)
+    c2 = _splitk(fpq, p, True, q, True, m, n, k, 2.0)
+    assert torch.equal(c1.view(torch.int16), c2.view(torch.int16))
+
+
+def test_gemm_bf16_splitk_rejects_small_workspace(fpq):
+    t = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((fpq.fpq_gemm_bf16_splitk_workspace_bytes(64, 64, 64) - 16,), dtype=torch.uint8, device="cuda")
+    with pytest.raises(fpq.FpqError):
+        fpq.fpq_gemm_bf16_splitk(t, 0, t, 0, 64, 64, 64, 1.0, t, ws)
+    with pytest.raises(fpq.FpqError):
+        fpq.fpq_gemm_bf16_splitk(t, 0, t, 0, 64, 64, 64, 1.0, t, None)
