@@ -117,13 +117,41 @@ class Step:
         """Work of one step in the unit's numerator (flops, or bytes for GB/s)."""
         return self.flops
 
+    # kernels that depend on nothing earlier in the step and run on a second
+    # stream in the timed step, joined back before `join_before`
+    side = ()
+    join_before = ""
+
     def kernels(self):  # list of (label, callable)
         raise NotImplementedError
+
+    def whole_step(self, side_stream):
+        """One step as the timed graph and the end-to-end loop run it: the
+        kernels named in `side` forked onto `side_stream` (they overlap the
+        others' ramp-up and tail), the rest in order on the current stream."""
+        cur = torch.cuda.current_stream()
+        forked = False
+        for name, fn in self.kernels():
+            if name in self.side:
+                if not forked:
+                    side_stream.wait_stream(cur)
+                    forked = True
+                with torch.cuda.stream(side_stream):
+                    fn()
+                continue
+            if forked and name == self.join_before:
+                cur.wait_stream(side_stream)
+                forked = False
+            fn()
+        if forked:
+            cur.wait_stream(side_stream)
 
 
 class DsFp8Gemm(Step):
     name = "ds_fp8_gemm"
     dominant = "gemm_fp8_f32scale"
+    side = ("quant_fp8_128x128",)      # B's quantizer runs beside A's
+    join_before = "gemm_fp8_f32scale"
 
     def __init__(self, fpq, dev, m=4096, n=2048, k=7168):
         self.f = fpq
@@ -161,13 +189,12 @@ class DsFp8Gemm(Step):
         return {"quant_fp8_1x128": ("GB/s", self.qa_bytes), "quant_fp8_128x128": ("GB/s", self.qb_bytes),
                 "gemm_fp8_f32scale": ("TFLOP/s", self.flops)}
 
-    def e2e_step(self, stream):
+    def e2e_step(self, stream, side_stream):
         """Host buffers in, host buffer out: the same step through the C ABI
         with the copies inside the timed region."""
         self.a.copy_(self.a_host, non_blocking=True)
         self.b.copy_(self.b_host, non_blocking=True)
-        for _, fn in self.kernels():
-            fn()
+        self.whole_step(side_stream)
         self.c_host.copy_(self.c, non_blocking=True)
         return self.a_host.numel() * 2 + self.b_host.numel() * 2, self.c.numel() * 2
 
@@ -212,7 +239,7 @@ class MoeGrouped(Step):
     def kernel_work(self):
         return {"quant_mxfp8": ("GB/s", self.qx_bytes), "gemm_grouped_mxfp8": ("TFLOP/s", self.flops)}
 
-    def e2e_step(self, stream):
+    def e2e_step(self, stream, side_stream):
         """Permuted tokens and the group offsets from pinned host memory in,
         the expert outputs back to pinned host memory, copies inside the
         timed region (the expert weights stay resident: serving)."""
@@ -231,6 +258,8 @@ class MoeGrouped(Step):
 class QatForward(Step):
     name = "qat_forward"
     dominant = "gemm_fp8_f32scale"
+    side = ("lora_merge_fq",)          # the weight merge runs beside X's quantizer
+    join_before = "gemm_fp8_f32scale"
 
     def __init__(self, fpq, dev):
         self.f = fpq
@@ -266,7 +295,7 @@ class QatForward(Step):
         return {"lora_merge_fq": ("GB/s", self.merge_bytes), "quant_fp8_1x128": ("GB/s", self.xq_bytes),
                 "gemm_fp8_f32scale": ("TFLOP/s", self.flops)}
 
-    def e2e_step(self, stream):
+    def e2e_step(self, stream, side_stream):
         """Base weight, LoRA factors and activations from pinned host memory
         in, the GEMM output back to pinned host memory, copies inside the
         timed region."""
@@ -275,8 +304,7 @@ class QatForward(Step):
             self.c_host = torch.empty(self.c.shape, dtype=self.c.dtype).pin_memory()
         for d, h in zip((self.w, self.la, self.lb, self.x), self.host):
             d.copy_(h, non_blocking=True)
-        for _, fn in self.kernels():
-            fn()
+        self.whole_step(side_stream)
         self.c_host.copy_(self.c, non_blocking=True)
         return sum(h.numel() * 2 for h in self.host), self.c.numel() * 2
 
@@ -287,6 +315,7 @@ class MoePrequant(Step):
     one batched call, to MXFP8 (1x32, E8M0) and to NVFP4 (1x16 E4M3 + a
     per-matrix fp32 scale).  The step's work is the algorithmic bytes."""
     name = "moe_prequant"
+    side = ("quant_nvfp4",)            # the two formats of a matrix are independent
     dominant = "quant_nvfp4"
     unit = "GB/s"
     dtype = "bf16 -> e4m3 / e2m1 codes (fp32 scale arithmetic)"
@@ -342,7 +371,7 @@ class MoePrequant(Step):
     def kernel_work(self):
         return {"quant_mxfp8": ("GB/s", self.mx_bytes), "quant_nvfp4": ("GB/s", self.nv_bytes)}
 
-    def e2e_step(self, stream):
+    def e2e_step(self, stream, side_stream):
         """bf16 expert stacks in pinned host memory in, every code and scale
         back to pinned host memory, copies inside the timed region."""
         if not self.host:
@@ -417,12 +446,18 @@ class QatBackward(Step):
             ("gemm_bf16_db", lambda: f.fpq_gemm_bf16_splitk(self.dw, 0, self.a, 0, n, r, k, aor, self.db, self.ws_b)),
         ]
 
+    def whole_step(self, side_stream):
+        """The public call: dX on the library's second stream beside dW."""
+        f = self.f
+        f.fpq_qat_backward(self.dy, self.x_fq, self.w_fq, self.a, self.b, self.m, self.n, self.k, self.r, self.aor,
+                           self.dx, self.dw, self.da, self.db, self.ws)
+
     def kernel_work(self):
         m, n, k, r = self.m, self.n, self.k, self.r
         return {"gemm_bf16_dx": ("TFLOP/s", 2.0 * m * n * k), "gemm_bf16_dw": ("TFLOP/s", 2.0 * m * n * k),
                 "gemm_bf16_da": ("TFLOP/s", 2.0 * r * n * k), "gemm_bf16_db": ("TFLOP/s", 2.0 * r * n * k)}
 
-    def e2e_step(self, stream):
+    def e2e_step(self, stream, side_stream):
         """dy from pinned host memory, the public fpq_qat_backward call, dx,
         dA and dB back to pinned host memory (dW_eff stays on the device)."""
         f = self.f
@@ -485,7 +520,7 @@ class Nvfp4Gemm(Step):
         return {"quant_nvfp4_a": ("GB/s", self.qa_bytes), "quant_nvfp4_b": ("GB/s", self.qb_bytes),
                 "gemm_nvfp4": ("TFLOP/s", self.flops)}
 
-    def e2e_step(self, stream):
+    def e2e_step(self, stream, side_stream):
         self.a.copy_(self.a_host, non_blocking=True)
         self.b.copy_(self.b_host, non_blocking=True)
         for _, fn in self.kernels():
@@ -696,6 +731,16 @@ def whole_job_rate(world: int, work_per_rank_step: float, steps: int, total_ms: 
 METRIC = "quantize GB/s vs HBM peak; block-scaled FP8 GEMM TFLOPS vs FP8 tensor peak"
 
 
+def launch_note(step) -> str:
+    fork = ""
+    if step.side:
+        fork = f" ({', '.join(step.side)} on a second stream beside the kernels before {step.join_before})"
+    elif type(step).whole_step is not Step.whole_step:
+        fork = f" ({' '.join((type(step).whole_step.__doc__ or '').split())})"
+    return (f"CUDA graph of the step replayed per timed step{fork}; per-kernel times from a second graph with "
+            f"events around each kernel, one after another")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -725,6 +770,8 @@ def main():
     kern = step.kernels()
     names = [n for n, _ in kern]
 
+    side_stream = torch.cuda.Stream()
+
     def one_step(events=None):
         for i, (_, fn) in enumerate(kern):
             if events is not None:
@@ -744,8 +791,9 @@ def main():
     # graphs of the same launches: `whole` records events only before the
     # first and after the last kernel, so consecutive kernels keep their
     # programmatic-dependent-launch overlap (the step time and the headline
-    # value come from it); `split` records events around every kernel (the
-    # per-kernel times and the roofline come from it).  The L2 flush runs
+    # value come from it; independent kernels may run on a second stream
+    # there); `split` records events around every kernel, one after another
+    # (the per-kernel times and the roofline come from it).  The L2 flush runs
     # outside the graphs before every replay; each replay's events are read
     # before the next replay overwrites them.
     def capture(events_per_kernel):
@@ -760,7 +808,7 @@ def main():
                     one_step(ev)
                 else:
                     ev[0][0].record()
-                    one_step()
+                    step.whole_step(side_stream)
                     ev[0][1].record()
         stream.wait_stream(cap)
         return g, ev
@@ -847,13 +895,13 @@ def main():
     e2e = None
     if hasattr(step, "e2e_step"):
         for _ in range(2):
-            step.e2e_step(stream)
+            step.e2e_step(stream, side_stream)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = max(3, min(args.steps, 20))
         e0.record(stream)
         for _ in range(reps):
-            hb, db = step.e2e_step(stream)
+            hb, db = step.e2e_step(stream, side_stream)
         e1.record(stream)
         e1.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / reps, pg, dev)
@@ -867,7 +915,7 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": step.unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": step.dtype, "data": "synthetic",
-            "config": dict(step.config, launch="CUDA graph of the step replayed per timed step; per-kernel times from a second graph with events around each kernel"), "quantize_gbs": quant_gbs,
+            "config": dict(step.config, launch=launch_note(step)), "quantize_gbs": quant_gbs,
             "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"] if quant_gbs is not None else None,
             "kernels": kernels_out, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.launches * args.steps, "clocks": clk.summary(), "clocks_kernel_timing": ck,

@@ -290,6 +290,11 @@ FPQ_API fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, i
  *               contraction across the SMs (at most 16 slices each, added in
  *               slice order by a second kernel, so results are repeatable)
  *
+ * The products are ordered on `stream` like any other work: dx, which no
+ * other product needs, runs on a library-owned second stream forked from
+ * `stream` by an event and joined back before the call returns (so the call
+ * may also be captured into a CUDA graph).
+ *
  * Requires m, n, k positive multiples of 8 and r a multiple of 8 in [8, 256];
  * every pointer 16-byte aligned.  Errors: FPQ_ERR_INVALID_ARG,
  * FPQ_ERR_ALIGNMENT, FPQ_ERR_WORKSPACE, FPQ_ERR_CUDA; device-side wait

@@ -15,6 +15,8 @@
 // utility.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -64,6 +66,33 @@ transpose_bf16_kernel(const uint16_t* __restrict__ in, uint16_t* __restrict__ ou
 
 inline size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
 
+// A second stream per device for the fork below, with the two events of
+// the fork and the join; created on first use.  The fork-join section holds
+// the mutex, so concurrent callers never interleave records and waits on
+// the shared events.
+constexpr int kForkDevices = 64;
+struct Fork {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+Fork g_fork[kForkDevices];
+std::mutex g_fork_mu;
+
+cudaError_t fork_state(Fork** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kForkDevices) return cudaErrorInvalidDevice;
+    Fork& f = g_fork[dev];
+    if (!f.side) {
+        if ((e = cudaStreamCreateWithFlags(&f.side, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&f.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&f.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    *out = &f;
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st) {
@@ -84,20 +113,34 @@ cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_
                                 const void* lora_b, int64_t m, int64_t n, int64_t k, int64_t r, float alpha_over_r,
                                 void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, int sms,
                                 cudaStream_t st) {
-    cudaError_t e;
     float* part_a = static_cast<float*>(ws);
     float* part_b = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round_up((size_t)kMaxSplits * (size_t)(r * k) * 4));
-    // dX [m, k] = dY Wfq: contraction over n; dY [m, n] K-major, Wfq [n, k] MN-major
-    if ((e = launch_gemm_bf16(dy, false, w_fq, true, m, k, n, 1.0f, dx, err, st)) != cudaSuccess) return e;
+    // dX does not depend on the other three products: it runs on a second
+    // stream, forked from and joined back into st, so that its tiles fill
+    // the SMs that dW's last partial wave leaves idle.  Works under stream
+    // capture (the fork and join become graph edges).
+    std::lock_guard<std::mutex> lock(g_fork_mu);
+    Fork* f = nullptr;
+    cudaError_t e = fork_state(&f);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaEventRecord(f->fork, st)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(f->side, f->fork, 0)) != cudaSuccess) return e;
     // dW [n, k] = dY^T Xfq: contraction over m; dY [m, n] and Xfq [m, k] MN-major
-    if ((e = launch_gemm_bf16(dy, true, x_fq, true, n, k, m, 1.0f, dw, err, st)) != cudaSuccess) return e;
+    e = launch_gemm_bf16(dy, true, x_fq, true, n, k, m, 1.0f, dw, err, st);
+    // dX [m, k] = dY Wfq: contraction over n; dY [m, n] K-major, Wfq [n, k] MN-major
+    if (e == cudaSuccess) e = launch_gemm_bf16(dy, false, w_fq, true, m, k, n, 1.0f, dx, err, f->side);
     // dA [r, k] = (alpha / r) B^T dW: contraction over n; B [n, r] and dW [n, k] MN-major
-    if ((e = launch_gemm_bf16_splitk(lora_b, true, dw, true, r, k, n, alpha_over_r, da, part_a,
-                                     bf16_split_count(r, k, n, sms), err, st)) != cudaSuccess)
-        return e;
+    if (e == cudaSuccess)
+        e = launch_gemm_bf16_splitk(lora_b, true, dw, true, r, k, n, alpha_over_r, da, part_a,
+                                    bf16_split_count(r, k, n, sms), err, st);
     // dB [n, r] = (alpha / r) dW A^T: contraction over k; dW [n, k] and A [r, k] K-major
-    return launch_gemm_bf16_splitk(dw, false, lora_a, false, n, r, k, alpha_over_r, db, part_b,
-                                   bf16_split_count(n, r, k, sms), err, st);
+    if (e == cudaSuccess)
+        e = launch_gemm_bf16_splitk(dw, false, lora_a, false, n, r, k, alpha_over_r, db, part_b,
+                                    bf16_split_count(n, r, k, sms), err, st);
+    // the join is made on every path, so a capture is never left forked
+    cudaError_t j = cudaEventRecord(f->join, f->side);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(st, f->join, 0);
+    return e != cudaSuccess ? e : j;
 }
 
 }  // namespace fpq
