@@ -6,8 +6,9 @@ benchmark's CPU-baseline leg may import this package.  It shares no code with
 the CUDA library (``mxfp8_block_scaled_warp_b200``) and never imports it; the
 CUDA library never imports this package.
 
-All arithmetic lives in ``oracle.c`` (plain C, no fast-math, no FMA
-contraction); this module only marshals numpy arrays into it.  What each
+All floating-point arithmetic lives in ``oracle.c`` (plain C, no fast-math,
+no FMA contraction); this module marshals numpy arrays into it, and holds
+the integer bookkeeping of the MoE dispatch (which rows go where).  What each
 function computes, and which page passage it follows, is stated in
 ``oracle.c``.
 
@@ -365,3 +366,71 @@ def qat_backward(dy, x_fq, w_fq, lora_a, lora_b, alpha_over_r: float):
     da = gemm_bf16_full(np.ascontiguousarray(lora_b.T), np.ascontiguousarray(dw16.T), alpha_over_r)
     db = gemm_bf16_full(dw16, lora_a, alpha_over_r)
     return dx, dw, da, db
+
+
+# ------------------------------------------------------------- MoE FP8 dispatch
+#
+# "DeepSeek-V3 Blog 5: Low-Precision Training", Reducing Communication
+# Overhead in MoE with FP8: token activations are quantized to FP8 before
+# they are sent to the GPUs that hold their experts.  The format is MXFP8
+# (E4M3 codes, E8M0 scale per 32 elements), the input format of the grouped
+# expert GEMM.  Only the bookkeeping below is written in Python (integers and
+# data movement); every code and scale comes from quant_mxfp8 above.
+#
+# Reading of the order (the page fixes none): rank r of `world` owns experts
+# [r L, (r + 1) L), L = E / world; its receive buffer holds the rows of its
+# local experts in expert order, each expert's rows from source rank 0, 1, ...
+# in turn, and within one source the pairs (token t, choice j) routed to that
+# expert in token order, then choice order.
+
+
+def moe_route_plan(topk_ids: np.ndarray, num_experts: int):
+    """counts[e] = number of (token, choice) pairs routed to expert e, and
+    slot[t, j] = the index of pair (t, j) among them, pairs numbered in token
+    order, then choice order."""
+    ids = np.asarray(topk_ids)
+    tokens, k = ids.shape
+    counts = np.zeros(num_experts, np.int64)
+    slot = np.zeros((tokens, k), np.int64)
+    for t in range(tokens):
+        for j in range(k):
+            e = int(ids[t, j])
+            slot[t, j] = counts[e]
+            counts[e] += 1
+    return counts, slot
+
+
+def moe_dispatch(xs, topk_ids_list, num_experts: int):
+    """The FP8 dispatch over len(xs) ranks: xs[s] bf16 [T_s, K] (uint16) and
+    topk_ids_list[s] int [T_s, k] are source rank s's activations and routing.
+    Returns, per receiving rank r, (codes uint8 [rows_r, K], scales uint8 E8M0
+    [rows_r, K/32], group_offsets int64 [L + 1]) with rows ordered as stated
+    above; group_offsets[l] is the first row of local expert l."""
+    world = len(xs)
+    assert num_experts % world == 0
+    L = num_experts // world
+    quant = [quant_mxfp8(_bf16(x)) for x in xs]
+    plans = [moe_route_plan(ids, num_experts) for ids in topk_ids_list]
+    out = []
+    for r in range(world):
+        rows_q, rows_s, offsets = [], [], [0]
+        for l in range(L):
+            e = r * L + l
+            for s in range(world):
+                ids = np.asarray(topk_ids_list[s])
+                _, slot = plans[s]
+                # pairs of source s routed to e, placed by their slot
+                seg = [None] * int(plans[s][0][e])
+                for t in range(ids.shape[0]):
+                    for j in range(ids.shape[1]):
+                        if int(ids[t, j]) == e:
+                            seg[int(slot[t, j])] = t
+                for t in seg:
+                    rows_q.append(quant[s][0][t])
+                    rows_s.append(quant[s][1][t])
+            offsets.append(len(rows_q))
+        k_cols = quant[0][0].shape[1]
+        codes = np.array(rows_q, np.uint8).reshape(-1, k_cols)
+        scales = np.array(rows_s, np.uint8).reshape(-1, k_cols // 32)
+        out.append((codes, scales, np.array(offsets, np.int64)))
+    return out

@@ -23,6 +23,9 @@ Recipe (seed = 1000 * workload + tensor index unless stated):
                   distinct experts of 64 by Gumbel-top-8 on log((e+1)^-1.1)
                   (seed 5001); rows are gathered by expert, then by token;
                   W [64, 2048, 7168] ~ N(0, 0.02), expert e with seed 5100 + e.
+  moe_dispatch    per source rank s: X_s [16384, 7168] ~ N(0, 1) (seed 5000 + 10 s)
+                  and its top-8 of 64 experts as above (seed 5001 + 10 s), kept as
+                  the [tokens, 8] choice matrix, highest score first.
 """
 from __future__ import annotations
 
@@ -30,8 +33,8 @@ import numpy as np
 import torch
 
 __all__ = [
-    "normal_bf16", "as_u16", "from_u16", "route_topk", "WORKLOADS",
-    "mxfp8_256x512", "ds_fp8_gemm", "qat_forward", "moe_prequant_matrix", "moe_grouped",
+    "normal_bf16", "as_u16", "from_u16", "route_choices", "route_topk", "WORKLOADS",
+    "mxfp8_256x512", "ds_fp8_gemm", "qat_forward", "moe_prequant_matrix", "moe_grouped", "moe_dispatch",
 ]
 
 
@@ -98,18 +101,25 @@ def moe_prequant_matrix(i: int) -> torch.Tensor:
     return normal_bf16(shape, 0.02, seed=4000 + i)
 
 
+def route_choices(tokens: int, experts: int = MOE_EXPERTS, topk: int = 8, zipf_s: float = 1.1,
+                  seed: int = 5001) -> torch.Tensor:
+    """[tokens, topk] int32: each token's `topk` distinct experts, drawn by
+    Gumbel-top-k with expert popularity (e+1)^-s, highest score first."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    logw = -zipf_s * torch.log(torch.arange(1, experts + 1, dtype=torch.float64))
+    u = torch.rand(tokens, experts, generator=g, dtype=torch.float64).clamp_min(1e-300)
+    gumbel = -torch.log(-torch.log(u))
+    return torch.topk(logw[None, :] + gumbel, topk, dim=1).indices.to(torch.int32).contiguous()
+
+
 def route_topk(tokens: int, experts: int = MOE_EXPERTS, topk: int = 8, zipf_s: float = 1.1,
                seed: int = 5001):
     """Gumbel-top-k routing with expert popularity (e+1)^-s: each token draws
     `topk` distinct experts (sampling without replacement, weights (e+1)^-s).
     Returns (perm_token [tokens*topk] int64: the token of each permuted row,
     offsets [experts+1] int32: expert e owns permuted rows [off[e], off[e+1]))."""
-    g = torch.Generator(device="cpu")
-    g.manual_seed(int(seed))
-    logw = -zipf_s * torch.log(torch.arange(1, experts + 1, dtype=torch.float64))
-    u = torch.rand(tokens, experts, generator=g, dtype=torch.float64).clamp_min(1e-300)
-    gumbel = -torch.log(-torch.log(u))
-    choice = torch.topk(logw[None, :] + gumbel, topk, dim=1).indices          # [tokens, topk]
+    choice = route_choices(tokens, experts, topk, zipf_s, seed).to(torch.int64)
     expert_of = choice.reshape(-1)
     token_of = torch.arange(tokens).repeat_interleave(topk)
     order = torch.argsort(expert_of * tokens + token_of)                        # by expert, then token
@@ -129,10 +139,21 @@ def moe_grouped(tokens: int = 16384, experts: int = MOE_EXPERTS, n: int = MOE_IN
     return out
 
 
+def moe_dispatch(tokens: int = 16384, experts: int = MOE_EXPERTS, k: int = MOE_HIDDEN, topk: int = 8,
+                 world: int = 1):
+    """Per source rank s: activations x_s bf16 [tokens, k] N(0,1) and its
+    routing [tokens, topk] (Gumbel-top-k as route_choices); rank 0 of one
+    rank is the moe_grouped tokens and routing."""
+    xs = [normal_bf16((tokens, k), 1.0, seed=5000 + 10 * s) for s in range(world)]
+    ids = [route_choices(tokens, experts, topk, seed=5001 + 10 * s) for s in range(world)]
+    return {"x": xs, "topk_ids": ids}
+
+
 WORKLOADS = {
     "mxfp8_256x512": "MXFP8 quantize+dequantize of bf16 256x512 + 64x256x512 MXFP8 GEMM",
     "ds_fp8_gemm": "1x128/128x128 FP8 quantize of A 4096x7168, B 2048x7168 + fp32-scaled GEMM",
     "qat_forward": "LoRA merge + 128x128 fake-quant of W 2048x7168, 1x128 of X 8192x7168 + GEMM",
     "moe_prequant": "64 experts x {gate, up 2048x7168; down 7168x2048} -> MXFP8 and NVFP4",
     "moe_grouped": "16384 tokens x 7168, top-8 of 64 experts, grouped MXFP8 GEMM N=2048",
+    "moe_dispatch": "16384 tokens x 7168, top-8 of 64 experts: MXFP8 quantize + scatter by expert",
 }
