@@ -307,6 +307,75 @@ FPQ_API fpq_status fpq_qat_backward(const void* dy, const void* x_fq, const void
                                     size_t workspace_bytes, void* stream);
 
 /*
+ * MoE FP8 dispatch ["DeepSeek-V3 Blog 5: Low-Precision Training", Reducing
+ * Communication Overhead in MoE with FP8: token activations are quantized to
+ * FP8 before they are sent to the GPUs that hold their experts].  Tokens are
+ * quantized to MXFP8 (E4M3 codes, E8M0 scale per 32, as fpq_quantize_block
+ * FPQ_MXFP8) and each token's codes and scales are written once per chosen
+ * expert, to the rows of that expert.
+ *
+ * Row order: with `world` ranks and E experts, rank r owns experts
+ * [r L, (r + 1) L), L = E / world.  A rank's receive buffer holds its local
+ * experts' rows in expert order; each expert's rows come from source rank
+ * 0, 1, ... in turn; from one source, the (token, choice) pairs routed to
+ * that expert in token order, then choice order (the pair's slot).  The
+ * buffer is the `aq`/`as` operand of fpq_grouped_scaled_gemm (FPQ_MXFP8)
+ * with `recv_offsets` as its group offsets.
+ *
+ * Calls, on the source rank's stream:
+ *   fpq_moe_route          per-expert counts of this rank's pairs, and the
+ *                          slot bases in the workspace;
+ *   (the ranks exchange counts: counts_all [world, E], e.g. an all-gather)
+ *   fpq_moe_dispatch_layout  destination row of slot 0 of every expert, and
+ *                          this rank's group offsets;
+ *   fpq_moe_dispatch_mxfp8 quantize + write every pair's row.
+ *
+ *   topk_ids    DEVICE int32 [tokens, topk], expert ids in [0, E); an id out
+ *               of range raises FPQ_ERR_DEVICE_BAD_INPUT and its pair is
+ *               dropped
+ *   counts      DEVICE int32 [E] (out)
+ *   workspace   fpq_moe_route_workspace_bytes(tokens, E) bytes, 16-byte
+ *               aligned, caller-owned; fpq_moe_route writes it and
+ *               fpq_moe_dispatch_mxfp8 (same tokens, topk, E) reads it
+ *   counts_all  DEVICE int32 [world, E]: row s = source rank s's counts
+ *   mode        FPQ_MOE_DIRECT: rows go straight into the receivers'
+ *               buffers (one GPU, or peer memory); dst_row0[e] = row of
+ *               slot 0 of expert e, from this rank, in rank e / L's buffer.
+ *               FPQ_MOE_PACK: rows go into this rank's send buffer, expert-
+ *               major in slot order (for a collective that moves each
+ *               (expert, source) segment to its receiver); dst_row0[e] =
+ *               rows of this rank's experts before e
+ *   dst_row0    DEVICE int64 [E] (out);  recv_offsets DEVICE int32 [L + 1]
+ *               (out): row of local expert l in this rank's receive buffer
+ *   x           DEVICE bf16 [tokens, hidden], hidden a positive multiple of 32
+ *   n_dest      number of destination buffers; expert e goes to buffer
+ *               e / (E / n_dest) (DIRECT: n_dest = world; PACK: 1)
+ *   dst_codes, dst_scales  DEVICE arrays of n_dest DEVICE pointers: uint8
+ *               [rows, hidden] codes and uint8 [rows, hidden/32] E8M0 scales
+ *               (16-byte aligned code buffers); peer pointers are allowed
+ *   dst_capacity  DEVICE int64 [n_dest]: rows of each buffer; a row outside
+ *               raises FPQ_ERR_DEVICE_BAD_INPUT and is not written
+ *
+ * Requires tokens >= 0, 1 <= topk <= 32, 1 <= E <= 1024, world >= 1 dividing
+ * E, 0 <= rank < world, n_dest >= 1 dividing E; the pointer arguments of
+ * fpq_moe_dispatch_mxfp8 16-byte aligned.  Errors: FPQ_ERR_INVALID_ARG,
+ * FPQ_ERR_ALIGNMENT, FPQ_ERR_WORKSPACE, FPQ_ERR_CUDA.
+ */
+#define FPQ_MOE_DIRECT 0
+#define FPQ_MOE_PACK 1
+FPQ_API size_t fpq_moe_route_workspace_bytes(int64_t tokens, int32_t num_experts);
+FPQ_API fpq_status fpq_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t topk, int32_t num_experts,
+                                 int32_t* counts, void* workspace, size_t workspace_bytes, void* stream);
+FPQ_API fpq_status fpq_moe_dispatch_layout(const int32_t* counts_all, int32_t world, int32_t num_experts,
+                                           int32_t rank, int32_t mode, int64_t* dst_row0, int32_t* recv_offsets,
+                                           void* stream);
+FPQ_API fpq_status fpq_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hidden, const int32_t* topk_ids,
+                                          int32_t topk, int32_t num_experts, const void* workspace,
+                                          size_t workspace_bytes, const int64_t* dst_row0, int32_t n_dest,
+                                          void* const* dst_codes, void* const* dst_scales,
+                                          const int64_t* dst_capacity, void* stream);
+
+/*
  * fpq_grouped_scaled_gemm -- per-expert product over a token-permuted
  * activation matrix (MoE routed experts) [FP "Quick start": routed MoE
  * expert projections; DS "Как FP8 связан с MoE-архитектурой DeepSeek V3"]:

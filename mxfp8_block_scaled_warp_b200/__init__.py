@@ -27,6 +27,8 @@ __all__ = [
     "fpq_lora_merge_fakequant", "fpq_scaled_gemm", "fpq_scaled_gemm_nvfp4", "fpq_grouped_scaled_gemm",
     "fpq_get_device_error", "fpq_gemm_bf16", "fpq_gemm_bf16_layout", "fpq_transpose_bf16",
     "fpq_gemm_bf16_splitk_workspace_bytes", "fpq_gemm_bf16_splitk", "fpq_qat_backward_workspace_bytes",
+    "fpq_moe_route_workspace_bytes", "fpq_moe_route", "fpq_moe_dispatch_layout", "fpq_moe_dispatch_mxfp8",
+    "MOE_DIRECT", "MOE_PACK",
     "fpq_qat_backward",
     "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
     "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "scaled_gemm_nvfp4", "grouped_scaled_gemm",
@@ -83,6 +85,10 @@ def _load() -> ctypes.CDLL:
         "fpq_gemm_bf16_splitk_workspace_bytes": (SZ, [I64, I64, I64]),
         "fpq_gemm_bf16_splitk": (I32, [P, I32, P, I32, I64, I64, I64, F, P, P, SZ, P]),
         "fpq_qat_backward_workspace_bytes": (SZ, [I64, I64, I64, I32]),
+        "fpq_moe_route_workspace_bytes": (SZ, [I64, I32]),
+        "fpq_moe_route": (I32, [P, I64, I32, I32, P, P, SZ, P]),
+        "fpq_moe_dispatch_layout": (I32, [P, I32, I32, I32, I32, P, P, P]),
+        "fpq_moe_dispatch_mxfp8": (I32, [P, I64, I64, P, I32, I32, P, SZ, P, I32, P, P, P, P]),
         "fpq_qat_backward": (I32, [P, P, P, P, P, I64, I64, I64, I32, F, P, P, P, P, P, SZ, P]),
         "fpq_quantize_nvfp4_noalloc": (I32, [P, I64, I64, I64, P, P, P, P]),
     }
@@ -168,6 +174,36 @@ def fpq_gemm_bf16_splitk(p, p_mn, q, q_mn, m, n, k, alpha, c, workspace, stream=
     _check(load().fpq_gemm_bf16_splitk(_ptr(p), int(p_mn), _ptr(q), int(q_mn), m, n, k, float(alpha), _ptr(c),
                                        _ptr(workspace) if workspace is not None else None, wsb, _stream(stream)),
            "fpq_gemm_bf16_splitk")
+
+
+MOE_DIRECT, MOE_PACK = 0, 1
+
+
+def fpq_moe_route_workspace_bytes(tokens: int, num_experts: int) -> int:
+    return load().fpq_moe_route_workspace_bytes(tokens, num_experts)
+
+
+def fpq_moe_route(topk_ids, tokens, topk, num_experts, counts, workspace, stream=None):
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().fpq_moe_route(_ptr(topk_ids) if tokens else None, tokens, topk, num_experts, _ptr(counts),
+                                _ptr(workspace) if workspace is not None else None, wsb, _stream(stream)),
+           "fpq_moe_route")
+
+
+def fpq_moe_dispatch_layout(counts_all, world, num_experts, rank, mode, dst_row0, recv_offsets, stream=None):
+    _check(load().fpq_moe_dispatch_layout(_ptr(counts_all), world, num_experts, rank, mode, _ptr(dst_row0),
+                                          _ptr(recv_offsets), _stream(stream)), "fpq_moe_dispatch_layout")
+
+
+def fpq_moe_dispatch_mxfp8(x, tokens, hidden, topk_ids, topk, num_experts, workspace, dst_row0, n_dest, dst_codes,
+                           dst_scales, dst_capacity, stream=None):
+    """dst_codes, dst_scales, dst_capacity: device int64 tensors of n_dest
+    entries (buffer addresses, and rows per buffer)."""
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().fpq_moe_dispatch_mxfp8(_ptr(x), tokens, hidden, _ptr(topk_ids), topk, num_experts,
+                                         _ptr(workspace) if workspace is not None else None, wsb, _ptr(dst_row0),
+                                         n_dest, _ptr(dst_codes), _ptr(dst_scales), _ptr(dst_capacity),
+                                         _stream(stream)), "fpq_moe_dispatch_mxfp8")
 
 
 def fpq_transpose_bf16(x, out, rows, cols, stream=None):

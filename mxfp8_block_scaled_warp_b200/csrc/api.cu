@@ -266,6 +266,82 @@ fpq_status fpq_gemm_bf16_layout(const void* p, int32_t p_mn, const void* q, int3
                      "bf16 gemm launch");
 }
 
+size_t fpq_moe_route_workspace_bytes(int64_t tokens, int32_t num_experts) {
+    if (tokens < 0 || num_experts < 1 || num_experts > 1024) return 0;
+    return fpq::moe_route_workspace_bytes(tokens, num_experts);
+}
+
+fpq_status fpq_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t topk, int32_t num_experts,
+                         int32_t* counts, void* workspace, size_t workspace_bytes, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (tokens < 0 || tokens > (1ll << 31) || topk < 1 || topk > 32 || num_experts < 1 || num_experts > 1024) {
+        set_detail("need tokens >= 0, topk in [1, 32], num_experts in [1, 1024]");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if (!counts || (tokens > 0 && !topk_ids)) {
+        set_detail("null pointer");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < fpq::moe_route_workspace_bytes(tokens, num_experts)) {
+        set_detail("need a 16-byte aligned workspace of fpq_moe_route_workspace_bytes() bytes");
+        return FPQ_ERR_WORKSPACE;
+    }
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_moe_route(topk_ids, tokens, topk, num_experts, counts, workspace, d->err,
+                                           (cudaStream_t)stream),
+                     "moe route launch");
+}
+
+fpq_status fpq_moe_dispatch_layout(const int32_t* counts_all, int32_t world, int32_t num_experts, int32_t rank,
+                                   int32_t mode, int64_t* dst_row0, int32_t* recv_offsets, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (world < 1 || num_experts < 1 || num_experts > 1024 || num_experts % world || rank < 0 || rank >= world ||
+        (mode != FPQ_MOE_DIRECT && mode != FPQ_MOE_PACK)) {
+        set_detail("need world >= 1 dividing num_experts in [1, 1024], 0 <= rank < world, a known mode");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if (!counts_all || !dst_row0 || !recv_offsets) {
+        set_detail("null pointer");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_moe_layout(counts_all, world, num_experts, rank, mode == FPQ_MOE_PACK, dst_row0,
+                                            recv_offsets, (cudaStream_t)stream),
+                     "moe layout launch");
+}
+
+fpq_status fpq_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hidden, const int32_t* topk_ids,
+                                  int32_t topk, int32_t num_experts, const void* workspace, size_t workspace_bytes,
+                                  const int64_t* dst_row0, int32_t n_dest, void* const* dst_codes,
+                                  void* const* dst_scales, const int64_t* dst_capacity, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (tokens < 0 || tokens > (1ll << 31) || hidden < 32 || hidden % 32 || hidden > (1 << 24) || topk < 1 ||
+        topk > 32 || num_experts < 1 || num_experts > 1024 || n_dest < 1 || num_experts % n_dest) {
+        set_detail("need tokens >= 0, hidden a positive multiple of 32, topk in [1, 32], num_experts in "
+                   "[1, 1024], n_dest >= 1 dividing num_experts");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if (tokens == 0) return FPQ_OK;
+    if ((st = check_ptrs({x, topk_ids, dst_row0, dst_codes, dst_scales, dst_capacity})) != FPQ_OK) return st;
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < fpq::moe_route_workspace_bytes(tokens, num_experts)) {
+        set_detail("need the workspace that fpq_moe_route wrote");
+        return FPQ_ERR_WORKSPACE;
+    }
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_moe_dispatch_mxfp8(x, tokens, hidden, topk_ids, topk, num_experts, workspace,
+                                                    dst_row0, n_dest, dst_codes, dst_scales, dst_capacity, d->err,
+                                                    (cudaStream_t)stream),
+                     "moe dispatch launch");
+}
+
 size_t fpq_gemm_bf16_splitk_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 1 || n < 1 || k < 1) return 0;
     return (size_t)fpq::kMaxSplits * (size_t)m * (size_t)n * 4;

@@ -53,6 +53,21 @@ cudaError_t launch_gemm_bf16_splitk(const void* p, bool p_mn, const void* q, boo
                                     int64_t k, float alpha, void* c, float* partial, int splits, uint32_t* err,
                                     cudaStream_t st);
 
+// MoE FP8 dispatch (moe_dispatch.cu).  The route workspace holds the
+// per-chunk histograms and slot bases; a chunk is moe_tokens_per_chunk(T)
+// consecutive tokens.
+int64_t moe_tokens_per_chunk(int64_t tokens);
+int64_t moe_chunks(int64_t tokens);
+size_t moe_route_workspace_bytes(int64_t tokens, int experts);
+cudaError_t launch_moe_route(const int32_t* ids, int64_t tokens, int topk, int experts, int32_t* counts,
+                             void* workspace, uint32_t* err, cudaStream_t st);
+cudaError_t launch_moe_layout(const int32_t* counts_all, int world, int experts, int rank, int pack,
+                              int64_t* dst_row0, int32_t* recv_offsets, cudaStream_t st);
+cudaError_t launch_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hidden, const int32_t* ids, int topk,
+                                      int experts, const void* workspace, const int64_t* dst_row0, int n_dest,
+                                      void* const* dst_codes, void* const* dst_scales, const int64_t* dst_capacity,
+                                      uint32_t* err, cudaStream_t st);
+
 // bf16 [R, C] -> [C, R] (R, C multiples of 8).
 cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t C, cudaStream_t st);
 
