@@ -529,8 +529,79 @@ class Nvfp4Gemm(Step):
         return self.a_host.numel() * 2 + self.b_host.numel() * 2, self.c.numel() * 2
 
 
+class MoeDispatch(Step):
+    """The FP8 MoE dispatch on one GPU: 16384 tokens x 7168 bf16, top-8 of 64
+    experts; route (per-chunk histograms + scan), layout, and the fused
+    kernel that quantizes each token row once to MXFP8 and writes it to the
+    rows of its 8 experts in the expert-grouped buffer (the grouped GEMM's
+    input).  On one GPU every destination is local."""
+    name = "moe_dispatch"
+    dominant = "moe_dispatch_mxfp8"
+    unit = "GB/s"
+    dtype = "bf16 -> e4m3 + e8m0 (scatter)"
+
+    def __init__(self, fpq, dev, tokens=16384, hidden=7168, experts=64, topk=8):
+        self.f = fpq
+        wl = workloads.moe_dispatch(tokens, experts, hidden, topk)
+        self.x_host, self.ids_host = wl["x"][0].pin_memory(), wl["topk_ids"][0].pin_memory()
+        self.x, self.ids = self.x_host.to(dev), self.ids_host.to(dev)
+        self.t, self.h, self.e, self.k = tokens, hidden, experts, topk
+        i32, i64, u8 = (dict(dtype=d, device=dev) for d in (torch.int32, torch.int64, torch.uint8))
+        self.counts = torch.empty((experts,), **i32)
+        wsb = fpq.fpq_moe_route_workspace_bytes(tokens, experts)
+        self.ws = torch.empty(((wsb + 15) // 16 * 16,), **u8)
+        self.row0 = torch.empty((experts,), **i64)
+        self.offs = torch.empty((experts + 1,), **i32)
+        rows = tokens * topk
+        self.q, self.s = torch.empty((rows, hidden), **u8), torch.empty((rows, hidden // 32), **u8)
+        self.qp = torch.tensor([self.q.data_ptr()], **i64)
+        self.sp = torch.tensor([self.s.data_ptr()], **i64)
+        self.cap = torch.tensor([rows], **i64)
+        self.offs_host = torch.empty((experts + 1,), dtype=torch.int32).pin_memory()
+        # algorithmic bytes: x read once, ids read twice (route, dispatch), codes + scales written once per pair
+        self.dispatch_bytes = tokens * hidden * 2 + tokens * topk * 4 + rows * (hidden + hidden // 32)
+        self.route_bytes = tokens * topk * 4
+        self.bytes = self.dispatch_bytes + self.route_bytes
+        self.quant_bytes = self.bytes
+        self.launches = 4
+        self.config = {"workload": "moe_dispatch: X 16384x7168 bf16 N(0,1), top-8 of 64 experts (Gumbel-top-8 on "
+                                   "log((e+1)^-1.1)) -> MXFP8 rows grouped by expert, one GPU (all destinations "
+                                   "local)", "tokens": tokens, "hidden": hidden, "experts": experts, "topk": topk,
+                       "l2": "flushed before every step (256 MiB write)"}
+
+    @property
+    def work(self):
+        return self.bytes
+
+    def kernels(self):
+        f = self.f
+        return [
+            ("moe_route", lambda: f.fpq_moe_route(self.ids, self.t, self.k, self.e, self.counts, self.ws)),
+            ("moe_layout", lambda: f.fpq_moe_dispatch_layout(self.counts, 1, self.e, 0, f.MOE_DIRECT, self.row0,
+                                                             self.offs)),
+            ("moe_dispatch_mxfp8", lambda: f.fpq_moe_dispatch_mxfp8(self.x, self.t, self.h, self.ids, self.k, self.e,
+                                                                    self.ws, self.row0, 1, self.qp, self.sp,
+                                                                    self.cap)),
+        ]
+
+    def kernel_work(self):
+        return {"moe_route": ("GB/s", self.route_bytes), "moe_layout": ("GB/s", self.e * 4 * 2),
+                "moe_dispatch_mxfp8": ("GB/s", self.dispatch_bytes)}
+
+    def e2e_step(self, stream, side_stream):
+        """Tokens and routing from pinned host memory in, the group offsets
+        back to the host (the grouped rows stay on the device for the expert
+        GEMM)."""
+        self.x.copy_(self.x_host, non_blocking=True)
+        self.ids.copy_(self.ids_host, non_blocking=True)
+        self.whole_step(side_stream)
+        self.offs_host.copy_(self.offs, non_blocking=True)
+        return self.x_host.numel() * 2 + self.ids_host.numel() * 4, self.offs.numel() * 4
+
+
 STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": QatForward,
-         "moe_prequant": MoePrequant, "nvfp4_gemm": Nvfp4Gemm, "qat_backward": QatBackward}
+         "moe_prequant": MoePrequant, "nvfp4_gemm": Nvfp4Gemm, "qat_backward": QatBackward,
+         "moe_dispatch": MoeDispatch}
 
 
 # ------------------------------------------------------------------ traffic from committed ncu summaries
@@ -539,7 +610,8 @@ def _source_hash(kernel: str) -> str | None:
     src = {"gemm_fp8_f32scale": "gemm_fp8_f32scale.cu", "gemm_grouped_mxfp8": "gemm_mxfp8.cu",
            "gemm_mxfp8": "gemm_mxfp8.cu", "quant_fp8_1x128": "quant_kernels.cu",
            "quant_mxfp8": "quant_kernels.cu", "lora_merge_fq": "merge_kernel.cu",
-           "gemm_nvfp4": "gemm_nvfp4.cu", "gemm_bf16_dx": "gemm_bf16.cu"}.get(kernel)
+           "gemm_nvfp4": "gemm_nvfp4.cu", "gemm_bf16_dx": "gemm_bf16.cu",
+           "moe_dispatch_mxfp8": "moe_dispatch.cu"}.get(kernel)
     if not src:
         return None
     with open(os.path.join(ROOT, "mxfp8_block_scaled_warp_b200", "csrc", src), "rb") as f:
@@ -572,6 +644,8 @@ def cpu_baseline(workload: str, budget_s: float = 12.0):
         return _cpu_baseline_prequant(oracle, budget_s)
     if workload == "nvfp4_gemm":
         return _cpu_baseline_nvfp4_gemm(oracle, budget_s)
+    if workload == "moe_dispatch":
+        return _cpu_baseline_moe_dispatch(oracle, budget_s)
     if workload != "ds_fp8_gemm":
         return None
     m, n, k = 4096, 2048, 7168
@@ -634,6 +708,28 @@ def _cpu_baseline_nvfp4_gemm(oracle, budget_s: float):
             "kind": "oracle",
             "sample": f"NVFP4 quantize of {rows} rows of each 7168-wide operand, {count} fp64 GEMM entries "
                       f"(K=7168); extrapolated to the full 4096x2048x7168 step ({step_s:.1f} s per step on one core)"}
+
+
+def _cpu_baseline_moe_dispatch(oracle, budget_s: float):
+    """The oracle's dispatch (route plan, MXFP8 quantization, placement) on
+    the first tokens of the workload (count sized to the budget),
+    extrapolated to the 16384-token step at its per-byte rate."""
+    wl = workloads.moe_dispatch(tokens=16384)
+    x, ids = workloads.as_u16(wl["x"][0]), wl["topk_ids"][0].numpy()
+    hidden, topk = x.shape[1], ids.shape[1]
+    per_tok = hidden * 2 + topk * 8 + topk * (hidden + hidden // 32)
+    n = 256
+    t0 = time.perf_counter()
+    oracle.moe_dispatch([x[:n]], [ids[:n]], 64)
+    per = (time.perf_counter() - t0) / n
+    n = int(max(256, min(16384, budget_s / max(per, 1e-9))))
+    t0 = time.perf_counter()
+    oracle.moe_dispatch([x[:n]], [ids[:n]], 64)
+    dt = time.perf_counter() - t0
+    work = 16384 * per_tok
+    return {"value": n * per_tok / dt / 1e9, "unit": "GB/s", "work": work, "cores": 1, "kind": "oracle",
+            "sample": f"oracle dispatch of the first {n} of 16384 tokens (top-8 of 64 experts, 7168 wide); "
+                      f"extrapolated to the whole step ({16384 / n * dt:.1f} s on one core)"}
 
 
 def _cpu_baseline_prequant(oracle, budget_s: float):
