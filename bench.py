@@ -6,10 +6,12 @@ quantize the weights B [2048, 7168] (fp32 scale per 128x128 block), then
 C = A B^T with fp32 accumulation and bf16 output (120.3 GFLOP).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload ds_fp8_gemm|qat_forward|moe_grouped|moe_prequant|mxfp8_256x512]
+                    [--workload ds_fp8_gemm|qat_forward|qat_backward|moe_grouped|moe_dispatch|
+                                moe_prequant|nvfp4_gemm]
 
 Prints one JSON line (rank 0).  `value` is whole-step throughput in TFLOP/s
-(GEMM flops of the step / step time, quantization included), with the
+(GEMM flops of the step / step time, quantization included; GB/s for the
+quantize-only and dispatch-only workloads), with the
 inputs resident in HBM and L2 flushed (256 MiB write) before every step; the
 per-kernel times, the quantize GB/s and the roofline of the dominant kernel
 come from CUDA events on the launching stream.  With N > 1 (torchrun) every
@@ -200,59 +202,81 @@ class DsFp8Gemm(Step):
 
 
 class MoeGrouped(Step):
+    """The expert up-projection of an MoE layer on one GPU: 16384 bf16
+    tokens x 7168, top-8 of 64 experts.  The FP8 dispatch (route, layout, and
+    the fused kernel that quantizes each token row once to MXFP8 and writes
+    it to the rows of its 8 experts) builds the expert-grouped operand; the
+    grouped MXFP8 GEMM multiplies it with the prequantized expert weights
+    64 x 2048 x 7168."""
     name = "moe_grouped"
     dominant = "gemm_grouped_mxfp8"
 
-    def __init__(self, fpq, dev):
+    def __init__(self, fpq, dev, tokens=16384, experts=64, topk=8):
         self.f = fpq
         wl = workloads.moe_grouped()
-        x_perm = wl["x"][wl["perm"]]
-        self.x = x_perm.to(dev)
-        self.offsets = wl["offsets"].to(dev)
+        self.x_host = wl["x"].pin_memory()
+        self.ids_host = workloads.route_choices(tokens, experts, topk, seed=5001).pin_memory()
+        self.x, self.ids = self.x_host.to(dev), self.ids_host.to(dev)
         self.w = wl["w"].to(dev)
         self.wq, self.ws = fpq.quantize(self.w, fpq.MXFP8)      # weights are prequantized once (serving)
         del self.w
-        self.total, self.k = self.x.shape
+        self.tokens, self.k = self.x.shape
+        self.topk, self.e = topk, experts
+        self.total = tokens * topk
         self.groups, self.n = self.wq.shape[0], self.wq.shape[1]
-        self.qx = torch.empty_like(self.x, dtype=torch.uint8)
-        self.sx = torch.empty((self.total, self.k // 32), dtype=torch.uint8, device=dev)
+        i32, i64, u8 = (dict(dtype=d, device=dev) for d in (torch.int32, torch.int64, torch.uint8))
+        self.counts_dev = torch.empty((experts,), **i32)
+        wsb = fpq.fpq_moe_route_workspace_bytes(tokens, experts)
+        self.rws = torch.empty(((wsb + 15) // 16 * 16,), **u8)
+        self.row0 = torch.empty((experts,), **i64)
+        self.offsets = torch.empty((experts + 1,), **i32)
+        self.qx = torch.empty((self.total, self.k), **u8)
+        self.sx = torch.empty((self.total, self.k // 32), **u8)
+        self.qp = torch.tensor([self.qx.data_ptr()], **i64)
+        self.sp = torch.tensor([self.sx.data_ptr()], **i64)
+        self.cap = torch.tensor([self.total], **i64)
         self.c = torch.empty((self.total, self.n), dtype=torch.bfloat16, device=dev)
+        self.c_host = torch.empty(self.c.shape, dtype=self.c.dtype).pin_memory()
         self.flops = 2.0 * self.total * self.n * self.k
-        self.qx_bytes = self.total * self.k * 3 + self.total * self.k // 32
-        self.quant_bytes = self.qx_bytes
-        self.launches = 2
-        self.counts = np.diff(wl["offsets"].numpy()).tolist()
-        self.config = {"workload": "moe_grouped: X 16384x7168 N(0,1), top-8 of 64 experts (Zipf 1.1 Gumbel-top-8), "
-                                   "131072 permuted rows -> MXFP8; grouped GEMM with MXFP8 expert weights 64x2048x7168",
-                       "expert_rows_max": max(self.counts), "expert_rows_min": min(self.counts),
+        self.route_bytes = self.total * 4
+        self.dispatch_bytes = self.tokens * self.k * 2 + self.total * 4 + self.total * (self.k + self.k // 32)
+        self.quant_bytes = self.route_bytes + self.dispatch_bytes
+        self.launches = 5
+        counts = np.bincount(self.ids_host.numpy().reshape(-1), minlength=experts)
+        self.config = {"workload": "moe_grouped: X 16384x7168 N(0,1), top-8 of 64 experts (Zipf 1.1 Gumbel-top-8); "
+                                   "FP8 dispatch (each token quantized once to MXFP8, 131072 rows grouped by "
+                                   "expert); grouped GEMM with MXFP8 expert weights 64x2048x7168",
+                       "expert_rows_max": int(counts.max()), "expert_rows_min": int(counts.min()),
                        "l2": "flushed before every step (256 MiB write)"}
 
     def kernels(self):
         f = self.f
         return [
-            ("quant_mxfp8", lambda: f.fpq_quantize_block(f.MXFP8, self.x, 1, self.total, self.k, self.qx, self.sx)),
+            ("moe_route", lambda: f.fpq_moe_route(self.ids, self.tokens, self.topk, self.e, self.counts_dev,
+                                                  self.rws)),
+            ("moe_layout", lambda: f.fpq_moe_dispatch_layout(self.counts_dev, 1, self.e, 0, f.MOE_DIRECT, self.row0,
+                                                             self.offsets)),
+            ("moe_dispatch_mxfp8", lambda: f.fpq_moe_dispatch_mxfp8(self.x, self.tokens, self.k, self.ids, self.topk,
+                                                                    self.e, self.rws, self.row0, 1, self.qp, self.sp,
+                                                                    self.cap)),
             ("gemm_grouped_mxfp8", lambda: f.fpq_grouped_scaled_gemm(f.MXFP8, self.qx, self.sx, self.wq, self.ws,
                                                                      self.offsets, self.groups, self.total, self.n,
                                                                      self.k, self.c, f.OUT_BF16)),
         ]
 
     def kernel_work(self):
-        return {"quant_mxfp8": ("GB/s", self.qx_bytes), "gemm_grouped_mxfp8": ("TFLOP/s", self.flops)}
+        return {"moe_route": ("GB/s", self.route_bytes), "moe_layout": ("GB/s", self.e * 8),
+                "moe_dispatch_mxfp8": ("GB/s", self.dispatch_bytes), "gemm_grouped_mxfp8": ("TFLOP/s", self.flops)}
 
     def e2e_step(self, stream, side_stream):
-        """Permuted tokens and the group offsets from pinned host memory in,
-        the expert outputs back to pinned host memory, copies inside the
-        timed region (the expert weights stay resident: serving)."""
-        if not hasattr(self, "x_host"):
-            self.x_host = self.x.cpu().pin_memory()
-            self.off_host = self.offsets.cpu().pin_memory()
-            self.c_host = torch.empty(self.c.shape, dtype=self.c.dtype).pin_memory()
+        """Tokens and their routing from pinned host memory in, the expert
+        outputs back to pinned host memory, copies inside the timed region
+        (the expert weights stay resident: serving)."""
         self.x.copy_(self.x_host, non_blocking=True)
-        self.offsets.copy_(self.off_host, non_blocking=True)
-        for _, fn in self.kernels():
-            fn()
+        self.ids.copy_(self.ids_host, non_blocking=True)
+        self.whole_step(side_stream)
         self.c_host.copy_(self.c, non_blocking=True)
-        return self.x.numel() * 2 + self.offsets.numel() * 4, self.c.numel() * 2
+        return self.x_host.numel() * 2 + self.ids_host.numel() * 4, self.c.numel() * 2
 
 
 class QatForward(Step):
