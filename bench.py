@@ -368,7 +368,7 @@ class MoePrequant(Step):
         self.nv_bytes = elems * (2 + 0.5 + 1 / 16) + 4 * 3 * experts
         self.quant_bytes = self.mx_bytes + self.nv_bytes
         self.launches = 6
-        self.config = {"workload": "moe_prequant: 64 experts x {gate, up 2048x7168; down 7168x2048} bf16 N(0,0.02) "
+        self.config = {"workload": f"moe_prequant: {experts} experts x {{gate, up 2048x7168; down 7168x2048}} bf16 N(0,0.02) "
                                    "-> MXFP8 (1x32 E8M0) and NVFP4 (1x16 E4M3 + fp32 per matrix); one batched call "
                                    "per projection and format",
                        "elements": elems, "l2": "flushed before every step (256 MiB write)"}
@@ -869,6 +869,8 @@ def main():
     ap.add_argument("--impl", default="fpq", choices=["fpq", "reference"])
     ap.add_argument("--workload", default="ds_fp8_gemm", choices=sorted(STEPS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="moe_prequant only: experts per projection (default 64; fewer for small profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -884,7 +886,7 @@ def main():
     dev = torch.device("cuda", local)
     pg = init_replicas(world, "nccl", dev)
 
-    step = STEPS[args.workload](fpq, dev)
+    step = STEPS[args.workload](fpq, dev, **({"experts": args.experts} if args.experts else {}))
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     kern = step.kernels()
