@@ -195,10 +195,10 @@ quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 // the whole matrix before any block of it can be encoded, so every matrix
 // is read twice: once for its amax ("A" tiles) and once to encode it ("B"
 // tiles).  Work items (tiles of 4096 units = 128 KB of input) are handed out
-// from a global counter in the order
-//   A(0), A(1), B(0), A(2), B(1), ..., A(n-1), B(n-2), B(n-1)
+// from a global counter in the order (lookahead LA = NV_LOOKAHEAD)
+//   A(0), ..., A(LA-1), A(LA), B(0), A(LA+1), B(1), ..., A(n-1), B(n-1-LA), B(n-LA), ..., B(n-1)
 // (each a run over all tiles of the matrix), so the encode of matrix b
-// starts one matrix of amax work after its own amax, and its second read is
+// starts LA matrices of amax work after its own amax, and its second read is
 // mostly served by L2.  A B tile of matrix b waits (bounded) until all A
 // tiles of b have published their amax.  An item only waits on items with
 // smaller indices, and the smallest unfinished item is always being run by
@@ -209,6 +209,7 @@ quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 // (64-bit), [4, 4 + batch) amax patterns, [4 + batch, 4 + 2 batch) number of
 // finished A tiles per matrix.
 constexpr int NV_UNITS_PER_THREAD = 16;        // units of one item per thread
+constexpr int NV_LOOKAHEAD = 1;                // matrices of amax work ahead of the encode
 constexpr int NV_TILE_UNITS = kThreads * NV_UNITS_PER_THREAD;
 
 // Per-tensor scale g = fp32(amax_T / 2688), 1 for an all-zero tensor.
@@ -252,16 +253,20 @@ struct NvItem {
 
 __device__ __forceinline__ NvItem nv_decode(unsigned long long item, int64_t batch, int64_t nT) {
     NvItem r;
-    const int64_t i = (int64_t)item;
-    if (i < nT) {
-        r.is_a = true; r.b = 0; r.t = i;
+    const int64_t i = (int64_t)item, blk = i / nT;
+    const int64_t la = min64(NV_LOOKAHEAD, batch);
+    r.t = i - blk * nT;
+    if (blk < la) {                                   // leading amax runs
+        r.is_a = true; r.b = blk;
         return r;
     }
-    const int64_t j = i - nT, blk = j / nT;
-    r.t = j - blk * nT;
-    if (blk == 2 * (batch - 1)) { r.is_a = false; r.b = batch - 1; }
-    else if ((blk & 1) == 0) { r.is_a = true; r.b = blk / 2 + 1; }
-    else { r.is_a = false; r.b = (blk - 1) / 2; }
+    const int64_t j = blk - la, pairs = 2 * (batch - la);
+    if (j < pairs) {                                  // A(la + p), B(p) alternating
+        r.is_a = (j & 1) == 0;
+        r.b = r.is_a ? la + j / 2 : j / 2;
+    } else {                                          // trailing encode runs
+        r.is_a = false; r.b = batch - la + (j - pairs);
+    }
     return r;
 }
 

@@ -54,7 +54,8 @@ def _buffers(rows, hidden):
 
 
 @pytest.mark.parametrize("tokens,hidden,experts,k", [(1, 32, 1, 1), (7, 64, 8, 3), (100, 7168, 64, 8),
-                                                     (5000, 512, 16, 4), (9500, 96, 64, 8), (300, 2048, 256, 6)])
+                                                     (5000, 512, 16, 4), (9500, 96, 64, 8), (300, 2048, 256, 6),
+                                                     (50, 128, 64, 32), (200, 64, 1024, 4)])
 def test_single_rank(fpq, orc, tokens, hidden, experts, k):
     x, ids = _x(tokens, hidden, 800 + tokens), _ids(tokens, experts, k, 801 + tokens)
     src = Source(fpq, x, ids, experts)
