@@ -194,7 +194,8 @@ quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 // One persistent kernel per call.  The per-tensor scale g needs the amax of
 // the whole matrix before any block of it can be encoded, so every matrix
 // is read twice: once for its amax ("A" tiles) and once to encode it ("B"
-// tiles).  Work items (tiles of 4096 units = 128 KB of input) are handed out
+// tiles).  Work items (tiles of 256 x upt units: 128 KB of input at the
+// largest upt) are handed out
 // from a global counter in the order (lookahead LA = NV_LOOKAHEAD)
 //   A(0), ..., A(LA-1), A(LA), B(0), A(LA+1), B(1), ..., A(n-1), B(n-1-LA), B(n-LA), ..., B(n-1)
 // (each a run over all tiles of the matrix), so the encode of matrix b
@@ -208,9 +209,12 @@ quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
 // Workspace (32-bit words, zeroed by the launcher): [0, 2) item counter
 // (64-bit), [4, 4 + batch) amax patterns, [4 + batch, 4 + 2 batch) number of
 // finished A tiles per matrix.
-constexpr int NV_UNITS_PER_THREAD = 16;        // units of one item per thread
+// Units of one item per thread (upt): NV_UNITS_PER_THREAD, halved by the
+// launcher (down to 1) until every resident CTA gets about two items per
+// pass.  A thread walks its units of an item one after another, so a small
+// input cut into few large items would serialise that many memory latencies.
+constexpr int NV_UNITS_PER_THREAD = 16;
 constexpr int NV_LOOKAHEAD = 1;                // matrices of amax work ahead of the encode
-constexpr int NV_TILE_UNITS = kThreads * NV_UNITS_PER_THREAD;
 
 // Per-tensor scale g = fp32(amax_T / 2688), 1 for an all-zero tensor.
 __device__ __forceinline__ float nvfp4_tensor_scale(uint32_t a) {
@@ -311,6 +315,7 @@ __device__ __forceinline__ void nvfp4_encode_unit(const Unit& v, float g, bool g
     *sdst = (uint8_t)code;
 }
 
+template <int upt>
 __global__ void __launch_bounds__(kThreads, NV_MIN_BLOCKS)
 quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint2* __restrict__ q,
                    uint8_t* __restrict__ s, float* __restrict__ g_out, uint32_t* __restrict__ ws,
@@ -325,7 +330,8 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
     unsigned long long* counter = reinterpret_cast<unsigned long long*>(ws);
     uint32_t* amax = ws + 4;
     uint32_t* done = ws + 4 + batch;
-    const int64_t nT = (upm + NV_TILE_UNITS - 1) / NV_TILE_UNITS;
+    constexpr int tile = kThreads * upt;
+    const int64_t nT = (upm + tile - 1) / tile;
     const unsigned long long total = (unsigned long long)(2 * batch * nT);
     init_scale_tables(tab6, 6.0f);
     if (threadIdx.x < 128) {
@@ -341,8 +347,8 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
         const NvItem w = nv_decode(item, batch, nT);
         // this item's units: [base, base + n) of matrix w.b, addressed by
         // 32-bit offsets from the item's first unit
-        const int64_t base = w.b * upm + w.t * NV_TILE_UNITS;
-        const int n = (int)min64(NV_TILE_UNITS, upm - w.t * NV_TILE_UNITS);
+        const int64_t base = w.b * upm + w.t * tile;
+        const int n = (int)min64(tile, upm - w.t * tile);
         const uint4* xi = x + 2 * base;
         const int u0 = threadIdx.x;
         // The amax pass keeps its lines in L2 (evict-last) for the encode pass,
@@ -353,10 +359,10 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
             Unit cur;
             if (u0 < n) cur = load_unit_hint(xi, u0, keep);
 #pragma unroll
-            for (int i = 0; i < NV_UNITS_PER_THREAD; ++i) {
+            for (int i = 0; i < upt; ++i) {
                 const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, keep);
+                if (i + 1 < upt && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, keep);
                 if (u < n) m = max(m, unit_absmax(cur));
                 cur = nxt;
             }
@@ -386,10 +392,10 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
             uint2* qi = q + base;
             uint8_t* si = s + base;
 #pragma unroll 1
-            for (int i = 0; i < NV_UNITS_PER_THREAD; ++i) {
+            for (int i = 0; i < upt; ++i) {
                 const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < NV_UNITS_PER_THREAD && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, drop);
+                if (i + 1 < upt && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, drop);
                 if (u < n) nvfp4_encode_unit(cur, g, g_ok, gb, rg, tab6, s_dec, s_inv, qi + u, si + u);
                 cur = nxt;
             }
@@ -502,10 +508,15 @@ cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows,
         uint32_t* ws = (uint32_t*)workspace;
         cudaError_t e = cudaMemsetAsync(ws, 0, nvfp4_workspace_words(batch) * sizeof(uint32_t), st);
         if (e != cudaSuccess) return e;
-        const int64_t items = 2 * batch * ((upm + NV_TILE_UNITS - 1) / NV_TILE_UNITS);
-        const int grid = (int)max64(1, min64(items, (int64_t)sms * NV_MIN_BLOCKS));
-        quant_nvfp4_kernel<<<grid, kThreads, 0, st>>>((const uint4*)x, batch, upm, (uint2*)q, (uint8_t*)scales,
-                                                      tensor_scale, ws, err);
+        const int64_t slots = (int64_t)sms * NV_MIN_BLOCKS;
+        int upt = NV_UNITS_PER_THREAD;
+        while (upt > 1 && batch * ((upm + (int64_t)kThreads * upt - 1) / ((int64_t)kThreads * upt)) < 2 * slots) upt /= 2;
+        const int64_t items = 2 * batch * ((upm + (int64_t)kThreads * upt - 1) / ((int64_t)kThreads * upt));
+        const int grid = (int)max64(1, min64(items, slots));
+        auto kern = upt == 16 ? quant_nvfp4_kernel<16> : upt == 8 ? quant_nvfp4_kernel<8>
+                  : upt == 4 ? quant_nvfp4_kernel<4> : upt == 2 ? quant_nvfp4_kernel<2> : quant_nvfp4_kernel<1>;
+        kern<<<grid, kThreads, 0, st>>>((const uint4*)x, batch, upm, (uint2*)q, (uint8_t*)scales, tensor_scale, ws,
+                                        err);
         break;
     }
     default:
