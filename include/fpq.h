@@ -109,6 +109,9 @@ FPQ_API const char* fpq_status_string(fpq_status status);
 
 /* Detail of the last failing call on this host thread ("" if none). */
 FPQ_API const char* fpq_last_error_detail(void);
+/* The same text under the name of its most common use: after FPQ_ERR_CUDA
+ * it holds the failing call and the CUDA error string. */
+FPQ_API const char* fpq_last_cuda_error(void);
 
 /* Bytes of device workspace fpq_quantize_block needs for `fmt` and `batch`
  * (NVFP4: 16 + 8 * batch bytes -- a work-item counter, and per batch item

@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "fpq_version": (I32, []),
         "fpq_status_string": (ctypes.c_char_p, [I32]),
         "fpq_last_error_detail": (ctypes.c_char_p, []),
+        "fpq_last_cuda_error": (ctypes.c_char_p, []),
         "fpq_quantize_workspace_bytes": (SZ, [I32, I64]),
         "fpq_quantize_block": (I32, [I32, P, I64, I64, I64, P, P, P, P, SZ, P]),
         "fpq_dequantize": (I32, [I32, P, P, P, I64, I64, I64, P, P]),

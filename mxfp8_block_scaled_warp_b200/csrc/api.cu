@@ -132,6 +132,7 @@ const char* fpq_status_string(fpq_status s) {
 }
 
 const char* fpq_last_error_detail(void) { return t_detail; }
+const char* fpq_last_cuda_error(void) { return t_detail; }
 
 size_t fpq_quantize_workspace_bytes(fpq_format fmt, int64_t batch) {
     return (fmt == FPQ_NVFP4 && batch > 0) ? sizeof(uint32_t) * (size_t)fpq::nvfp4_workspace_words(batch) : 0;
