@@ -154,6 +154,29 @@ FPQ_API fpq_status fpq_dequantize(fpq_format fmt, const void* q, const void* sca
                           int64_t cols, void* out, void* stream);
 
 /*
+ * fpq_quantize_block_strided, fpq_dequantize_strided -- the same two
+ * operations on strided matrices: the bf16 operand and the code operand each
+ * have a row stride (ld_*) and a batch stride (bs_*), counted in ELEMENTS
+ * (for NVFP4 codes, two elements per byte); scales stay dense row-major as
+ * above.  Element (b, r, c) of the bf16 operand is at x + b*bs_x + r*ld_x + c
+ * (likewise out with ld_out, bs_out), and its code at element offset
+ * b*bs_q + r*ld_q + c of q.  Results are the same bytes as the dense calls
+ * on the same logical matrices.
+ *
+ * Requires, besides the dense calls' rules: every ld and bs a multiple of 16,
+ * ld >= cols, bs >= rows*ld when batch > 1.  The library does not check that
+ * strided operands do not overlap.  Errors: as the dense calls.
+ */
+FPQ_API fpq_status fpq_quantize_block_strided(fpq_format fmt, const void* x, int64_t ld_x, int64_t bs_x,
+                                              int64_t batch, int64_t rows, int64_t cols, void* q, int64_t ld_q,
+                                              int64_t bs_q, void* scales, float* tensor_scale, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+FPQ_API fpq_status fpq_dequantize_strided(fpq_format fmt, const void* q, int64_t ld_q, int64_t bs_q,
+                                          const void* scales, const float* tensor_scale, int64_t batch,
+                                          int64_t rows, int64_t cols, void* out, int64_t ld_out, int64_t bs_out,
+                                          void* stream);
+
+/*
  * fpq_lora_merge_fakequant -- the weight side of the QAT forward [QAT]:
  *   delta[n,k] = sum_{j<r} B[n,j] * A[j,k]   (fp32, fused multiply-adds,
  *                                              j ascending, from zero)

@@ -28,6 +28,7 @@ __all__ = [
     "fpq_get_device_error", "fpq_gemm_bf16", "fpq_gemm_bf16_layout", "fpq_transpose_bf16",
     "fpq_gemm_bf16_splitk_workspace_bytes", "fpq_gemm_bf16_splitk", "fpq_qat_backward_workspace_bytes",
     "fpq_moe_route_workspace_bytes", "fpq_moe_route", "fpq_moe_dispatch_layout", "fpq_moe_dispatch_mxfp8",
+    "fpq_quantize_block_strided", "fpq_dequantize_strided",
     "MOE_DIRECT", "MOE_PACK",
     "fpq_qat_backward",
     "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
@@ -87,6 +88,8 @@ def _load() -> ctypes.CDLL:
         "fpq_gemm_bf16_splitk": (I32, [P, I32, P, I32, I64, I64, I64, F, P, P, SZ, P]),
         "fpq_qat_backward_workspace_bytes": (SZ, [I64, I64, I64, I32]),
         "fpq_moe_route_workspace_bytes": (SZ, [I64, I32]),
+        "fpq_quantize_block_strided": (I32, [I32, P, I64, I64, I64, I64, I64, P, I64, I64, P, P, P, SZ, P]),
+        "fpq_dequantize_strided": (I32, [I32, P, I64, I64, P, P, I64, I64, I64, P, I64, I64, P]),
         "fpq_moe_route": (I32, [P, I64, I32, I32, P, P, SZ, P]),
         "fpq_moe_dispatch_layout": (I32, [P, I32, I32, I32, I32, P, P, P]),
         "fpq_moe_dispatch_mxfp8": (I32, [P, I64, I64, P, I32, I32, P, SZ, P, I32, P, P, P, P]),
@@ -175,6 +178,34 @@ def fpq_gemm_bf16_splitk(p, p_mn, q, q_mn, m, n, k, alpha, c, workspace, stream=
     _check(load().fpq_gemm_bf16_splitk(_ptr(p), int(p_mn), _ptr(q), int(q_mn), m, n, k, float(alpha), _ptr(c),
                                        _ptr(workspace) if workspace is not None else None, wsb, _stream(stream)),
            "fpq_gemm_bf16_splitk")
+
+
+def _ptr_rows(t: torch.Tensor | None):
+    """Address of a row-strided view (rows may be apart; each row contiguous)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the library must live on a CUDA device")
+    if t.stride(-1) != 1:
+        raise ValueError("the last dimension must be contiguous")
+    return t.data_ptr()
+
+
+def fpq_quantize_block_strided(fmt, x, ld_x, bs_x, batch, rows, cols, q, ld_q, bs_q, scales, tensor_scale=None,
+                               workspace=None, stream=None):
+    """x, q: views whose first element is (0, 0, 0); strides in elements
+    (NVFP4 codes: two per byte).  Scales dense."""
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().fpq_quantize_block_strided(fmt, _ptr_rows(x), ld_x, bs_x, batch, rows, cols, _ptr_rows(q), ld_q,
+                                             bs_q, _ptr(scales), _ptr(tensor_scale), _ptr(workspace), wsb,
+                                             _stream(stream)), "fpq_quantize_block_strided")
+
+
+def fpq_dequantize_strided(fmt, q, ld_q, bs_q, scales, tensor_scale, batch, rows, cols, out, ld_out, bs_out,
+                           stream=None):
+    _check(load().fpq_dequantize_strided(fmt, _ptr_rows(q), ld_q, bs_q, _ptr(scales), _ptr(tensor_scale), batch,
+                                         rows, cols, _ptr_rows(out), ld_out, bs_out, _stream(stream)),
+           "fpq_dequantize_strided")
 
 
 MOE_DIRECT, MOE_PACK = 0, 1

@@ -171,6 +171,66 @@ fpq_status fpq_dequantize(fpq_format fmt, const void* q, const void* scales, con
                                             (cudaStream_t)stream), "dequantize launch");
 }
 
+namespace {
+fpq_status check_strides(int64_t batch, int64_t rows, int64_t cols, int64_t ld, int64_t bs, const char* what) {
+    if (ld < cols || ld % 16 || ld > (1ll << 40) || (batch > 1 && (bs < rows * ld || bs % 16 || bs > (1ll << 44)))) {
+        set_detail(what);
+        return FPQ_ERR_INVALID_ARG;
+    }
+    return FPQ_OK;
+}
+}  // namespace
+
+fpq_status fpq_quantize_block_strided(fpq_format fmt, const void* x, int64_t ld_x, int64_t bs_x, int64_t batch,
+                                      int64_t rows, int64_t cols, void* q, int64_t ld_q, int64_t bs_q, void* scales,
+                                      float* tensor_scale, void* workspace, size_t workspace_bytes, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st = check_quant_shape(fmt, batch, rows, cols);
+    if (st != FPQ_OK) return st;
+    if ((st = check_strides(batch, rows, cols, ld_x, bs_x, "x strides: need ld >= cols, ld and bs multiples of 16, "
+                                                            "bs >= rows * ld")) != FPQ_OK)
+        return st;
+    if ((st = check_strides(batch, rows, cols, ld_q, bs_q, "q strides: need ld >= cols, ld and bs multiples of 16, "
+                                                            "bs >= rows * ld")) != FPQ_OK)
+        return st;
+    if ((st = check_ptrs({x, q, scales})) != FPQ_OK) return st;
+    if (fmt == FPQ_NVFP4) {
+        if ((st = check_ptrs({tensor_scale})) != FPQ_OK) return st;
+        if (!workspace || workspace_bytes < fpq_quantize_workspace_bytes(fmt, batch) || !aligned16(workspace)) {
+            set_detail("NVFP4 needs a 16-byte aligned workspace of fpq_quantize_workspace_bytes() bytes");
+            return FPQ_ERR_WORKSPACE;
+        }
+    }
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    const fpq::OperandStrides os{ld_x, batch > 1 ? bs_x : rows * ld_x, ld_q, batch > 1 ? bs_q : rows * ld_q};
+    return from_cuda(fpq::launch_quantize(fmt, x, batch, rows, cols, q, scales, tensor_scale, workspace, d->err,
+                                          d->sms, (cudaStream_t)stream, &os),
+                     "quantize launch");
+}
+
+fpq_status fpq_dequantize_strided(fpq_format fmt, const void* q, int64_t ld_q, int64_t bs_q, const void* scales,
+                                  const float* tensor_scale, int64_t batch, int64_t rows, int64_t cols, void* out,
+                                  int64_t ld_out, int64_t bs_out, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st = check_quant_shape(fmt, batch, rows, cols);
+    if (st != FPQ_OK) return st;
+    if ((st = check_strides(batch, rows, cols, ld_q, bs_q, "q strides: need ld >= cols, ld and bs multiples of 16, "
+                                                            "bs >= rows * ld")) != FPQ_OK)
+        return st;
+    if ((st = check_strides(batch, rows, cols, ld_out, bs_out, "out strides: need ld >= cols, ld and bs multiples of "
+                                                                "16, bs >= rows * ld")) != FPQ_OK)
+        return st;
+    if ((st = check_ptrs({q, scales, out})) != FPQ_OK) return st;
+    if (fmt == FPQ_NVFP4 && (st = check_ptrs({tensor_scale})) != FPQ_OK) return st;
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    const fpq::OperandStrides os{ld_q, batch > 1 ? bs_q : rows * ld_q, ld_out, batch > 1 ? bs_out : rows * ld_out};
+    return from_cuda(fpq::launch_dequantize(fmt, q, scales, tensor_scale, batch, rows, cols, out, d->sms,
+                                            (cudaStream_t)stream, &os),
+                     "dequantize launch");
+}
+
 fpq_status fpq_lora_merge_fakequant(const void* w, const void* lora_a, const void* lora_b, int64_t n,
                                     int64_t k, int32_t r, float alpha_over_r, void* wq, float* ws,
                                     void* w_fq, void* stream) {

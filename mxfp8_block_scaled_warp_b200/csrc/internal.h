@@ -12,14 +12,21 @@ namespace fpq {
 // counter per matrix.
 inline int64_t nvfp4_workspace_words(int64_t batch) { return 4 + 2 * batch; }
 
-// Quantize `batch` dense row-major bf16 matrices [rows, cols] (fmt: fpq_format).
+// Row and batch strides, in elements, of a kernel's input and output
+// operands (multiples of 16); nullptr means both are dense.  Scales are
+// always dense row-major.
+struct OperandStrides {
+    int64_t ld_in, bs_in, ld_out, bs_out;
+};
+
+// Quantize `batch` row-major bf16 matrices [rows, cols] (fmt: fpq_format).
 cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows, int64_t cols,
                             void* q, void* scales, float* tensor_scale, void* workspace,
-                            uint32_t* err, int sms, cudaStream_t st);
+                            uint32_t* err, int sms, cudaStream_t st, const OperandStrides* strides = nullptr);
 
 cudaError_t launch_dequantize(int fmt, const void* q, const void* scales, const float* tensor_scale,
                               int64_t batch, int64_t rows, int64_t cols, void* out, int sms,
-                              cudaStream_t st);
+                              cudaStream_t st, const OperandStrides* strides = nullptr);
 
 cudaError_t launch_lora_merge_fakequant(const void* w, const void* a, const void* b, int64_t n,
                                         int64_t k, int r, float alpha_over_r, void* wq, float* ws,

@@ -53,9 +53,10 @@ __device__ __forceinline__ float fp32_scale(uint32_t a) {
 
 // ----------------------------------------------------------------- MXFP8
 
+template <bool S>
 __global__ void __launch_bounds__(kThreads, 3)
 quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* __restrict__ s,
-                   int64_t units) {
+                   int64_t units, UnitStrides m) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
     for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll; base < units; base += stride) {
@@ -63,7 +64,7 @@ quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* 
 #pragma unroll
         for (int i = 0; i < kUnroll; ++i) {
             int64_t u = base + i * kThreads + threadIdx.x;
-            if (u < units) v[i] = load_unit(x, u);
+            if (u < units) v[i] = load_unit(x, in_unit<S>(m, u));
         }
 #pragma unroll
         for (int i = 0; i < kUnroll; ++i) {
@@ -76,7 +77,7 @@ quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* 
             uint4 out;
             if (e == 128) out = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
             else out = scale_to_e4m3(v[i], pow2_neg(e));
-            st_v4(q + u, out);
+            st_v4(q + out_unit<S>(m, u), out);
             if ((u & 1) == 0) s[u >> 1] = (uint8_t)(e + 127);
         }
     }
@@ -89,22 +90,23 @@ quant_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, uint8_t* 
 // the grid is sized to exactly that residency (grid-stride loop).
 constexpr int Q1_MIN_BLOCKS = 6;
 
+template <bool S>
 __global__ void __launch_bounds__(kThreads, Q1_MIN_BLOCKS)
 quant_fp8_1x128_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
-                       float* __restrict__ s, int64_t units) {
+                       float* __restrict__ s, int64_t units, UnitStrides m) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     __shared__ ScaleTables tab;                      // s = fp32(amax / 448) and its bracket, by mantissa
     init_scale_tables(tab, 448.0f);
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     Unit cur;
-    if (u < units) cur = load_unit(x, u);
+    if (u < units) cur = load_unit(x, in_unit<S>(m, u));
     __syncthreads();
     // The 8 lanes of a block are in range or out of range together (units
     // and stride are multiples of 8), so the shuffles stay converged.
     for (; u - threadIdx.x < units; u += stride) {
         Unit nxt;
-        if (u + stride < units) nxt = load_unit(x, u + stride);
+        if (u + stride < units) nxt = load_unit(x, in_unit<S>(m, u + stride));
         const uint32_t a = group_max<8>(u < units ? unit_absmax(cur) : 0u);
         if (u < units) {
             // exponent field >= 10 keeps s = fp32(amax / 448) and 1/s normal
@@ -120,7 +122,7 @@ quant_fp8_1x128_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
                 sc = fp32_scale(a);
                 out = divide_to_e4m3(cur, sc);
             }
-            st_v4(q + u, out);
+            st_v4(q + out_unit<S>(m, u), out);
             if ((u & 7) == 0) s[u >> 3] = sc;
         }
         cur = nxt;
@@ -141,9 +143,11 @@ constexpr int QB_THREADS = 512;
 constexpr int QB_CHUNKS = 128 * 16 / QB_THREADS;
 constexpr int QB_WARPS = QB_THREADS / 32;
 
+// S: strided operands (row and batch strides in elements); dense otherwise.
+template <bool S>
 __global__ void __launch_bounds__(QB_THREADS, 2048 / QB_THREADS)
 quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s,
-                         int64_t rows, int64_t cols) {
+                         int64_t rows, int64_t cols, int64_t ldx, int64_t bsx, int64_t ldq, int64_t bsq) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     __shared__ uint32_t red[QB_WARPS];
     const int64_t nbr = (rows + 127) / 128, nbc = cols / 128;
@@ -152,12 +156,13 @@ quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
     const int rmax = (int)min64(128, rows - bi * 128);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row0 = b * rows + bi * 128;
-    const uint8_t* xb = x + (row0 * cols + bj * 128) * 2;
+    if (!S) ldx = ldq = cols;
+    const uint8_t* xb = S ? x + (b * bsx + bi * 128 * ldx + bj * 128) * 2 : x + (row0 * cols + bj * 128) * 2;
     uint4 v[QB_CHUNKS];
 #pragma unroll
     for (int i = 0; i < QB_CHUNKS; ++i) {
         const int c = threadIdx.x + QB_THREADS * i, r = c >> 4;
-        v[i] = r < rmax ? ld_stream(xb + (int64_t)r * cols * 2 + (c & 15) * 16) : make_uint4(0, 0, 0, 0);
+        v[i] = r < rmax ? ld_stream(xb + (int64_t)r * ldx * 2 + (c & 15) * 16) : make_uint4(0, 0, 0, 0);
     }
     uint32_t m = 0;
 #pragma unroll
@@ -173,7 +178,7 @@ quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
     if (threadIdx.x == 0) s[idx] = sc;
     const bool fast = reciprocal_ok(sc);
     const QuotientBracket br = quotient_bracket(fast ? sc : 1.0f);
-    uint8_t* qb = q + row0 * cols + bj * 128;
+    uint8_t* qb = S ? q + b * bsq + bi * 128 * ldq + bj * 128 : q + row0 * cols + bj * 128;
 #pragma unroll
     for (int i = 0; i < QB_CHUNKS; ++i) {
         const int c = threadIdx.x + QB_THREADS * i, r = c >> 4, c8 = (c & 15) * 8;
@@ -184,7 +189,7 @@ quant_fp8_128x128_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ q,
             for (int j = 0; j < 4; ++j)
                 e[j] = fast ? e4m3x2_of_quotients(bf16_lo(w[j]), bf16_hi(w[j]), br)
                             : f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(w[j]), sc), __fdiv_rn(bf16_hi(w[j]), sc));
-            st_v2(qb + (int64_t)r * cols + c8, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
+            st_v2(qb + (int64_t)r * ldq + c8, make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16)));
         }
     }
 }
@@ -315,11 +320,11 @@ __device__ __forceinline__ void nvfp4_encode_unit(const Unit& v, float g, bool g
     *sdst = (uint8_t)code;
 }
 
-template <int upt>
+template <int upt, bool S>
 __global__ void __launch_bounds__(kThreads, NV_MIN_BLOCKS)
 quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint2* __restrict__ q,
                    uint8_t* __restrict__ s, float* __restrict__ g_out, uint32_t* __restrict__ ws,
-                   uint32_t* err) {
+                   uint32_t* err, UnitStrides m) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     __shared__ ScaleTables tab6;                 // fp32(amax_b / 6) by mantissa
     __shared__ float s_dec[128];                 // dec(c) for E4M3 codes c = 0..126
@@ -355,19 +360,21 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
         // which reads them a matrix later and lets them go (evict-first).
         if (w.is_a) {
             const uint64_t keep = l2_policy_evict_last();
-            uint32_t m = 0;
+            uint32_t am = 0;
             Unit cur;
-            if (u0 < n) cur = load_unit_hint(xi, u0, keep);
+            if (u0 < n) cur = S ? load_unit_hint(x, in_unit<S>(m, base + u0), keep) : load_unit_hint(xi, u0, keep);
 #pragma unroll
             for (int i = 0; i < upt; ++i) {
                 const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < upt && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, keep);
-                if (u < n) m = max(m, unit_absmax(cur));
+                if (i + 1 < upt && u + kThreads < n)
+                    nxt = S ? load_unit_hint(x, in_unit<S>(m, base + u + kThreads), keep)
+                            : load_unit_hint(xi, u + kThreads, keep);
+                if (u < n) am = max(am, unit_absmax(cur));
                 cur = nxt;
             }
-            m = group_max<32>(m);
-            if ((threadIdx.x & 31) == 0) s_wmax[threadIdx.x >> 5] = m;
+            am = group_max<32>(am);
+            if ((threadIdx.x & 31) == 0) s_wmax[threadIdx.x >> 5] = am;
             __syncthreads();
             if (threadIdx.x == 0) {
                 uint32_t mm = 0;
@@ -380,7 +387,8 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
         } else {
             const uint64_t drop = l2_policy_evict_first();
             Unit cur;
-            if (u0 < n) cur = load_unit_hint(xi, u0, drop);    // the input is ready; only g must wait
+            if (u0 < n)                                 // the input is ready; only g must wait
+                cur = S ? load_unit_hint(x, in_unit<S>(m, base + u0), drop) : load_unit_hint(xi, u0, drop);
             if (threadIdx.x == 0) s_ok = wait_count(done + w.b, (uint32_t)nT, err) ? 1 : 0;
             __syncthreads();
             if (!s_ok) return;
@@ -395,8 +403,12 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
             for (int i = 0; i < upt; ++i) {
                 const int u = u0 + i * kThreads;
                 Unit nxt;
-                if (i + 1 < upt && u + kThreads < n) nxt = load_unit_hint(xi, u + kThreads, drop);
-                if (u < n) nvfp4_encode_unit(cur, g, g_ok, gb, rg, tab6, s_dec, s_inv, qi + u, si + u);
+                if (i + 1 < upt && u + kThreads < n)
+                    nxt = S ? load_unit_hint(x, in_unit<S>(m, base + u + kThreads), drop)
+                            : load_unit_hint(xi, u + kThreads, drop);
+                if (u < n)
+                    nvfp4_encode_unit(cur, g, g_ok, gb, rg, tab6, s_dec, s_inv,
+                                      S ? q + out_unit<S>(m, base + u) : qi + u, si + u);
                 cur = nxt;
             }
         }
@@ -419,15 +431,15 @@ __device__ __forceinline__ void store_bf16x16(uint4* out, int64_t u, const float
 
 // fmt: 0 = 1x128 (fp32 scale per 8 units), 2 = MXFP8 (E8M0 per 2 units),
 // 1 = 128x128 (fp32 scale per 128x128 block).
-template <int kFmt>
+template <int kFmt, bool S>
 __global__ void __launch_bounds__(kThreads, 3)
 dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales, uint4* __restrict__ out,
-                   int64_t units, int64_t rows, int64_t cols) {
+                   int64_t units, int64_t rows, int64_t cols, UnitStrides m) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     const int64_t units_per_row = cols / 16;
     for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
-        uint4 c = ld_stream(q + u);
+        uint4 c = ld_stream(q + in_unit<S>(m, u));
         float sc;
         if (kFmt == 2) {
             uint32_t code = ((const uint8_t*)scales)[u >> 1];
@@ -449,27 +461,28 @@ dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales,
             f[4 * j + 0] = lo.x * sc; f[4 * j + 1] = lo.y * sc;
             f[4 * j + 2] = hi.x * sc; f[4 * j + 3] = hi.y * sc;
         }
-        store_bf16x16(out, u, f);
+        store_bf16x16(out, out_unit<S>(m, u), f);
     }
 }
 
+template <bool S>
 __global__ void __launch_bounds__(kThreads, 3)
 dequant_nvfp4_kernel(const uint2* __restrict__ q, const uint8_t* __restrict__ s, const float* __restrict__ g,
-                     uint4* __restrict__ out, int64_t units, int64_t units_per_matrix) {
+                     uint4* __restrict__ out, int64_t units, int64_t units_per_matrix, UnitStrides m) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
-        uint2 c = q[u];
-        const float S = e4m3_to_f32(s[u]) * g[u / units_per_matrix];
+        uint2 c = q[in_unit<S>(m, u)];
+        const float Sc = e4m3_to_f32(s[u]) * g[u / units_per_matrix];
         uint32_t w[2] = {c.x, c.y};
         float f[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             float2 e = e2m1x2_to_f32x2((w[j >> 2] >> (8 * (j & 3))) & 0xFFu);
-            f[2 * j] = e.x * S;
-            f[2 * j + 1] = e.y * S;
+            f[2 * j] = e.x * Sc;
+            f[2 * j + 1] = e.y * Sc;
         }
-        store_bf16x16(out, u, f);
+        store_bf16x16(out, out_unit<S>(m, u), f);
     }
 }
 
@@ -483,24 +496,53 @@ int grid_for(int64_t work_items, int per_cta, int sms) {
 
 // ----------------------------------------------------------------- launchers
 
+namespace {
+// Unit strides of an operand pair; `strided` false when both are dense.
+UnitStrides unit_strides(const OperandStrides* os, int64_t rows, int64_t cols, bool& strided) {
+    const int64_t upr = cols / 16;
+    UnitStrides m{upr, rows * upr, upr, rows * upr, upr, rows * upr};
+    strided = false;
+    if (os) {
+        m.in_ld = os->ld_in / 16;
+        m.in_bs = os->bs_in / 16;
+        m.out_ld = os->ld_out / 16;
+        m.out_bs = os->bs_out / 16;
+        strided = m.in_ld != upr || m.in_bs != rows * upr || m.out_ld != upr || m.out_bs != rows * upr;
+    }
+    return m;
+}
+}  // namespace
+
 cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows, int64_t cols,
                             void* q, void* scales, float* tensor_scale, void* workspace,
-                            uint32_t* err, int sms, cudaStream_t st) {
+                            uint32_t* err, int sms, cudaStream_t st, const OperandStrides* strides) {
     const int64_t n = batch * rows * cols, units = n / 16;
+    bool sd = false;
+    const UnitStrides m = unit_strides(strides, rows, cols, sd);
     switch (fmt) {
-    case FPQ_MXFP8:
-        quant_mxfp8_kernel<<<grid_for(units, kThreads * kUnroll, sms), kThreads, 0, st>>>(
-            (const uint4*)x, (uint4*)q, (uint8_t*)scales, units);
+    case FPQ_MXFP8: {
+        const int grid = grid_for(units, kThreads * kUnroll, sms);
+        if (sd) quant_mxfp8_kernel<true><<<grid, kThreads, 0, st>>>((const uint4*)x, (uint4*)q, (uint8_t*)scales,
+                                                                    units, m);
+        else quant_mxfp8_kernel<false><<<grid, kThreads, 0, st>>>((const uint4*)x, (uint4*)q, (uint8_t*)scales,
+                                                                  units, m);
         break;
-    case FPQ_FP8_1x128:
-        quant_fp8_1x128_kernel<<<(int)max64(1, min64((units + kThreads - 1) / kThreads, (int64_t)sms * Q1_MIN_BLOCKS)),
-                                 kThreads, 0, st>>>(
-            (const uint4*)x, (uint4*)q, (float*)scales, units);
+    }
+    case FPQ_FP8_1x128: {
+        const int grid = (int)max64(1, min64((units + kThreads - 1) / kThreads, (int64_t)sms * Q1_MIN_BLOCKS));
+        if (sd) quant_fp8_1x128_kernel<true><<<grid, kThreads, 0, st>>>((const uint4*)x, (uint4*)q, (float*)scales,
+                                                                        units, m);
+        else quant_fp8_1x128_kernel<false><<<grid, kThreads, 0, st>>>((const uint4*)x, (uint4*)q, (float*)scales,
+                                                                      units, m);
         break;
+    }
     case FPQ_FP8_128x128: {
         const int64_t nblocks = batch * ((rows + 127) / 128) * (cols / 128);
-        quant_fp8_128x128_kernel<<<(unsigned)nblocks, QB_THREADS, 0, st>>>((const uint8_t*)x, (uint8_t*)q,
-                                                                          (float*)scales, rows, cols);
+        const int64_t ldx = strides ? strides->ld_in : cols, bsx = strides ? strides->bs_in : rows * cols;
+        const int64_t ldq = strides ? strides->ld_out : cols, bsq = strides ? strides->bs_out : rows * cols;
+        (sd ? quant_fp8_128x128_kernel<true> : quant_fp8_128x128_kernel<false>)<<<(unsigned)nblocks, QB_THREADS, 0,
+                                                                                 st>>>(
+            (const uint8_t*)x, (uint8_t*)q, (float*)scales, rows, cols, ldx, bsx, ldq, bsq);
         break;
     }
     case FPQ_NVFP4: {
@@ -513,10 +555,14 @@ cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows,
         while (upt > 1 && batch * ((upm + (int64_t)kThreads * upt - 1) / ((int64_t)kThreads * upt)) < 2 * slots) upt /= 2;
         const int64_t items = 2 * batch * ((upm + (int64_t)kThreads * upt - 1) / ((int64_t)kThreads * upt));
         const int grid = (int)max64(1, min64(items, slots));
-        auto kern = upt == 16 ? quant_nvfp4_kernel<16> : upt == 8 ? quant_nvfp4_kernel<8>
-                  : upt == 4 ? quant_nvfp4_kernel<4> : upt == 2 ? quant_nvfp4_kernel<2> : quant_nvfp4_kernel<1>;
+        auto kern = sd ? (upt == 16 ? quant_nvfp4_kernel<16, true> : upt == 8 ? quant_nvfp4_kernel<8, true>
+                          : upt == 4 ? quant_nvfp4_kernel<4, true> : upt == 2 ? quant_nvfp4_kernel<2, true>
+                          : quant_nvfp4_kernel<1, true>)
+                       : (upt == 16 ? quant_nvfp4_kernel<16, false> : upt == 8 ? quant_nvfp4_kernel<8, false>
+                          : upt == 4 ? quant_nvfp4_kernel<4, false> : upt == 2 ? quant_nvfp4_kernel<2, false>
+                          : quant_nvfp4_kernel<1, false>);
         kern<<<grid, kThreads, 0, st>>>((const uint4*)x, batch, upm, (uint2*)q, (uint8_t*)scales, tensor_scale, ws,
-                                        err);
+                                        err, m);
         break;
     }
     default:
@@ -526,26 +572,33 @@ cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows,
 }
 
 cudaError_t launch_dequantize(int fmt, const void* q, const void* scales, const float* tensor_scale,
-                              int64_t batch, int64_t rows, int64_t cols, void* out, int sms, cudaStream_t st) {
+                              int64_t batch, int64_t rows, int64_t cols, void* out, int sms, cudaStream_t st,
+                              const OperandStrides* strides) {
     const int64_t units = batch * rows * cols / 16;
     const int grid = grid_for(units, kThreads, sms);
+    bool sd = false;
+    const UnitStrides m = unit_strides(strides, rows, cols, sd);
+#define FPQ_DEQ(F)                                                                                                \
+    (sd ? dequant_fp8_kernel<F, true> : dequant_fp8_kernel<F, false>)<<<grid, kThreads, 0, st>>>(                 \
+        (const uint4*)q, scales, (uint4*)out, units, rows, cols, m)
     switch (fmt) {
     case FPQ_MXFP8:
-        dequant_fp8_kernel<2><<<grid, kThreads, 0, st>>>((const uint4*)q, scales, (uint4*)out, units, rows, cols);
+        FPQ_DEQ(2);
         break;
     case FPQ_FP8_1x128:
-        dequant_fp8_kernel<0><<<grid, kThreads, 0, st>>>((const uint4*)q, scales, (uint4*)out, units, rows, cols);
+        FPQ_DEQ(0);
         break;
     case FPQ_FP8_128x128:
-        dequant_fp8_kernel<1><<<grid, kThreads, 0, st>>>((const uint4*)q, scales, (uint4*)out, units, rows, cols);
+        FPQ_DEQ(1);
         break;
     case FPQ_NVFP4:
-        dequant_nvfp4_kernel<<<grid, kThreads, 0, st>>>((const uint2*)q, (const uint8_t*)scales, tensor_scale,
-                                                        (uint4*)out, units, rows * cols / 16);
+        (sd ? dequant_nvfp4_kernel<true> : dequant_nvfp4_kernel<false>)<<<grid, kThreads, 0, st>>>(
+            (const uint2*)q, (const uint8_t*)scales, tensor_scale, (uint4*)out, units, rows * cols / 16, m);
         break;
     default:
         return cudaErrorInvalidValue;
     }
+#undef FPQ_DEQ
     return cudaGetLastError();
 }
 

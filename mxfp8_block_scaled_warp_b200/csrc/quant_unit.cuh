@@ -58,4 +58,30 @@ __device__ __forceinline__ uint4 scale_to_e4m3(const Unit& v, float mul) {
     return make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
 }
 
+// Strided operands.  Flat unit u of `batch` [rows, cols] matrices (u =
+// (b rows + r) cols / 16 + c) lives at unit b bs + r ld + c of an operand
+// with row stride ld and batch stride bs, both counted in units of 16
+// elements (whatever the element width).  Dense operands (S = false) use u
+// itself.
+struct UnitStrides {
+    int64_t upr, upm;          // units per row, per matrix
+    int64_t in_ld, in_bs;      // the kernel's input operand
+    int64_t out_ld, out_bs;    // the kernel's output operand
+};
+
+__device__ __forceinline__ int64_t unit_at(int64_t u, int64_t upr, int64_t upm, int64_t ld, int64_t bs) {
+    const int64_t b = u / upm, rem = u - b * upm, r = rem / upr;
+    return b * bs + r * ld + (rem - r * upr);
+}
+
+template <bool S>
+__device__ __forceinline__ int64_t in_unit(const UnitStrides& m, int64_t u) {
+    return S ? unit_at(u, m.upr, m.upm, m.in_ld, m.in_bs) : u;
+}
+
+template <bool S>
+__device__ __forceinline__ int64_t out_unit(const UnitStrides& m, int64_t u) {
+    return S ? unit_at(u, m.upr, m.upm, m.out_ld, m.out_bs) : u;
+}
+
 }  // namespace fpq
