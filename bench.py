@@ -670,6 +670,12 @@ def cpu_baseline(workload: str, budget_s: float = 12.0):
         return _cpu_baseline_nvfp4_gemm(oracle, budget_s)
     if workload == "moe_dispatch":
         return _cpu_baseline_moe_dispatch(oracle, budget_s)
+    if workload == "qat_forward":
+        return _cpu_baseline_qat_forward(oracle, budget_s)
+    if workload == "qat_backward":
+        return _cpu_baseline_qat_backward(oracle, budget_s)
+    if workload == "moe_grouped":
+        return _cpu_baseline_moe_grouped(oracle, budget_s)
     if workload != "ds_fp8_gemm":
         return None
     m, n, k = 4096, 2048, 7168
@@ -732,6 +738,89 @@ def _cpu_baseline_nvfp4_gemm(oracle, budget_s: float):
             "kind": "oracle",
             "sample": f"NVFP4 quantize of {rows} rows of each 7168-wide operand, {count} fp64 GEMM entries "
                       f"(K=7168); extrapolated to the full 4096x2048x7168 step ({step_s:.1f} s per step on one core)"}
+
+
+def _timed_entries(fn, probe_count, budget_s):
+    """Seconds per entry of fn(count), calibrated on probe_count entries and
+    then measured on as many as the budget allows; returns (per, count)."""
+    t0 = time.perf_counter()
+    fn(probe_count)
+    per = (time.perf_counter() - t0) / probe_count
+    count = int(max(probe_count, min(200000, budget_s / max(per, 1e-9))))
+    t0 = time.perf_counter()
+    fn(count)
+    return (time.perf_counter() - t0) / count, count
+
+
+def _cpu_baseline_qat_forward(oracle, budget_s: float):
+    """The oracle's LoRA merge + 128x128 fake-quant on the first 128 rows of
+    W, its 1x128 quantize of 64 rows of X and fp64 GEMM entries (K = 7168),
+    extrapolated to the whole 8192x2048x7168 step."""
+    m, n, k = 8192, 2048, 7168
+    wl = workloads.qat_forward()
+    w, la, lb, x = (workloads.as_u16(wl[t]) for t in ("w", "lora_a", "lora_b", "x"))
+    t0 = time.perf_counter()
+    qw, sw, _ = oracle.lora_merge_fakequant(w[:128], la, lb[:128], wl["alpha_over_r"])
+    t_merge = (time.perf_counter() - t0) / 128
+    t0 = time.perf_counter()
+    qx, sx = oracle.quant_fp8_1x128(x[:64])
+    t_qx = (time.perf_counter() - t0) / 64
+    rng = np.random.default_rng(0)
+    per, count = _timed_entries(lambda c: oracle.gemm_entries(0, qx, sx, 1, qw, sw, rng.integers(0, 64, c),
+                                                              rng.integers(0, 128, c)), 64, budget_s * 0.8)
+    step_s = t_merge * n + t_qx * m + per * m * n
+    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "work": 2.0 * m * n * k, "cores": 1,
+            "kind": "oracle",
+            "sample": f"LoRA merge + 128x128 fake-quant of 128 rows of W, 1x128 quantize of 64 rows of X, {count} "
+                      f"fp64 GEMM entries (K=7168); extrapolated to the full step ({step_s:.1f} s on one core)"}
+
+
+def _cpu_baseline_qat_backward(oracle, budget_s: float):
+    """The oracle's fp64 bf16-product entries at the contraction lengths of
+    the four products (2048 for dX and dA, 8192 for dW_eff, 7168 for dB),
+    extrapolated to every entry of the step."""
+    m, n, k, r = 8192, 2048, 7168, 16
+    rng = np.random.default_rng(0)
+    per_k = {}
+    counts = {}
+    for kk in (2048, 7168, 8192):
+        p = workloads.as_u16(workloads.normal_bf16((64, kk), 1.0, seed=6000 + kk))
+        q = workloads.as_u16(workloads.normal_bf16((64, kk), 0.02, seed=6001 + kk))
+        per_k[kk], counts[kk] = _timed_entries(
+            lambda c: oracle.gemm_bf16_entries(p, q, rng.integers(0, 64, c), rng.integers(0, 64, c)), 32,
+            budget_s / 3)
+    step_s = per_k[2048] * (m * k + r * k) + per_k[8192] * n * k + per_k[7168] * n * r
+    flops = 2.0 * (2 * m * n * k + 2 * r * n * k)
+    return {"value": flops / step_s / 1e12, "unit": "TFLOP/s", "work": flops, "cores": 1, "kind": "oracle",
+            "sample": f"{sum(counts.values())} fp64 bf16-product entries at K = 2048, 7168 and 8192; extrapolated "
+                      f"to dX, dW_eff, dA and dB in full ({step_s:.0f} s on one core)"}
+
+
+def _cpu_baseline_moe_grouped(oracle, budget_s: float):
+    """The oracle's dispatch of the first tokens and grouped MXFP8 GEMM
+    entries (K = 7168) against two quantized expert slices, extrapolated to
+    the 16384-token step (131072 rows x 2048 columns)."""
+    tokens, experts, k, n, topk = 16384, 64, 7168, 2048, 8
+    wl = workloads.moe_dispatch(tokens=tokens)
+    x, ids = workloads.as_u16(wl["x"][0]), wl["topk_ids"][0].numpy()
+    nt = 256
+    t0 = time.perf_counter()
+    codes, scales, offs = oracle.moe_dispatch([x[:nt]], [ids[:nt]], experts)[0]
+    t_tok = (time.perf_counter() - t0) / nt
+    wq, ws = oracle.quant_mxfp8(np.stack([workloads.as_u16(workloads.normal_bf16((64, k), 0.02, seed=5100 + e))
+                                          for e in range(2)]))
+    rows = min(codes.shape[0], 256)
+    off2 = np.array([0, rows // 2, rows], np.int64)
+    rng = np.random.default_rng(0)
+    per, count = _timed_entries(lambda c: oracle.grouped_gemm_entries(2, codes[:rows], scales[:rows], wq, ws, off2,
+                                                                      rng.integers(0, rows, c),
+                                                                      rng.integers(0, 64, c)), 64, budget_s * 0.8)
+    step_s = t_tok * tokens + per * tokens * topk * n
+    flops = 2.0 * tokens * topk * n * k
+    return {"value": flops / step_s / 1e12, "unit": "TFLOP/s", "work": flops, "cores": 1, "kind": "oracle",
+            "sample": f"oracle dispatch of {nt} tokens, {count} fp64 grouped MXFP8 GEMM entries (K=7168) against "
+                      f"two quantized expert slices; extrapolated to the 16384-token step ({step_s:.0f} s on one "
+                      f"core)"}
 
 
 def _cpu_baseline_moe_dispatch(oracle, budget_s: float):
