@@ -382,7 +382,8 @@ FPQ_API fpq_status fpq_qat_backward(const void* dy, const void* x_fq, const void
  *   dst_capacity  DEVICE int64 [n_dest]: rows of each buffer; a row outside
  *               raises FPQ_ERR_DEVICE_BAD_INPUT and is not written
  *
- * Requires tokens >= 0, 1 <= topk <= 32, 1 <= E <= 1024, world >= 1 dividing
+ * Requires tokens >= 0, 1 <= topk <= 32, tokens * topk < 2^31 (counts and
+ * group offsets are int32), 1 <= E <= 1024, world >= 1 dividing
  * E, 0 <= rank < world, n_dest >= 1 dividing E; the pointer arguments of
  * fpq_moe_dispatch_mxfp8 16-byte aligned.  Errors: FPQ_ERR_INVALID_ARG,
  * FPQ_ERR_ALIGNMENT, FPQ_ERR_WORKSPACE, FPQ_ERR_CUDA.

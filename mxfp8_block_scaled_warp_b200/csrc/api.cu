@@ -336,8 +336,10 @@ fpq_status fpq_moe_route(const int32_t* topk_ids, int64_t tokens, int32_t topk, 
                          int32_t* counts, void* workspace, size_t workspace_bytes, void* stream) {
     t_detail[0] = 0;
     fpq_status st;
-    if (tokens < 0 || tokens > (1ll << 31) || topk < 1 || topk > 32 || num_experts < 1 || num_experts > 1024) {
-        set_detail("need tokens >= 0, topk in [1, 32], num_experts in [1, 1024]");
+    if (tokens < 0 || topk < 1 || topk > 32 || tokens * topk >= (1ll << 31) || num_experts < 1 ||
+        num_experts > 1024) {
+        set_detail("need tokens >= 0, topk in [1, 32], tokens * topk < 2^31 (int32 counts), num_experts in "
+                   "[1, 1024]");
         return FPQ_ERR_INVALID_ARG;
     }
     if (!counts || (tokens > 0 && !topk_ids)) {
@@ -382,8 +384,9 @@ fpq_status fpq_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hidden,
                                   void* const* dst_scales, const int64_t* dst_capacity, void* stream) {
     t_detail[0] = 0;
     fpq_status st;
-    if (tokens < 0 || tokens > (1ll << 31) || hidden < 32 || hidden % 32 || hidden > (1 << 24) || topk < 1 ||
-        topk > 32 || num_experts < 1 || num_experts > 1024 || n_dest < 1 || num_experts % n_dest) {
+    if (tokens < 0 || hidden < 32 || hidden % 32 || hidden > (1 << 24) || topk < 1 || topk > 32 ||
+        tokens * topk >= (1ll << 31) || num_experts < 1 || num_experts > 1024 || n_dest < 1 ||
+        num_experts % n_dest) {
         set_detail("need tokens >= 0, hidden a positive multiple of 32, topk in [1, 32], num_experts in "
                    "[1, 1024], n_dest >= 1 dividing num_experts");
         return FPQ_ERR_INVALID_ARG;

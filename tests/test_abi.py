@@ -67,6 +67,28 @@ def test_host_side_validation(lib):
     assert L.fpq_scaled_gemm(f.MXFP8, ok_ptr, ok_ptr, f.MXFP8, ok_ptr, ok_ptr, 64, 250, 128, ok_ptr, 0, None) == 1
 
 
+def test_moe_dispatch_host_side_validation(lib):
+    L, _ = lib
+    P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    L.fpq_moe_route.restype = I32
+    L.fpq_moe_route.argtypes = [P, I64, I32, I32, P, P, ctypes.c_size_t, P]
+    L.fpq_moe_dispatch_layout.restype = I32
+    L.fpq_moe_dispatch_layout.argtypes = [P, I32, I32, I32, I32, P, P, P]
+    L.fpq_moe_dispatch_mxfp8.restype = I32
+    L.fpq_moe_dispatch_mxfp8.argtypes = [P, I64, I64, P, I32, I32, P, ctypes.c_size_t, P, I32, P, P, P, P]
+    ok = 1 << 20
+    assert L.fpq_moe_route(ok, 16, 33, 8, ok, ok, 1 << 20, None) == 1            # topk above 32
+    assert L.fpq_moe_route(ok, 1 << 27, 32, 8, ok, ok, 1 << 30, None) == 1       # 2^32 pairs: int32 counts overflow
+    assert L.fpq_moe_route(ok, 16, 2, 2048, ok, ok, 1 << 20, None) == 1          # too many experts
+    assert L.fpq_moe_route(ok, 16, 2, 8, ok, None, 0, None) == 7                 # no workspace
+    assert L.fpq_moe_dispatch_layout(ok, 3, 8, 0, 0, ok, ok, None) == 1          # world does not divide E
+    assert L.fpq_moe_dispatch_layout(ok, 2, 8, 2, 0, ok, ok, None) == 1          # rank out of range
+    assert L.fpq_moe_dispatch_layout(ok, 2, 8, 0, 5, ok, ok, None) == 1          # unknown mode
+    assert L.fpq_moe_dispatch_mxfp8(ok, 16, 48, ok, 2, 8, ok, 1 << 20, ok, 1, ok, ok, ok, None) == 1  # hidden % 32
+    assert L.fpq_moe_dispatch_mxfp8(ok, 16, 64, ok, 2, 8, ok, 1 << 20, ok, 3, ok, ok, ok, None) == 1  # n_dest ∤ E
+    assert L.fpq_moe_dispatch_mxfp8(ok + 4, 16, 64, ok, 2, 8, ok, 1 << 20, ok, 1, ok, ok, ok, None) == 2
+
+
 def test_no_device_is_unsupported_not_fallback(lib):
     """Valid arguments on a machine without a GPU: the call refuses with
     FPQ_ERR_UNSUPPORTED instead of computing anything on the host."""
