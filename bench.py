@@ -975,6 +975,8 @@ def main():
     dev = torch.device("cuda", local)
     pg = init_replicas(world, "nccl", dev)
 
+    if args.experts and args.workload != "moe_prequant":
+        raise SystemExit("--experts applies to --workload moe_prequant only")
     step = STEPS[args.workload](fpq, dev, **({"experts": args.experts} if args.experts else {}))
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
