@@ -268,7 +268,8 @@ FPQ_API fpq_status fpq_gemm_bf16_layout(const void* p, int32_t p_mn, const void*
  * fpq_gemm_bf16_splitk -- as fpq_gemm_bf16_layout for products with few
  * output tiles and a long contraction (m or n small, as for the LoRA
  * gradients of the QAT backward): the contraction is cut into up to 16
- * slices spread over the SMs, each slice's fp32 sums go to the workspace,
+ * slices spread over the SMs (about one CTA per SM; a product with many
+ * output tiles takes one slice), each slice's fp32 sums go to the workspace,
  * and a second kernel adds the slices in order, multiplies by alpha and
  * rounds to bf16 (so results are repeatable run to run).
  *

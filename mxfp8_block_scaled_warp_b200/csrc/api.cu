@@ -408,7 +408,7 @@ fpq_status fpq_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hidden,
 
 size_t fpq_gemm_bf16_splitk_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 1 || n < 1 || k < 1) return 0;
-    return (size_t)fpq::kMaxSplits * (size_t)m * (size_t)n * 4;
+    return (size_t)fpq::bf16_split_bound(m, n, k) * (size_t)m * (size_t)n * 4;
 }
 
 fpq_status fpq_gemm_bf16_splitk(const void* p, int32_t p_mn, const void* q, int32_t q_mn, int64_t m, int64_t n,

@@ -325,12 +325,18 @@ cudaError_t launch_gemm_bf16(const void* p, bool p_mn, const void* q, bool q_mn,
     return launch_any(p, p_mn, q, q_mn, m, n, k, alpha, c, err, nullptr, 1, 0, st);
 }
 
-int bf16_split_count(int64_t m, int64_t n, int64_t k, int sms) {
+int bf16_split_bound(int64_t m, int64_t n, int64_t k) {
     const int64_t tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int64_t kt = (k + BK - 1) / BK;
-    int64_t splits = (int64_t)sms / tiles;                            // one wave (one CTA per SM)
-    splits = std::min<int64_t>(splits, std::min<int64_t>(kMaxSplits, kt / 2));   // at least two K tiles each
-    return (int)std::max<int64_t>(splits, 1);
+    // at most kSplitSms / tiles slices (kSplitSms is above any SM count), at
+    // most kMaxSplits, at least two K tiles each
+    return (int)std::max<int64_t>(1, std::min<int64_t>(kSplitSms / tiles, std::min<int64_t>(kMaxSplits, kt / 2)));
+}
+
+int bf16_split_count(int64_t m, int64_t n, int64_t k, int sms) {
+    const int64_t tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
+    const int64_t splits = (int64_t)std::min(sms, kSplitSms) / tiles;     // one wave (one CTA per SM)
+    return (int)std::max<int64_t>(1, std::min<int64_t>(splits, bf16_split_bound(m, n, k)));
 }
 
 cudaError_t launch_gemm_bf16_splitk(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n,

@@ -55,6 +55,8 @@ cudaError_t launch_gemm_bf16(const void* p, bool p_mn, const void* q, bool q_mn,
 // `splits` K slices in `partial` ([splits, m, n] fp32), then a reduce kernel
 // writes bf16(alpha * sum) to c; m * n a multiple of 4.
 constexpr int kMaxSplits = 16;
+constexpr int kSplitSms = 256;
+int bf16_split_bound(int64_t m, int64_t n, int64_t k);          // slices the workspace must hold
 int bf16_split_count(int64_t m, int64_t n, int64_t k, int sms);
 cudaError_t launch_gemm_bf16_splitk(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n,
                                     int64_t k, float alpha, void* c, float* partial, int splits, uint32_t* err,
