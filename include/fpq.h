@@ -9,16 +9,21 @@
  *    on `stream` (a cudaStream_t passed as void*, NULL = the legacy default
  *    stream) and returns without synchronizing.  The caller must keep every
  *    buffer alive until the stream has passed the enqueued work.
- *  - Tensors are dense and row-major; batched tensors are batch-major with
- *    no padding ([batch][rows][cols]).  bf16 values are raw 16-bit patterns.
+ *  - Tensors are row-major; batched tensors are batch-major with no padding
+ *    ([batch][rows][cols]), except where an entry point takes explicit row
+ *    and batch strides (the *_strided calls).  bf16 values are raw 16-bit
+ *    patterns.
+ *  - Scratch memory is a caller-owned workspace, sized by the matching
+ *    *_workspace_bytes call.
  *  - Every pointer must be 16-byte aligned.
  *  - Scales are DEQUANTIZATION MULTIPLIERS ("scale inverse"): an element's
  *    value is approximately decode(code) * scale.
  *  - Return values are synchronous status codes (fpq_status).  On any error
  *    nothing is enqueued.  FPQ_ERR_CUDA carries the CUDA error text in
  *    fpq_last_error_detail() (per thread).  Faults detected inside a kernel
- *    (a bounded wait that ran out, a malformed group offset list) are written
- *    to a device-side error word read by fpq_get_device_error().
+ *    (a bounded wait that ran out, a malformed group offset list, an expert
+ *    id out of range) are written to a device-side error word read by
+ *    fpq_get_device_error().
  *  - There is no CPU fallback: a missing or non-sm_100 device gives
  *    FPQ_ERR_UNSUPPORTED.
  *
@@ -39,11 +44,19 @@
  *        dequantization and FP8 matmul kernels).
  *  [B5]  "DeepSeek-V3 Blog 5: Low-Precision Training -- The FP8 Revolution":
  *        "The Solution: Block-Wise Quantization", "Hardware Optimization"
- *        (FP8 products promoted to higher precision before accumulation).
+ *        (FP8 products promoted to higher precision before accumulation),
+ *        "Reducing Communication Overhead in MoE with FP8" (activations sent
+ *        to the experts' GPUs in FP8: the MoE dispatch calls).
  *  [QAT] "DeepSeek R1 and V3 get quantization-aware fine-tuning on
  *        Fireworks": "Synopsis"/"Interpretation" (LoRA merged into the base
  *        weight, merged bf16 weight converted to block-wise FP8, forward
- *        pass fake-quantizes merged weights and activations).
+ *        pass fake-quantizes merged weights and activations; the adapters
+ *        are trained through it: the QAT backward calls).
+ *
+ * Families: block quantize / dequantize (dense and strided); the LoRA merge
+ * with weight fake-quant; block-scaled GEMMs (fp32 scales, MXFP8, NVFP4,
+ * grouped MXFP8); the bf16 GEMMs of the QAT backward; the MoE FP8 dispatch;
+ * status and error queries.
  */
 #ifndef FPQ_H
 #define FPQ_H
