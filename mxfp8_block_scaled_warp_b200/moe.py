@@ -85,8 +85,9 @@ def dispatch(x: torch.Tensor, topk_ids: torch.Tensor, num_experts: int, group=No
         codes, scales = torch.empty((rows, hidden), **u8), torch.empty((rows, hidden // 32), **u8)
         _dispatch_into(x, topk_ids, num_experts, ws, dst_row0, [(codes, scales)], stream)
         return Dispatched(codes, scales, offsets, counts_all)
-    counts_all = torch.empty((world, num_experts), dtype=torch.int32, device=dev)
-    dist.all_gather_into_tensor(counts_all, counts, group=group)
+    counts_flat = torch.empty((world * num_experts,), dtype=torch.int32, device=dev)
+    dist.all_gather_into_tensor(counts_flat, counts, group=group)     # flat output: every backend takes it
+    counts_all = counts_flat.view(world, num_experts)
     fpq_moe_dispatch_layout(counts_all, world, num_experts, rank, MOE_PACK, dst_row0, offsets, stream)
     rows = tokens * topk_ids.shape[1]
     send_q, send_s = torch.empty((rows, hidden), **u8), torch.empty((rows, hidden // 32), **u8)

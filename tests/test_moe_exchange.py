@@ -98,3 +98,66 @@ def test_segment_plan_single_rank():
     assert sends == [(0, 0, 0, 2), (0, 2, 2, 3)]
     assert recvs == [(0, 0, 0, 2), (0, 2, 2, 3)]
     assert rows == 5
+
+
+def _dispatch_worker(rank, world, port, q):
+    """moe.dispatch on gloo ranks with its three device steps (route, layout,
+    the quantize + pack kernel) stood in for by the oracle's definitions; the
+    counts all-gather, the segment plan and the transfers run as written."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    import oracle
+    import workloads
+    from mxfp8_block_scaled_warp_b200 import moe
+
+    def fake_route(topk_ids, num_experts, stream=None):
+        counts, _ = oracle.moe_route_plan(topk_ids.numpy(), num_experts)
+        return torch.from_numpy(counts.astype(np.int32)), None
+
+    def fake_layout(counts_all, world_, num_experts, rank_, mode, dst_row0, offsets, stream=None):
+        c = counts_all.numpy().astype(np.int64)
+        L = num_experts // world_
+        assert mode == moe.MOE_PACK
+        dst_row0.copy_(torch.from_numpy(np.concatenate([[0], np.cumsum(c[rank_])[:-1]])))
+        tot = c.sum(axis=0)[rank_ * L:(rank_ + 1) * L]
+        offsets.copy_(torch.from_numpy(np.concatenate([[0], np.cumsum(tot)]).astype(np.int32)))
+
+    def fake_pack(x, topk_ids, num_experts, ws, dst_row0, buffers, stream=None):
+        q, s, _ = oracle.moe_dispatch([workloads.as_u16(x)], [topk_ids.numpy()], num_experts)[0]
+        buffers[0][0].copy_(torch.from_numpy(q))
+        buffers[0][1].copy_(torch.from_numpy(s))
+
+    moe.route, moe.fpq_moe_dispatch_layout, moe._dispatch_into = fake_route, fake_layout, fake_pack
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        xs, ids = _inputs(world)
+        d = moe.dispatch(workloads.from_u16(xs[rank]), torch.from_numpy(ids[rank].astype(np.int32)), EXPERTS,
+                         group=dist.group.WORLD)
+        q.put((rank, d.codes.numpy(), d.scales.numpy(), d.group_offsets.numpy(), d.counts_all.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_dispatch_orchestration_two_ranks():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_dispatch_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict((r, rest) for r, *rest in (q.get(timeout=180) for _ in range(world)))
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    sys.path.insert(0, ROOT)
+    import oracle
+    xs, ids = _inputs(world)
+    want = oracle.moe_dispatch(xs, ids, EXPERTS)
+    counts = np.stack([oracle.moe_route_plan(i, EXPERTS)[0] for i in ids])
+    for r in range(world):
+        codes, scales, offs, counts_all = got[r]
+        assert np.array_equal(codes, want[r][0]) and np.array_equal(scales, want[r][1])
+        assert np.array_equal(offs, want[r][2])
+        assert np.array_equal(counts_all, counts)
