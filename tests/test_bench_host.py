@@ -1,0 +1,41 @@
+"""Host logic of bench.py without a GPU: every workload's oracle CPU
+baseline (the reference arm) returns a well-formed, positive figure in the
+workload's unit; the launch note names the kernels a step forks; traffic
+from a profile summary is used only while the kernel's source is unchanged."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+@pytest.mark.parametrize("workload", sorted(bench.STEPS))
+def test_cpu_baseline_every_workload(workload):
+    r = bench.cpu_baseline(workload, budget_s=0.3)
+    assert r is not None, f"no oracle timing for {workload}"
+    step = bench.STEPS[workload]
+    assert r["unit"] == step.unit and r["value"] > 0 and r["work"] > 0
+    assert r["kind"] == "oracle" and r["cores"] == 1 and r["sample"]
+
+
+def test_launch_note_names_forked_kernels():
+    note = bench.launch_note(object.__new__(bench.DsFp8Gemm))
+    assert "quant_fp8_128x128 on a second stream" in note
+    assert "second stream" not in bench.launch_note(object.__new__(bench.Nvfp4Gemm))
+
+
+def test_traffic_only_for_unchanged_source(tmp_path, monkeypatch):
+    h = bench._source_hash("moe_dispatch_mxfp8")
+    assert h
+    (tmp_path / "profiles").mkdir()
+    f = tmp_path / "profiles" / "moe_dispatch_mxfp8__moe_dispatch.md"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "_source_hash", lambda kernel: h)   # the real source's hash
+    f.write_text(f"source_sha256_16: {h}\ndram_bytes_per_launch: 123456\n")
+    assert bench._traffic("moe_dispatch_mxfp8", "moe_dispatch") == 123456.0
+    f.write_text("source_sha256_16: 0000000000000000\ndram_bytes_per_launch: 123456\n")
+    assert bench._traffic("moe_dispatch_mxfp8", "moe_dispatch") is None
