@@ -21,6 +21,11 @@
 // 32 (w & 3) .. + 31 and columns 128 (w >> 2) .. + 127 of the accumulator,
 // times alpha, to bf16, staged in 128-byte-swizzled boxes and written by
 // TMA stores (which clip rows past M and columns past N).
+// Split-K mode, for products with few output tiles and a long contraction
+// (the LoRA gradients): the grid is tiles x slices, each CTA runs its slice
+// of the K tiles and stores its fp32 sums (without alpha) to a partial
+// buffer; reduce_partials_kernel then adds the slices in slice order, times
+// alpha, to bf16, so results do not depend on scheduling.
 // Every wait on an mbarrier is bounded by wall time (4 s); on expiry the
 // kernel records FPQ_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
 #include <cuda.h>
