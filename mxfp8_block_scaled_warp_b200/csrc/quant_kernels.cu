@@ -9,7 +9,10 @@
 // lane as eight 32-bit words.  A block of the format is 2 units (MXFP8 1x32),
 // 8 units (1x128) or 1 unit (NVFP4 1x16); because every row length is a
 // multiple of the block, blocks never straddle rows and a flat unit index
-// addresses both the data and the row-major scale arrays.
+// addresses both the data and the row-major scale arrays.  Each streaming
+// kernel also has a strided instance (template flag S): data and codes then
+// live at row and batch strides, the flat unit index is mapped to (matrix,
+// row, column unit) once per unit, and the scales stay dense.
 #include <cuda_fp16.h>
 
 #include <cuda.h>
