@@ -106,6 +106,7 @@ class ClockSampler:
 class Step:
     """A workload bound to device buffers; run() enqueues one step."""
     name = ""
+    CONFIG: dict = {}          # the workload's description and shape (both bench arms print it)
     flops = 0.0
     quant_bytes = 0.0
     launches = 0
@@ -151,6 +152,10 @@ class Step:
 
 class DsFp8Gemm(Step):
     name = "ds_fp8_gemm"
+    CONFIG = {"workload": "ds_fp8_gemm: A bf16 4096x7168 N(0,1) -> E4M3 with fp32 scale per 1x128 tile; "
+                          "B bf16 2048x7168 N(0,0.02) -> E4M3 with fp32 scale per 128x128 block; "
+                          "C = A B^T fp32 accumulate, bf16 out",
+              "m": 4096, "n": 2048, "k": 7168, "l2": "flushed before every step (256 MiB write)"}
     dominant = "gemm_fp8_f32scale"
     side = ("quant_fp8_128x128",)      # B's quantizer runs beside A's
     join_before = "gemm_fp8_f32scale"
@@ -173,10 +178,7 @@ class DsFp8Gemm(Step):
         self.qb_bytes = n * k * (2 + 1) + ((n + 127) // 128) * (k // 128) * 4
         self.quant_bytes = self.qa_bytes + self.qb_bytes
         self.launches = 3
-        self.config = {"workload": "ds_fp8_gemm: A bf16 4096x7168 N(0,1) -> E4M3 with fp32 scale per 1x128 tile; "
-                                   "B bf16 2048x7168 N(0,0.02) -> E4M3 with fp32 scale per 128x128 block; "
-                                   "C = A B^T fp32 accumulate, bf16 out",
-                       "m": m, "n": n, "k": k, "l2": "flushed before every step (256 MiB write)"}
+        self.config = dict(self.CONFIG)
 
     def kernels(self):
         f = self.f
@@ -210,6 +212,9 @@ class MoeGrouped(Step):
     64 x 2048 x 7168."""
     name = "moe_grouped"
     dominant = "gemm_grouped_mxfp8"
+    CONFIG = {"workload": "moe_grouped: X 16384x7168 N(0,1), top-8 of 64 experts (Zipf 1.1 Gumbel-top-8); "
+                          "FP8 dispatch (each token quantized once to MXFP8, 131072 rows grouped by "
+                          "expert); grouped GEMM with MXFP8 expert weights 64x2048x7168", "l2": "flushed before every step (256 MiB write)"}
 
     def __init__(self, fpq, dev, tokens=16384, experts=64, topk=8):
         self.f = fpq
@@ -243,11 +248,7 @@ class MoeGrouped(Step):
         self.quant_bytes = self.route_bytes + self.dispatch_bytes
         self.launches = 5
         counts = np.bincount(self.ids_host.numpy().reshape(-1), minlength=experts)
-        self.config = {"workload": "moe_grouped: X 16384x7168 N(0,1), top-8 of 64 experts (Zipf 1.1 Gumbel-top-8); "
-                                   "FP8 dispatch (each token quantized once to MXFP8, 131072 rows grouped by "
-                                   "expert); grouped GEMM with MXFP8 expert weights 64x2048x7168",
-                       "expert_rows_max": int(counts.max()), "expert_rows_min": int(counts.min()),
-                       "l2": "flushed before every step (256 MiB write)"}
+        self.config = dict(self.CONFIG, expert_rows_max=int(counts.max()), expert_rows_min=int(counts.min()))
 
     def kernels(self):
         f = self.f
@@ -282,6 +283,8 @@ class MoeGrouped(Step):
 class QatForward(Step):
     name = "qat_forward"
     dominant = "gemm_fp8_f32scale"
+    CONFIG = {"workload": "qat_forward: merge W 2048x7168 + (32/16) B A (r=16) -> 128x128 FP8 fake-quant; "
+                          "X 8192x7168 -> 1x128 FP8; C = X W_eff^T", "l2": "flushed before every step (256 MiB write)"}
     side = ("lora_merge_fq",)          # the weight merge runs beside X's quantizer
     join_before = "gemm_fp8_f32scale"
 
@@ -302,8 +305,7 @@ class QatForward(Step):
         self.xq_bytes = self.m * self.k * 3 + self.m * (self.k // 128) * 4
         self.quant_bytes = self.merge_bytes + self.xq_bytes
         self.launches = 3
-        self.config = {"workload": "qat_forward: merge W 2048x7168 + (32/16) B A (r=16) -> 128x128 FP8 fake-quant; "
-                                   "X 8192x7168 -> 1x128 FP8; C = X W_eff^T", "l2": "flushed before every step"}
+        self.config = dict(self.CONFIG)
 
     def kernels(self):
         f = self.f
@@ -339,6 +341,9 @@ class MoePrequant(Step):
     one batched call, to MXFP8 (1x32, E8M0) and to NVFP4 (1x16 E4M3 + a
     per-matrix fp32 scale).  The step's work is the algorithmic bytes."""
     name = "moe_prequant"
+    CONFIG = {"workload": "moe_prequant: 64 experts x {gate, up 2048x7168; down 7168x2048} bf16 N(0,0.02) "
+                          "-> MXFP8 (1x32 E8M0) and NVFP4 (1x16 E4M3 + fp32 per matrix); one batched call "
+                          "per projection and format", "l2": "flushed before every step (256 MiB write)"}
     side = ("quant_nvfp4",)            # the two formats of a matrix are independent
     dominant = "quant_nvfp4"
     unit = "GB/s"
@@ -368,10 +373,9 @@ class MoePrequant(Step):
         self.nv_bytes = elems * (2 + 0.5 + 1 / 16) + 4 * 3 * experts
         self.quant_bytes = self.mx_bytes + self.nv_bytes
         self.launches = 6
-        self.config = {"workload": f"moe_prequant: {experts} experts x {{gate, up 2048x7168; down 7168x2048}} bf16 N(0,0.02) "
-                                   "-> MXFP8 (1x32 E8M0) and NVFP4 (1x16 E4M3 + fp32 per matrix); one batched call "
-                                   "per projection and format",
-                       "elements": elems, "l2": "flushed before every step (256 MiB write)"}
+        self.config = dict(self.CONFIG, elements=elems)
+        if experts != 64:
+            self.config["workload"] = self.CONFIG["workload"].replace("64 experts", f"{experts} experts")
 
     @property
     def work(self) -> float:
@@ -424,6 +428,10 @@ class QatBackward(Step):
     one so that each product is timed (dA and dB with their reductions)."""
     name = "qat_backward"
     dominant = "gemm_bf16_dx"
+    CONFIG = {"workload": "qat_backward: dy 8192x2048 N(0,1); x_fq = 1x128 fake-quant of x 8192x7168 "
+                          "N(0,1); w_fq = 128x128 fake-quant of W + 2 B A (W 2048x7168 N(0,0.02), r = 16); "
+                          "dx = dy w_fq, dW = dy^T x_fq, dA = 2 B^T dW, dB = 2 dW A^T, bf16",
+              "m": 8192, "n": 2048, "k": 7168, "r": 16, "l2": "flushed before every step (256 MiB write)"}
     dtype = "bf16xbf16->f32 (bf16 out)"
     tensor_ratio = 1.0
 
@@ -456,10 +464,7 @@ class QatBackward(Step):
         self.flops = 2.0 * (2 * m * n * k + 2 * r * n * k)
         self.quant_bytes = 0.0          # no quantize kernel in this step
         self.launches = 6                # dA and dB: split-K GEMM + slice reduction each
-        self.config = {"workload": "qat_backward: dy 8192x2048 N(0,1); x_fq = 1x128 fake-quant of x 8192x7168 "
-                                   "N(0,1); w_fq = 128x128 fake-quant of W + 2 B A (W 2048x7168 N(0,0.02), r = 16); "
-                                   "dx = dy w_fq, dW = dy^T x_fq, dA = 2 B^T dW, dB = 2 dW A^T, bf16",
-                       "m": m, "n": n, "k": k, "r": r, "l2": "flushed before every step (256 MiB write)"}
+        self.config = dict(self.CONFIG)
 
     def kernels(self):
         f, m, n, k, r, aor = self.f, self.m, self.n, self.k, self.r, self.aor
@@ -500,6 +505,10 @@ class Nvfp4Gemm(Step):
     on the tensor cores (kind::mxf4nvf4, CTA pairs)."""
     name = "nvfp4_gemm"
     dominant = "gemm_nvfp4"
+    CONFIG = {"workload": "nvfp4_gemm: A bf16 4096x7168 N(0,1) and B bf16 2048x7168 N(0,0.02) -> packed "
+                          "E2M1 with E4M3 scale per 16 and fp32 tensor scale; C = gA gB A B^T fp32 "
+                          "accumulate, bf16 out",
+              "m": 4096, "n": 2048, "k": 7168, "l2": "flushed before every step (256 MiB write)"}
     dtype = "e2m1xe2m1->f32 (bf16 in/out)"
     tensor_ratio = 4.0         # dense fp4 / bf16, nominal 9 / 2.25
 
@@ -524,10 +533,7 @@ class Nvfp4Gemm(Step):
         self.qb_bytes = n * k * (2 + 0.5 + 1 / 16) + 4
         self.quant_bytes = self.qa_bytes + self.qb_bytes
         self.launches = 3      # two quantize kernels (each after a workspace memset) and the GEMM
-        self.config = {"workload": "nvfp4_gemm: A bf16 4096x7168 N(0,1) and B bf16 2048x7168 N(0,0.02) -> packed "
-                                   "E2M1 with E4M3 scale per 16 and fp32 tensor scale; C = gA gB A B^T fp32 "
-                                   "accumulate, bf16 out",
-                       "m": m, "n": n, "k": k, "l2": "flushed before every step (256 MiB write)"}
+        self.config = dict(self.CONFIG)
 
     def kernels(self):
         f = self.f
@@ -561,6 +567,9 @@ class MoeDispatch(Step):
     input).  On one GPU every destination is local."""
     name = "moe_dispatch"
     dominant = "moe_dispatch_mxfp8"
+    CONFIG = {"workload": "moe_dispatch: X 16384x7168 bf16 N(0,1), top-8 of 64 experts (Gumbel-top-8 on "
+                          "log((e+1)^-1.1)) -> MXFP8 rows grouped by expert, one GPU (all destinations "
+                          "local)", "tokens": 16384, "hidden": 7168, "experts": 64, "topk": 8, "l2": "flushed before every step (256 MiB write)"}
     unit = "GB/s"
     dtype = "bf16 -> e4m3 + e8m0 (scatter)"
 
@@ -588,10 +597,7 @@ class MoeDispatch(Step):
         self.bytes = self.dispatch_bytes + self.route_bytes
         self.quant_bytes = self.bytes
         self.launches = 4
-        self.config = {"workload": "moe_dispatch: X 16384x7168 bf16 N(0,1), top-8 of 64 experts (Gumbel-top-8 on "
-                                   "log((e+1)^-1.1)) -> MXFP8 rows grouped by expert, one GPU (all destinations "
-                                   "local)", "tokens": tokens, "hidden": hidden, "experts": experts, "topk": topk,
-                       "l2": "flushed before every step (256 MiB write)"}
+        self.config = dict(self.CONFIG)
 
     @property
     def work(self):
@@ -895,7 +901,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": work / (v * scale) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload},
+            "data": "synthetic", "config": dict(STEPS[args.workload].CONFIG),
             "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle", "sample": r["sample"]},
             "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
