@@ -1,22 +1,28 @@
 """Benchmark of the block-scaled FP8 hot path on B200.
 
-One step = one pass of the fine-grained FP8 GEMM workload: quantize the
-activations A [4096, 7168] (bf16 -> E4M3, fp32 scale per 1x128 tile),
-quantize the weights B [2048, 7168] (fp32 scale per 128x128 block), then
-C = A B^T with fp32 accumulation and bf16 output (120.3 GFLOP).
+One step (default workload `moe_grouped`, the largest single-GPU case) =
+the expert up-projection of an MoE layer: 16384 bf16 tokens x 7168 routed
+top-8 over 64 experts; the FP8 dispatch (route histograms and scan, layout,
+one fused kernel that quantizes each token row once to MXFP8 and writes it
+to the rows of its 8 experts) builds the expert-grouped operand [131072,
+7168], and the grouped MXFP8 GEMM multiplies it with the prequantized expert
+weights 64 x [2048, 7168], fp32 accumulation, bf16 out (3.848 TFLOP).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload ds_fp8_gemm|qat_forward|qat_backward|moe_grouped|moe_dispatch|
-                                moe_prequant|nvfp4_gemm]
+                    [--workload moe_grouped|ds_fp8_gemm|qat_forward|qat_backward|moe_dispatch|
+                                moe_prequant|nvfp4_gemm|dequant]
 
 Prints one JSON line (rank 0).  `value` is whole-step throughput in TFLOP/s
 (GEMM flops of the step / step time, quantization included; GB/s for the
-quantize-only and dispatch-only workloads), with the
-inputs resident in HBM and L2 flushed (256 MiB write) before every step; the
+quantize-, dequantize- and dispatch-only workloads), with the inputs
+resident in HBM and L2 flushed (256 MiB write) before every step; the
 per-kernel times, the quantize GB/s and the roofline of the dominant kernel
 come from CUDA events on the launching stream.  With N > 1 (torchrun) every
 rank runs an independent replica (the path has no exchange step): the time
-is the max over ranks and `value` counts all ranks' work.
+is the max over ranks and `value` counts all ranks' work.  `cpu_baseline`
+is the oracle timed on a bounded sample, on one thread and on every host
+core; `--impl reference` times the oracle alone (every host core), one
+sample of the workload per step.
 """
 from __future__ import annotations
 
@@ -629,9 +635,110 @@ class MoeDispatch(Step):
         return self.x_host.numel() * 2 + self.ids_host.numel() * 4, self.offs.numel() * 4
 
 
+class Dequant(Step):
+    """bf16 reconstruction of block-quantized tensors ("FP8 в DeepSeek V3",
+    Практический смысл для инференс-инфраструктуры: FP8 weights converted
+    back to BF16 where the hardware has no FP8 path): the 64-expert stacks
+    of the prequant workload (gate, up [2048, 7168], down [7168, 2048]) from
+    MXFP8 and from NVFP4, and the fine-grained operands (A 4096x7168 with
+    1x128 fp32 scales, B 2048x7168 with 128x128 fp32 scales).  The codes
+    and scales are made by the library once, outside the step; the step's
+    work is the algorithmic bytes (codes and scales read, bf16 written)."""
+    name = "dequant"
+    CONFIG = {"workload": "dequant: 64 experts x {gate, up 2048x7168; down 7168x2048} from MXFP8 (1x32 E8M0) "
+                          "and from NVFP4 (1x16 E4M3 + fp32 per matrix), A 4096x7168 from 1x128 fp32 scales, "
+                          "B 2048x7168 from 128x128 fp32 scales -> bf16",
+              "l2": "flushed before every step (256 MiB write)"}
+    dominant = "dequant_mxfp8"
+    unit = "GB/s"
+    dtype = "e4m3 / e2m1 codes -> bf16 (fp32 scale arithmetic)"
+
+    def __init__(self, fpq, dev, experts=64):
+        self.f = fpq
+        self.e = experts
+        shapes = {"gate": (2048, 7168), "up": (2048, 7168), "down": (7168, 2048)}
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.mats = {}
+        for i, (nm, (r, c)) in enumerate(shapes.items()):
+            g = torch.Generator(device=dev)
+            g.manual_seed(4000 + i)
+            x = torch.empty((experts, r, c), dtype=torch.bfloat16, device=dev)
+            for e in range(experts):
+                x[e] = (torch.randn(r, c, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+            mq, ms = fpq.quantize(x, fpq.MXFP8)
+            nq, ns, ng = fpq.quantize(x, fpq.NVFP4)
+            self.mats[nm] = (r, c, mq, ms, nq, ns, ng, x)     # x is overwritten: it is the bf16 output
+        wl = workloads.ds_fp8_gemm()
+        a, b = wl["a"].to(dev), wl["b"].to(dev)
+        self.aq, self.as_ = fpq.quantize(a, fpq.FP8_1x128)
+        self.bq, self.bs = fpq.quantize(b, fpq.FP8_128x128)
+        self.a_out, self.b_out = a, b
+        elems = sum(experts * r * c for r, c, *_ in self.mats.values())
+        self.mx_bytes = elems * (1 + 1 / 32 + 2)
+        self.nv_bytes = elems * (0.5 + 1 / 16 + 2) + 4 * 3 * experts
+        self.a_bytes = a.numel() * 3 + self.as_.numel() * 4
+        self.b_bytes = b.numel() * 3 + self.bs.numel() * 4
+        self.quant_bytes = self.mx_bytes + self.nv_bytes + self.a_bytes + self.b_bytes
+        self.launches = 8
+        self.config = dict(self.CONFIG)
+
+    @property
+    def work(self) -> float:
+        return self.quant_bytes
+
+    def kernels(self):
+        f = self.f
+
+        def mx():
+            for r, c, mq, ms, _, _, _, out in self.mats.values():
+                f.fpq_dequantize(f.MXFP8, mq, ms, None, self.e, r, c, out)
+
+        def nv():
+            for r, c, _, _, nq, ns, ng, out in self.mats.values():
+                f.fpq_dequantize(f.NVFP4, nq, ns, ng, self.e, r, c, out)
+
+        return [("dequant_mxfp8", mx), ("dequant_nvfp4", nv),
+                ("dequant_fp8_1x128", lambda: f.fpq_dequantize(f.FP8_1x128, self.aq, self.as_, None, 1, 4096, 7168,
+                                                               self.a_out)),
+                ("dequant_fp8_128x128", lambda: f.fpq_dequantize(f.FP8_128x128, self.bq, self.bs, None, 1, 2048,
+                                                                 7168, self.b_out))]
+
+    def kernel_work(self):
+        return {"dequant_mxfp8": ("GB/s", self.mx_bytes), "dequant_nvfp4": ("GB/s", self.nv_bytes),
+                "dequant_fp8_1x128": ("GB/s", self.a_bytes), "dequant_fp8_128x128": ("GB/s", self.b_bytes)}
+
+    def e2e_step(self, stream, side_stream):
+        """Codes and scales from pinned host memory in, every bf16 result
+        back to pinned host memory, copies inside the timed region."""
+        if not hasattr(self, "host"):
+            self.host = []
+            for r, c, mq, ms, nq, ns, ng, out in self.mats.values():
+                self.host.append(([(t, t.cpu().pin_memory()) for t in (mq, ms, nq, ns, ng)],
+                                  (out, torch.empty(out.shape, dtype=out.dtype).pin_memory())))
+            self.host_ab = [(t, t.cpu().pin_memory()) for t in (self.aq, self.as_, self.bq, self.bs)]
+            self.host_ab_out = [(t, torch.empty(t.shape, dtype=t.dtype).pin_memory()) for t in (self.a_out, self.b_out)]
+        hb = db = 0
+        for ins, _ in self.host:
+            for d, h in ins:
+                d.copy_(h, non_blocking=True)
+                hb += h.numel() * h.element_size()
+        for d, h in self.host_ab:
+            d.copy_(h, non_blocking=True)
+            hb += h.numel() * h.element_size()
+        for _, fn in self.kernels():
+            fn()
+        for _, (d, h) in self.host:
+            h.copy_(d, non_blocking=True)
+            db += d.numel() * d.element_size()
+        for d, h in self.host_ab_out:
+            h.copy_(d, non_blocking=True)
+            db += d.numel() * d.element_size()
+        return hb, db
+
+
 STEPS = {"ds_fp8_gemm": DsFp8Gemm, "moe_grouped": MoeGrouped, "qat_forward": QatForward,
          "moe_prequant": MoePrequant, "nvfp4_gemm": Nvfp4Gemm, "qat_backward": QatBackward,
-         "moe_dispatch": MoeDispatch}
+         "moe_dispatch": MoeDispatch, "dequant": Dequant}
 
 
 # ------------------------------------------------------------------ traffic from committed ncu summaries
@@ -664,245 +771,246 @@ def _traffic(kernel: str, workload: str):
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
+#
+# A workload on the oracle is a list of phases; each phase is `total` units
+# of one kind (quantized rows, 128-row strips, dispatched tokens, fp64 GEMM
+# entries) with `work` of the line's unit per unit (flops, or bytes for the
+# GB/s workloads).  A timed sample runs the same fraction f of every phase's
+# units; each phase's units are split into contiguous ranges over the host
+# threads (the oracle's C calls release the GIL, so the threads run in
+# parallel).  The whole-step time is extrapolated per phase (its measured
+# time x total / units run), and `value` = the step's work / that time.
 
-def cpu_baseline(workload: str, budget_s: float = 12.0):
-    """Time the oracle (as it stands, single thread) on a bounded sample of
-    the workload and extrapolate to the whole step in TFLOP/s."""
+class OraclePhase:
+    def __init__(self, label: str, total: int, work: float, fn):
+        self.label, self.total, self.work, self.fn = label, int(total), float(work), fn
+
+
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_phases(phases, fraction: float, threads: int):
+    """Run `fraction` of every phase's units (at least one unit each) on
+    `threads` threads; returns [(units, seconds)] per phase."""
+    from concurrent.futures import ThreadPoolExecutor
+    out = []
+    with ThreadPoolExecutor(threads) as ex:
+        for ph in phases:
+            n = int(max(1, min(ph.total, round(fraction * ph.total))))
+            cuts = np.linspace(0, n, min(threads, n) + 1).astype(np.int64)
+            t0 = time.perf_counter()
+            list(ex.map(lambda i: ph.fn(int(cuts[i]), int(cuts[i + 1])), range(len(cuts) - 1)))
+            out.append((n, time.perf_counter() - t0))
+    return out
+
+
+def extrapolate(phases, runs):
+    """(seconds of the whole step, work of the whole step) from a sample."""
+    step_s = sum(dt * ph.total / n for ph, (n, dt) in zip(phases, runs))
+    return step_s, sum(ph.total * ph.work for ph in phases)
+
+
+def _entries(fn, rows: int, cols: int):
+    """fn(rr, cc) over entry indices [lo, hi) spread across a rows x cols
+    sample of quantized operands (each entry costs the same)."""
+    def run(lo, hi):
+        i = np.arange(lo, hi, dtype=np.int64)
+        return fn(i % rows, (i * 7) % cols)
+    return run
+
+
+def oracle_phases(workload: str, oracle):
+    """(phases, unit, description) of a workload on the oracle, or None."""
+    k = 7168
+    if workload in ("ds_fp8_gemm", "nvfp4_gemm"):
+        m, n = 4096, 2048
+        wl = workloads.ds_fp8_gemm(m, n, k)
+        a, b = workloads.as_u16(wl["a"]), workloads.as_u16(wl["b"])
+        if workload == "ds_fp8_gemm":
+            qa, sa = oracle.quant_fp8_1x128(a[:64])
+            qb, sb = oracle.quant_fp8_128x128(b[:256])
+            return [OraclePhase("1x128 quantize of A (rows)", m, 0.0, lambda lo, hi: oracle.quant_fp8_1x128(a[lo:hi])),
+                    OraclePhase("128x128 quantize of B (128-row strips)", n // 128, 0.0,
+                                lambda lo, hi: oracle.quant_fp8_128x128(b[128 * lo:128 * hi])),
+                    OraclePhase("fp64 GEMM entries (K=7168)", m * n, 2.0 * k,
+                                _entries(lambda r, c: oracle.gemm_entries(0, qa, sa, 1, qb, sb, r, c), 64, 256))], \
+                "TFLOP/s", "4096x2048x7168 fine-grained FP8 step"
+        qa, sa, ga = oracle.quant_nvfp4(a[:64])
+        qb, sb, gb = oracle.quant_nvfp4(b[:256])
+        return [OraclePhase("NVFP4 quantize of A (rows)", m, 0.0, lambda lo, hi: oracle.quant_nvfp4(a[lo:hi])),
+                OraclePhase("NVFP4 quantize of B (rows)", n, 0.0, lambda lo, hi: oracle.quant_nvfp4(b[lo:hi])),
+                OraclePhase("fp64 GEMM entries (K=7168)", m * n, 2.0 * k,
+                            _entries(lambda r, c: oracle.gemm_entries(3, qa, sa, 3, qb, sb, r, c, ag=ga, bg=gb),
+                                     64, 256))], \
+            "TFLOP/s", "4096x2048x7168 NVFP4 step"
+    if workload == "qat_forward":
+        m, n = 8192, 2048
+        wl = workloads.qat_forward()
+        w, la, lb, x = (workloads.as_u16(wl[t]) for t in ("w", "lora_a", "lora_b", "x"))
+        aor = wl["alpha_over_r"]
+        qw, sw, _ = oracle.lora_merge_fakequant(w[:128], la, lb[:128], aor)
+        qx, sx = oracle.quant_fp8_1x128(x[:64])
+        return [OraclePhase("LoRA merge + 128x128 fake-quant of W (128-row strips)", n // 128, 0.0,
+                            lambda lo, hi: oracle.lora_merge_fakequant(w[128 * lo:128 * hi], la,
+                                                                       lb[128 * lo:128 * hi], aor)),
+                OraclePhase("1x128 quantize of X (rows)", m, 0.0, lambda lo, hi: oracle.quant_fp8_1x128(x[lo:hi])),
+                OraclePhase("fp64 GEMM entries (K=7168)", m * n, 2.0 * k,
+                            _entries(lambda r, c: oracle.gemm_entries(0, qx, sx, 1, qw, sw, r, c), 64, 128))], \
+            "TFLOP/s", "8192x2048x7168 QAT forward step"
+    if workload == "qat_backward":
+        m, n, r = 8192, 2048, 16
+        phases = []
+        for kk, total, what in ((2048, m * k + r * k, "dX and dA"), (8192, n * k, "dW_eff"), (7168, n * r, "dB")):
+            p = workloads.as_u16(workloads.normal_bf16((64, kk), 1.0, seed=6000 + kk))
+            q = workloads.as_u16(workloads.normal_bf16((64, kk), 0.02, seed=6001 + kk))
+            phases.append(OraclePhase(f"fp64 bf16-product entries of {what} (K={kk})", total, 2.0 * kk,
+                                      _entries(lambda rr, cc, p=p, q=q: oracle.gemm_bf16_entries(p, q, rr, cc),
+                                               64, 64)))
+        return phases, "TFLOP/s", "QAT backward step (dX, dW_eff, dA, dB)"
+    if workload in ("moe_grouped", "moe_dispatch"):
+        tokens, experts, topk, n = 16384, 64, 8, 2048
+        wl = workloads.moe_dispatch(tokens=tokens)
+        x, ids = workloads.as_u16(wl["x"][0]), wl["topk_ids"][0].numpy()
+        per_tok = k * 2 + topk * 8 + topk * (k + k // 32)
+        dispatch = OraclePhase("dispatch (route, MXFP8 quantize, placement) of tokens", tokens,
+                               per_tok if workload == "moe_dispatch" else 0.0,
+                               lambda lo, hi: oracle.moe_dispatch([x[lo:hi]], [ids[lo:hi]], experts))
+        if workload == "moe_dispatch":
+            return [dispatch], "GB/s", "16384-token top-8 FP8 dispatch"
+        codes, scales, _ = oracle.moe_dispatch([x[:32]], [ids[:32]], experts)[0]
+        rows = codes.shape[0]
+        wq, ws = oracle.quant_mxfp8(np.stack([workloads.as_u16(workloads.normal_bf16((64, k), 0.02, seed=5100 + e))
+                                              for e in range(2)]))
+        off2 = np.array([0, rows // 2, rows], np.int64)
+        return [dispatch,
+                OraclePhase("fp64 grouped MXFP8 GEMM entries (K=7168)", tokens * topk * n, 2.0 * k,
+                            _entries(lambda rr, cc: oracle.grouped_gemm_entries(2, codes, scales, wq, ws, off2, rr, cc),
+                                     rows, 64))], \
+            "TFLOP/s", "16384-token step (dispatch + grouped GEMM, 131072x2048x7168)"
+    if workload in ("moe_prequant", "dequant"):
+        x = workloads.as_u16(workloads.normal_bf16((2048, k), 0.02, 4000))
+        rows_total = 64 * 3 * 2048            # gate, up [2048, 7168] and down [7168, 2048]: 7168-element rows
+
+        def rows_of(lo, hi):
+            return x[np.arange(lo, hi) % 2048]
+
+        if workload == "moe_prequant":
+            return [OraclePhase("MXFP8 quantize (7168-element rows)", rows_total, k * (3 + 1 / 32),
+                                lambda lo, hi: oracle.quant_mxfp8(rows_of(lo, hi))),
+                    OraclePhase("NVFP4 quantize (7168-element rows)", rows_total, k * (2.5 + 1 / 16),
+                                lambda lo, hi: oracle.quant_nvfp4(rows_of(lo, hi)))], \
+                "GB/s", "64-expert prequant step"
+        mq, ms = oracle.quant_mxfp8(x[:256])
+        nq, ns, ng = oracle.quant_nvfp4(x[:256])
+        a = workloads.as_u16(workloads.ds_fp8_gemm()["a"][:256])
+        aq, as_ = oracle.quant_fp8_1x128(a)
+        bq, bs = oracle.quant_fp8_128x128(x[:256])
+        return [OraclePhase("MXFP8 dequantize (7168-element rows)", rows_total, k * (1 + 1 / 32 + 2),
+                            lambda lo, hi: oracle.dequant_mxfp8(mq[np.arange(lo, hi) % 256],
+                                                                ms[np.arange(lo, hi) % 256])),
+                OraclePhase("NVFP4 dequantize (7168-element rows)", rows_total, k * (0.5 + 1 / 16 + 2),
+                            lambda lo, hi: oracle.dequant_nvfp4(nq[np.arange(lo, hi) % 256],
+                                                                ns[np.arange(lo, hi) % 256], ng)),
+                OraclePhase("1x128 dequantize of A (rows)", 4096, k * 3 + (k // 128) * 4,
+                            lambda lo, hi: oracle.dequant_fp8_1x128(aq[np.arange(lo, hi) % 256],
+                                                                    as_[np.arange(lo, hi) % 256])),
+                OraclePhase("128x128 dequantize of B (128-row strips)", 16, 128 * k * 3 + (k // 128) * 4,
+                            lambda lo, hi: [oracle.dequant_fp8_128x128(bq[:128], bs[:1]) for _ in range(lo, hi)])], \
+            "GB/s", "dequantize step (64-expert MXFP8 and NVFP4 stacks, 1x128 A, 128x128 B)"
+    return None
+
+
+def cpu_baseline(workload: str, budget_s: float = 8.0, threads: int | None = None):
+    """The oracle as it stands, timed on a bounded sample of the workload:
+    once on one thread and once with the sample's units split over every
+    host core (about `budget_s` seconds each); both extrapolated to the
+    whole step in the workload's unit."""
     import oracle
     oracle.build()
-    if workload == "moe_prequant":
-        return _cpu_baseline_prequant(oracle, budget_s)
-    if workload == "nvfp4_gemm":
-        return _cpu_baseline_nvfp4_gemm(oracle, budget_s)
-    if workload == "moe_dispatch":
-        return _cpu_baseline_moe_dispatch(oracle, budget_s)
-    if workload == "qat_forward":
-        return _cpu_baseline_qat_forward(oracle, budget_s)
-    if workload == "qat_backward":
-        return _cpu_baseline_qat_backward(oracle, budget_s)
-    if workload == "moe_grouped":
-        return _cpu_baseline_moe_grouped(oracle, budget_s)
-    if workload != "ds_fp8_gemm":
+    oracle.lib()
+    spec = oracle_phases(workload, oracle)
+    if spec is None:
         return None
-    m, n, k = 4096, 2048, 7168
-    wl = workloads.ds_fp8_gemm(m, n, k)
-    a, b = workloads.as_u16(wl["a"]), workloads.as_u16(wl["b"])
-    t0 = time.perf_counter()
-    rows_a = 64
-    qa, sa = oracle.quant_fp8_1x128(a[:rows_a])
-    t_qa = (time.perf_counter() - t0) / (rows_a * k)
-    t0 = time.perf_counter()
-    qb, sb = oracle.quant_fp8_128x128(b[:256])
-    t_qb = (time.perf_counter() - t0) / (256 * k)
-    # GEMM entries: calibrate, then fill the remaining budget
-    spent = (t_qa * rows_a + t_qb * 256) * k
-    probe = 64
-    rr = np.arange(probe) % rows_a
-    cc = np.arange(probe) % 256
-    t0 = time.perf_counter()
-    oracle.gemm_entries(0, qa, sa, 1, qb, sb, rr, cc)
-    per = (time.perf_counter() - t0) / probe
-    count = int(max(probe, min(200000, (budget_s - spent) / max(per, 1e-9))))
-    rng = np.random.default_rng(0)
-    rr, cc = rng.integers(0, rows_a, count), rng.integers(0, 256, count)
-    t0 = time.perf_counter()
-    oracle.gemm_entries(0, qa, sa, 1, qb, sb, rr, cc)
-    per = (time.perf_counter() - t0) / count
-    step_s = t_qa * m * k + t_qb * n * k + per * m * n
-    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "work": 2.0 * m * n * k, "cores": 1,
-            "kind": "oracle",
-            "sample": f"1x128 quantize of {rows_a} rows and 128x128 quantize of 256 rows of the 7168-wide "
-                      f"operands, {count} fp64 GEMM entries (K=7168); extrapolated to the full 4096x2048x7168 "
-                      f"step ({step_s:.1f} s per step on one core)"}
+    phases, unit, what = spec
+    threads = threads or host_threads()
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    calib = run_phases(phases, 0.0, 1)                      # one unit of each phase
+    full_1 = extrapolate(phases, calib)[0]
+    f1 = budget_s / full_1
+    one = run_phases(phases, f1, 1)
+    one_s, work = extrapolate(phases, one)
+    many = run_phases(phases, f1 * threads, threads)
+    many_s, _ = extrapolate(phases, many)
 
+    def sample(runs):
+        return "; ".join(f"{n} of {ph.total} {ph.label}" for ph, (n, _) in zip(phases, runs))
 
-def _cpu_baseline_nvfp4_gemm(oracle, budget_s: float):
-    """The oracle's NVFP4 quantizer on leading rows of both operands and its
-    fp64 GEMM entries (K = 7168), extrapolated to the whole 4096x2048x7168
-    step (both quantizes and every entry)."""
-    m, n, k = 4096, 2048, 7168
-    wl = workloads.ds_fp8_gemm(m, n, k)
-    a, b = workloads.as_u16(wl["a"]), workloads.as_u16(wl["b"])
-    rows = 64
-    t0 = time.perf_counter()
-    qa, sa, ga = oracle.quant_nvfp4(a[:rows])
-    qb, sb, gb = oracle.quant_nvfp4(b[:rows])
-    t_q = (time.perf_counter() - t0) / (2 * rows * k)
-    probe = 64
-    rr, cc = np.arange(probe) % rows, (np.arange(probe) * 7) % rows
-    t0 = time.perf_counter()
-    oracle.gemm_entries(3, qa, sa, 3, qb, sb, rr, cc, ag=ga, bg=gb)
-    per = (time.perf_counter() - t0) / probe
-    count = int(max(probe, min(200000, (budget_s - t_q * 2 * rows * k) / max(per, 1e-9))))
-    rng = np.random.default_rng(0)
-    rr, cc = rng.integers(0, rows, count), rng.integers(0, rows, count)
-    t0 = time.perf_counter()
-    oracle.gemm_entries(3, qa, sa, 3, qb, sb, rr, cc, ag=ga, bg=gb)
-    per = (time.perf_counter() - t0) / count
-    step_s = t_q * (m + n) * k + per * m * n
-    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "work": 2.0 * m * n * k, "cores": 1,
-            "kind": "oracle",
-            "sample": f"NVFP4 quantize of {rows} rows of each 7168-wide operand, {count} fp64 GEMM entries "
-                      f"(K=7168); extrapolated to the full 4096x2048x7168 step ({step_s:.1f} s per step on one core)"}
-
-
-def _timed_entries(fn, probe_count, budget_s):
-    """Seconds per entry of fn(count), calibrated on probe_count entries and
-    then measured on as many as the budget allows; returns (per, count)."""
-    t0 = time.perf_counter()
-    fn(probe_count)
-    per = (time.perf_counter() - t0) / probe_count
-    count = int(max(probe_count, min(200000, budget_s / max(per, 1e-9))))
-    t0 = time.perf_counter()
-    fn(count)
-    return (time.perf_counter() - t0) / count, count
-
-
-def _cpu_baseline_qat_forward(oracle, budget_s: float):
-    """The oracle's LoRA merge + 128x128 fake-quant on the first 128 rows of
-    W, its 1x128 quantize of 64 rows of X and fp64 GEMM entries (K = 7168),
-    extrapolated to the whole 8192x2048x7168 step."""
-    m, n, k = 8192, 2048, 7168
-    wl = workloads.qat_forward()
-    w, la, lb, x = (workloads.as_u16(wl[t]) for t in ("w", "lora_a", "lora_b", "x"))
-    t0 = time.perf_counter()
-    qw, sw, _ = oracle.lora_merge_fakequant(w[:128], la, lb[:128], wl["alpha_over_r"])
-    t_merge = (time.perf_counter() - t0) / 128
-    t0 = time.perf_counter()
-    qx, sx = oracle.quant_fp8_1x128(x[:64])
-    t_qx = (time.perf_counter() - t0) / 64
-    rng = np.random.default_rng(0)
-    per, count = _timed_entries(lambda c: oracle.gemm_entries(0, qx, sx, 1, qw, sw, rng.integers(0, 64, c),
-                                                              rng.integers(0, 128, c)), 64, budget_s * 0.8)
-    step_s = t_merge * n + t_qx * m + per * m * n
-    return {"value": 2.0 * m * n * k / step_s / 1e12, "unit": "TFLOP/s", "work": 2.0 * m * n * k, "cores": 1,
-            "kind": "oracle",
-            "sample": f"LoRA merge + 128x128 fake-quant of 128 rows of W, 1x128 quantize of 64 rows of X, {count} "
-                      f"fp64 GEMM entries (K=7168); extrapolated to the full step ({step_s:.1f} s on one core)"}
-
-
-def _cpu_baseline_qat_backward(oracle, budget_s: float):
-    """The oracle's fp64 bf16-product entries at the contraction lengths of
-    the four products (2048 for dX and dA, 8192 for dW_eff, 7168 for dB),
-    extrapolated to every entry of the step."""
-    m, n, k, r = 8192, 2048, 7168, 16
-    rng = np.random.default_rng(0)
-    per_k = {}
-    counts = {}
-    for kk in (2048, 7168, 8192):
-        p = workloads.as_u16(workloads.normal_bf16((64, kk), 1.0, seed=6000 + kk))
-        q = workloads.as_u16(workloads.normal_bf16((64, kk), 0.02, seed=6001 + kk))
-        per_k[kk], counts[kk] = _timed_entries(
-            lambda c: oracle.gemm_bf16_entries(p, q, rng.integers(0, 64, c), rng.integers(0, 64, c)), 32,
-            budget_s / 3)
-    step_s = per_k[2048] * (m * k + r * k) + per_k[8192] * n * k + per_k[7168] * n * r
-    flops = 2.0 * (2 * m * n * k + 2 * r * n * k)
-    return {"value": flops / step_s / 1e12, "unit": "TFLOP/s", "work": flops, "cores": 1, "kind": "oracle",
-            "sample": f"{sum(counts.values())} fp64 bf16-product entries at K = 2048, 7168 and 8192; extrapolated "
-                      f"to dX, dW_eff, dA and dB in full ({step_s:.0f} s on one core)"}
-
-
-def _cpu_baseline_moe_grouped(oracle, budget_s: float):
-    """The oracle's dispatch of the first tokens and grouped MXFP8 GEMM
-    entries (K = 7168) against two quantized expert slices, extrapolated to
-    the 16384-token step (131072 rows x 2048 columns)."""
-    tokens, experts, k, n, topk = 16384, 64, 7168, 2048, 8
-    wl = workloads.moe_dispatch(tokens=tokens)
-    x, ids = workloads.as_u16(wl["x"][0]), wl["topk_ids"][0].numpy()
-    nt = 256
-    t0 = time.perf_counter()
-    codes, scales, offs = oracle.moe_dispatch([x[:nt]], [ids[:nt]], experts)[0]
-    t_tok = (time.perf_counter() - t0) / nt
-    wq, ws = oracle.quant_mxfp8(np.stack([workloads.as_u16(workloads.normal_bf16((64, k), 0.02, seed=5100 + e))
-                                          for e in range(2)]))
-    rows = min(codes.shape[0], 256)
-    off2 = np.array([0, rows // 2, rows], np.int64)
-    rng = np.random.default_rng(0)
-    per, count = _timed_entries(lambda c: oracle.grouped_gemm_entries(2, codes[:rows], scales[:rows], wq, ws, off2,
-                                                                      rng.integers(0, rows, c),
-                                                                      rng.integers(0, 64, c)), 64, budget_s * 0.8)
-    step_s = t_tok * tokens + per * tokens * topk * n
-    flops = 2.0 * tokens * topk * n * k
-    return {"value": flops / step_s / 1e12, "unit": "TFLOP/s", "work": flops, "cores": 1, "kind": "oracle",
-            "sample": f"oracle dispatch of {nt} tokens, {count} fp64 grouped MXFP8 GEMM entries (K=7168) against "
-                      f"two quantized expert slices; extrapolated to the 16384-token step ({step_s:.0f} s on one "
-                      f"core)"}
-
-
-def _cpu_baseline_moe_dispatch(oracle, budget_s: float):
-    """The oracle's dispatch (route plan, MXFP8 quantization, placement) on
-    the first tokens of the workload (count sized to the budget),
-    extrapolated to the 16384-token step at its per-byte rate."""
-    wl = workloads.moe_dispatch(tokens=16384)
-    x, ids = workloads.as_u16(wl["x"][0]), wl["topk_ids"][0].numpy()
-    hidden, topk = x.shape[1], ids.shape[1]
-    per_tok = hidden * 2 + topk * 8 + topk * (hidden + hidden // 32)
-    n = 256
-    t0 = time.perf_counter()
-    oracle.moe_dispatch([x[:n]], [ids[:n]], 64)
-    per = (time.perf_counter() - t0) / n
-    n = int(max(256, min(16384, budget_s / max(per, 1e-9))))
-    t0 = time.perf_counter()
-    oracle.moe_dispatch([x[:n]], [ids[:n]], 64)
-    dt = time.perf_counter() - t0
-    work = 16384 * per_tok
-    return {"value": n * per_tok / dt / 1e9, "unit": "GB/s", "work": work, "cores": 1, "kind": "oracle",
-            "sample": f"oracle dispatch of the first {n} of 16384 tokens (top-8 of 64 experts, 7168 wide); "
-                      f"extrapolated to the whole step ({16384 / n * dt:.1f} s on one core)"}
-
-
-def _cpu_baseline_prequant(oracle, budget_s: float):
-    """The oracle's MXFP8 and NVFP4 quantizers on leading rows of one
-    2048x7168 expert matrix (rows sized to the budget), extrapolated to the
-    whole 64-expert step at their per-byte rates."""
-    k = 7168
-    x = workloads.as_u16(workloads.normal_bf16((2048, k), 0.02, 4000))
-    rates = {}
-    for fmt, bpe in (("mxfp8", 3 + 1 / 32), ("nvfp4", 2.5 + 1 / 16)):
-        fn = oracle.quant_mxfp8 if fmt == "mxfp8" else oracle.quant_nvfp4
-        rows = 16
-        t0 = time.perf_counter()
-        fn(x[:rows])
-        per_row = (time.perf_counter() - t0) / rows
-        rows = int(max(16, min(2048, budget_s / 2 / max(per_row, 1e-9))))
-        t0 = time.perf_counter()
-        fn(x[:rows])
-        rates[fmt] = (rows * k * bpe, time.perf_counter() - t0, rows, bpe)
-    elems = 64 * 3 * 2048 * 7168
-    work = sum(elems * bpe for (_, _, _, bpe) in rates.values())
-    step_s = sum(elems * bpe * t / b for (b, t, _, bpe) in rates.values())
-    return {"value": work / step_s / 1e9, "unit": "GB/s", "work": work, "cores": 1, "kind": "oracle",
-            "sample": f"MXFP8 quantize of {rates['mxfp8'][2]} rows and NVFP4 quantize of {rates['nvfp4'][2]} rows "
-                      f"of one 2048x7168 expert matrix; extrapolated to the 64-expert step ({step_s:.1f} s per step "
-                      f"on one core)"}
+    return {"value": work / many_s / scale, "unit": unit, "work": work, "cores": threads, "kind": "oracle",
+            "cpu": cpu_model(),
+            "sample": f"{sample(many)}; {sum(dt for _, dt in many):.1f} s on {threads} threads, extrapolated to the "
+                      f"{what} ({many_s:.0f} s)",
+            "one_core": {"value": work / one_s / scale, "unit": unit, "cores": 1,
+                         "sample": f"{sample(one)}; {sum(dt for _, dt in one):.1f} s on one thread, extrapolated "
+                                   f"to the {what} ({one_s:.0f} s)"}}
 
 
 # ------------------------------------------------------------------ main
 
 def run_reference(args, rank, world):
-    """The reference arm: the CPU oracle timed as it stands."""
+    """The reference arm: the CPU oracle as it stands, on every host core.
+    Each step runs the same bounded sample of the workload (a fixed fraction
+    of every phase's units, sized so that warm-up and timed steps end within
+    about two minutes); `ms_per_step` is the measured time of a sampled step
+    and `value` the workload's rate over the timed steps."""
     if rank != 0:
         return
-    if cpu_baseline(args.workload, budget_s=1.0) is None:
+    import oracle
+    oracle.build()
+    oracle.lib()
+    spec = oracle_phases(args.workload, oracle)
+    if spec is None:
         print(json.dumps({"impl": "reference", "unavailable": f"no oracle timing defined for {args.workload}"}))
         return
-    vals = []
-    for _ in range(args.warmup - 1):
-        cpu_baseline(args.workload, budget_s=1.0)
-    t_total = 0.0
+    phases, unit, what = spec
+    threads = host_threads()
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    per_step_s = args.ref_step_s or min(4.0, max(0.5, 120.0 / (args.steps + args.warmup)))
+    full_1 = extrapolate(phases, run_phases(phases, 0.0, 1))[0]
+    frac = per_step_s * threads / full_1
+    for _ in range(args.warmup):
+        run_phases(phases, frac, threads)
+    runs, step_ms = [], []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        r = cpu_baseline(args.workload, budget_s=3.0)
-        t_total += time.perf_counter() - t0
-        vals.append(r["value"])
-    v = statistics.median(vals)
-    unit, work = r["unit"], r["work"]
-    scale = 1e12 if unit == "TFLOP/s" else 1e9
+        runs.append(run_phases(phases, frac, threads))
+        step_ms.append((time.perf_counter() - t0) * 1e3)
+    agg = [(sum(r[i][0] for r in runs), sum(r[i][1] for r in runs)) for i in range(len(phases))]
+    step_s, work = extrapolate(phases, agg)
+    v = work / step_s / scale
+    sample = "; ".join(f"{n} of {ph.total} {ph.label}" for ph, (n, _) in zip(phases, runs[0]))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": work / (v * scale) * 1e3,
+            "warmup": args.warmup, "ms_per_step": statistics.mean(step_ms),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": dict(STEPS[args.workload].CONFIG),
-            "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle", "sample": r["sample"]},
+            "step": f"a fixed sample of the {what} per step ({sample}); value = the whole step's work over its "
+                    f"time extrapolated per phase from the timed steps ({step_s:.0f} s per whole step)",
+            "cpu_baseline": {"value": v, "unit": unit, "cores": threads, "kind": "oracle", "cpu": cpu_model(),
+                             "sample": sample},
             "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
@@ -962,8 +1070,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fpq", choices=["fpq", "reference"])
-    ap.add_argument("--workload", default="ds_fp8_gemm", choices=sorted(STEPS))
+    ap.add_argument("--workload", default="moe_grouped", choices=sorted(STEPS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-step-s", type=float, default=None,
+                    help="reference arm: seconds of oracle work per sampled step (default: about two minutes "
+                         "over warm-up and timed steps, 0.5 to 4 s per step)")
     ap.add_argument("--experts", type=int, default=None,
                     help="moe_prequant only: experts per projection (default 64; fewer for small profiler captures)")
     args = ap.parse_args()
@@ -1134,7 +1245,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": step.unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": step.dtype, "data": "synthetic",
-            "config": dict(step.config, launch=launch_note(step)), "quantize_gbs": quant_gbs,
+            "config": dict(step.CONFIG), "workload_detail": step.config, "launch": launch_note(step),
+            "quantize_gbs": quant_gbs,
             "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"] if quant_gbs is not None else None,
             "kernels": kernels_out, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.launches * args.steps, "clocks": clk.summary(), "clocks_kernel_timing": ck,

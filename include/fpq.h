@@ -451,12 +451,18 @@ FPQ_API fpq_status fpq_grouped_scaled_gemm(fpq_format fmt, const void* aq, const
  * workspace for the largest batch) on every GPU that loads the library, held
  * until the process
  * exits.  No call allocates or frees anything.  batch > the maximum gives
- * FPQ_ERR_INVALID_ARG.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture.  All calls on a device share the
- * array, so calls that may overlap on the GPU (different streams, no
- * ordering between them) race and must not be issued; calls on one stream
- * are safe.
+ * FPQ_ERR_INVALID_ARG.  The first call of this function on a device looks
+ * up the array's device address (cudaGetSymbolAddress) with that device
+ * current and caches it per device ordinal; that lookup is separate from the
+ * one every other entry point makes for the device error word, so a caller
+ * that has already used other entry points on the device must still make
+ * one call of this function outside any stream capture before capturing it.
+ * The cached address assumes the device's primary context for the life of
+ * the process: after cudaDeviceReset, or under a non-primary driver context
+ * on the same ordinal, it no longer names the live array.  All calls on a
+ * device share the array, so calls that may overlap on the GPU (different
+ * streams, no ordering between them) race and must not be issued; calls on
+ * one stream are safe.
  */
 #define FPQ_NOALLOC_NVFP4_MAX_BATCH 4096
 FPQ_API fpq_status fpq_quantize_nvfp4_noalloc(const void* x, int64_t batch, int64_t rows, int64_t cols,

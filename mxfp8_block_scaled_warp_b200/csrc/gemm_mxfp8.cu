@@ -16,9 +16,10 @@
 //           (K = 32 each, scale byte selected per MMA), tcgen05.commit
 //   warps 4-7 epilogue: tcgen05.ld of the accumulator, convert, store
 // Every wait on an mbarrier is bounded by wall time (4 s, or
-// FPQ_WAIT_TIMEOUT_MS); on expiry the kernel records FPQ_ERR_DEVICE_TIMEOUT in
+// FPQ_WAIT_TIMEOUT_MS, read once per process); on expiry the kernel records FPQ_ERR_DEVICE_TIMEOUT in
 // the device error word and unwinds (TMEM freed, no store).  For testing
-// that path, FPQ_DEBUG_GEMM_STALL=1 makes the producer declare more TMA bytes
+// that path, FPQ_DEBUG_GEMM_STALL=1 (also read once per process, so a test sets
+// it before the process's first launch) makes the producer declare more TMA bytes
 // per stage than it loads, so the stage barriers never complete: every load
 // it issues still lands, and the waits run out instead of hanging.
 #include <cstdlib>
@@ -663,15 +664,22 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
 int pair_smem_bytes() { return (int)sizeof(PairSmem) + 1024; }
 
-// Wait limit and the stall switch for the timeout test (see the file header).
+// Wait limit and the stall switch for the timeout test (see the file header),
+// read from the environment once per process, at the first launch.
 uint64_t wait_timeout_ns() {
-    const char* v = std::getenv("FPQ_WAIT_TIMEOUT_MS");
-    const long ms = v ? std::atol(v) : 0;
-    return ms > 0 ? (uint64_t)ms * 1000000ull : kDefaultTimeoutNs;
+    static const uint64_t ns = [] {
+        const char* v = std::getenv("FPQ_WAIT_TIMEOUT_MS");
+        const long ms = v ? std::atol(v) : 0;
+        return ms > 0 ? (uint64_t)ms * 1000000ull : kDefaultTimeoutNs;
+    }();
+    return ns;
 }
 uint32_t debug_extra_tx() {
-    const char* v = std::getenv("FPQ_DEBUG_GEMM_STALL");
-    return (v && v[0] == '1') ? 16u : 0u;
+    static const uint32_t tx = [] {
+        const char* v = std::getenv("FPQ_DEBUG_GEMM_STALL");
+        return (v && v[0] == '1') ? 16u : 0u;
+    }();
+    return tx;
 }
 
 // CTA pairs need the scale rows on 16-byte boundaries (K a multiple of 512)

@@ -28,7 +28,10 @@ std::mutex g_mu;
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// once per device (with that device current) and cached by device ordinal.
+// The cache assumes the device's primary context for the life of the
+// process (no cudaDeviceReset, no other driver context on the ordinal); the
+// device error word of the other entry points is cached the same way.
 fpq_status scratch_on_current_device(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {

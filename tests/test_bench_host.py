@@ -1,7 +1,11 @@
 """Host logic of bench.py without a GPU: every workload's oracle CPU
-baseline (the reference arm) returns a well-formed, positive figure in the
-workload's unit; the launch note names the kernels a step forks; traffic
-from a profile summary is used only while the kernel's source is unchanged."""
+baseline (one thread and all host cores) returns a well-formed, positive
+figure in the workload's unit; the reference arm prints one line whose
+config is the device arm's and whose step time is measured; the launch note
+names the kernels a step forks; traffic from a profile summary is used only
+while the kernel's source is unchanged."""
+import argparse
+import json
 import os
 import sys
 
@@ -19,7 +23,29 @@ def test_cpu_baseline_every_workload(workload):
     assert r is not None, f"no oracle timing for {workload}"
     step = bench.STEPS[workload]
     assert r["unit"] == step.unit and r["value"] > 0 and r["work"] > 0
-    assert r["kind"] == "oracle" and r["cores"] == 1 and r["sample"]
+    assert r["kind"] == "oracle" and r["cores"] == bench.host_threads() and r["sample"] and r["cpu"]
+    one = r["one_core"]
+    assert one["cores"] == 1 and one["value"] > 0 and one["unit"] == step.unit and one["sample"]
+
+
+def test_run_phases_covers_every_unit_once():
+    seen = []
+    ph = bench.OraclePhase("units", 1000, 1.0, lambda lo, hi: seen.extend(range(lo, hi)))
+    runs = bench.run_phases([ph], 0.25, 3)
+    assert runs[0][0] == 250 and sorted(seen) == list(range(250))
+    step_s, work = bench.extrapolate([ph], [(250, 2.0)])
+    assert step_s == pytest.approx(8.0) and work == 1000.0
+
+
+def test_reference_line(capsys):
+    args = argparse.Namespace(workload="qat_backward", steps=2, warmup=1, ref_step_s=0.1)
+    bench.run_reference(args, 0, 1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOP/s"
+    assert line["config"] == bench.STEPS["qat_backward"].CONFIG
+    assert 0 < line["ms_per_step"] < 60_000            # a measured sampled step, not an extrapolation
+    assert line["cpu_baseline"]["cores"] == bench.host_threads()
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
 
 
 def test_launch_note_names_forked_kernels():
