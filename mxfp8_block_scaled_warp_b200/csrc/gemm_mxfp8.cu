@@ -365,13 +365,15 @@ gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
 int smem_bytes() { return (int)sizeof(Smem) + 1024; }
 
-// ============================================================== CTA pair
-// A cluster of two CTAs computes one 256 x 256 tile with tcgen05 cta_group::2
-// (grouped: 256 rows of one group).  CTA r stages A rows a_row0 = row_begin +
-// 256 mt + 128 r and B rows n0 + 128 r of each 128-wide K tile in its own
-// shared memory and receives its 128 accumulator rows in its own TMEM; per SM
-// a K tile is 16 + 16 KB of codes instead of 16 + 32 KB, which is what bounds
-// the one-CTA kernel (the TMA feed from L2).  The leader issues the MMAs
+// ============================================================== CTA pairs, persistent
+// A cluster of two CTAs computes 256 x 256 output tiles with tcgen05
+// cta_group::2 (grouped: 256 rows of one group), walking the tile list
+// pair, pair + P, pair + 2P, ... (P = the pairs launched, at most one per
+// two SMs).  CTA r of the pair stages A rows row_begin + 256 mt + 128 r and
+// B rows n0 + 128 r of every 128-wide K tile in its own shared memory and
+// receives its 128 accumulator rows in its own TMEM; per SM a K tile is
+// 16 + 16 KB of codes instead of the one-CTA kernel's 16 + 32 KB (the TMA
+// feed from L2 is what bounds that kernel).  The leader issues the MMAs
 // (M = 256, N = 256, 4 x K = 32 per K tile, scale byte selected per MMA) and
 // the scale copies, and commits to the barriers of both CTAs.
 //
@@ -381,10 +383,19 @@ int smem_bytes() { return (int)sizeof(Smem) + 1024; }
 // 4-7 rearrange a landed chunk in place into the TMEM-copy atoms of its K
 // tiles (warp 4 + i: K tiles 2i, 2i + 1) and arrive on the leader's sfr.
 //
+// TMEM holds one 256-column accumulator and the scale columns of the ring's
+// stages, so the accumulator is handed over instead of double-buffered: the
+// eight epilogue warps (8-15; warp w reads TMEM lanes 32 (w & 3) .. + 31 and
+// columns 128 ((w - 8) >> 2) .. + 127) read their block into registers,
+// arrive on the leader's tmem_empty, and only then convert and store to C,
+// while the code and scale producers, which run ahead by the ring's depth,
+// and the MMAs of the next tile proceed.  Each thread stores one row segment
+// (rows outside the group and columns past N skipped).
+//
 // Warp roles in both CTAs: warp 0 code-tile TMA producer; warp 1 scale-chunk
 // TMA producer; warp 2 TMEM allocator (leader: MMA issuer); warps 4-7 scale
-// loaders; then all eight warps run the epilogue: whole 32-row blocks inside
-// the group by TMA stores, a block crossing the group's end by masked stores.
+// loaders; warps 8-15 epilogue.  The pipeline counters (ring stage, scale
+// chunk, tile parity) run on across tiles.
 constexpr int P_STAGES = 6;
 constexpr int P_A_TILE = 128 * BK, P_B_TILE = 128 * BK;
 constexpr int P_SF_CH = 8;                                   // K tiles per scale chunk
@@ -395,7 +406,8 @@ static_assert(P_SF_CH * P_TILE_ATOMS == P_SFC_BYTES, "in-place rearrangement");
 static_assert(P_SF_CH == 8, "loader warp 4 + i takes K tiles 2i and 2i + 1 of a chunk");
 constexpr uint32_t P_SF_COL0 = 256;
 static_assert(P_SF_COL0 + P_STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM columns (pair)");
-constexpr int P_EPI_WARP_BYTES = 32 * 128 * 4;               // a warp's 32 x 128 block of C, fp32
+constexpr int P_THREADS = 512;
+constexpr int P_EPI_WARP0 = 8, P_EPI_WARPS = 8;
 
 struct __align__(1024) PairSmem {
     uint8_t a[P_STAGES][P_A_TILE];
@@ -406,38 +418,55 @@ struct __align__(1024) PairSmem {
     uint64_t sff[2];            // this CTA's scale chunk has landed
     uint64_t sfr[2];            // leader's copy used: atoms of both CTAs written (8 warps)
     uint64_t sf_empty[2];       // both CTAs: the leader's commit after a chunk's last MMAs
-    uint64_t tmem_full;         // both CTAs: the leader's commit after the last MMA
+    uint64_t tmem_full;         // both CTAs: the leader's commit after a tile's last MMA
+    uint64_t tmem_empty;        // leader's copy used: the epilogue warps of both CTAs read the accumulator
     uint32_t tmem_base;
-    int32_t tile_valid;
-    int32_t group;
-    int32_t row_begin, row_end;
-    int32_t m_tile, n_tile;
+    int32_t tiles;              // pair tiles of the whole product (0: nothing to do or malformed offsets)
     int32_t off[kMaxGroups + 1];
 };
-static_assert(8 * P_EPI_WARP_BYTES <= P_STAGES * (P_A_TILE + P_B_TILE), "epilogue staging exceeds the ring");
 
-// Byte offset of 16-byte chunk j (0-7) of row r in a box of 128-byte rows
-// stored with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t box_off(int r, int j) { return (uint32_t)(r * 128 + 16 * (j ^ (r & 7))); }
+// Number of 2 BM-row tiles of the product, run by one warp; grouped offsets
+// are validated as in map_tile (malformed: reported once, 0 tiles).
+__device__ int count_tiles(int bm, const int32_t* off, bool grouped, int groups, int64_t M, int n_tiles, int lane,
+                           uint32_t* err) {
+    if (!grouped) return (int)((M + bm - 1) / bm) * n_tiles;
+    bool bad = off[0] != 0 || off[groups] != (int32_t)M;
+    int total = 0;
+    for (int c0 = 0; c0 < groups; c0 += 32) {
+        const int e = c0 + lane;
+        const int32_t b0 = e < groups ? off[e] : 0, b1 = e < groups ? off[e + 1] : 0;
+        if (b1 < b0) bad = true;
+        int tiles = b1 > b0 ? ((b1 - b0 + bm - 1) / bm) * n_tiles : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tiles += __shfl_xor_sync(0xFFFFFFFFu, tiles, o);
+        total += tiles;
+    }
+    if (__any_sync(0xFFFFFFFFu, bad)) {
+        if (blockIdx.x == 0 && lane == 0) raise_device_error(err, FPQ_ERR_DEVICE_BAD_INPUT);
+        return 0;
+    }
+    return total;
+}
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
 gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                       const __grid_constant__ CUtensorMap tmC, const int32_t* __restrict__ offsets, int groups,
-                       int64_t M, int64_t N, int64_t K, void* __restrict__ C, int c_f32, uint32_t* err,
-                       uint64_t timeout_ns, uint32_t extra_tx) {
+                       const int32_t* __restrict__ offsets, int groups, int64_t M, int64_t N, int64_t K,
+                       void* __restrict__ C, int c_f32, uint32_t* err, uint64_t timeout_ns, uint32_t extra_tx) {
     extern __shared__ uint8_t smem_raw[];
     PairSmem& sm = *reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
+    const bool grouped = offsets != nullptr;
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
     const int n_tiles = (int)((N + BN - 1) / BN);
     const int KT = (int)(K / BK);
     const int NC = (KT + P_SF_CH - 1) / P_SF_CH;
 
-    if (offsets != nullptr) {
+    if (grouped) {
         pdl_wait();    // the group offsets may come from the preceding grid
-        for (int i = threadIdx.x; i <= groups; i += NUM_THREADS) sm.off[i] = offsets[i];
+        for (int i = threadIdx.x; i <= groups; i += P_THREADS) sm.off[i] = offsets[i];
     }
     if (threadIdx.x == 32) {
         for (int s = 0; s < P_STAGES; ++s) {
@@ -450,24 +479,18 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             mbar_init(&sm.sf_empty[b], 1);
         }
         mbar_init(&sm.tmem_full, 1);
+        mbar_init(&sm.tmem_empty, 2 * P_EPI_WARPS);
         fence_barrier_init();
     }
     __syncthreads();
     if (warp == 0) {
-        // both CTAs of the pair map the same pair tile
-        const TileMap tm = map_tile((int)(blockIdx.x >> 1), 2 * BM, sm.off, offsets != nullptr, groups, M, n_tiles,
-                                    lane, err);
-        if (lane == 0) {
-            sm.tile_valid = tm.valid;
-            sm.group = tm.g;
-            sm.m_tile = tm.mt;
-            sm.n_tile = tm.nt;
-            sm.row_begin = tm.rb;
-            sm.row_end = tm.re;
-        }
+        const int t = count_tiles(2 * BM, sm.off, grouped, groups, M, n_tiles, lane, err);
+        if (lane == 0) sm.tiles = t;
     }
     __syncthreads();
-    if (!sm.tile_valid) return;      // the same decision in both CTAs
+    // the same count in both CTAs of a pair: both leave here or neither
+    const int my_tiles = sm.tiles > pair ? (sm.tiles - pair + npairs - 1) / npairs : 0;
+    if (my_tiles == 0) return;
 
     if (warp == 2) {
         tmem_alloc_pair(&sm.tmem_base, TMEM_COLS);
@@ -479,73 +502,97 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     const uint32_t tmem = sm.tmem_base;
     pdl_wait();
 
-    const int64_t a_row0 = (int64_t)sm.row_begin + (int64_t)sm.m_tile * 2 * BM + 128 * (int64_t)rank;
-    const int64_t a_rows_end = sm.row_end;
-    const int64_t n0 = (int64_t)sm.n_tile * BN;
-    const int64_t bt_row0 = (int64_t)sm.group * N + n0;       // the tile's first B row (flattened)
-
     if (warp == 0) {
         // ---------------------------------------------------------- code-tile TMA producer
-        if (elect_one()) {
+        if (lane == 0) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
-            tma_prefetch_desc(&tmC);
-            for (int kt = 0; kt < KT; ++kt) {
-                const int s = kt % P_STAGES;
-                const uint32_t ph = (uint32_t)(kt / P_STAGES) & 1u;
-                if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err, timeout_ns)) break;
-                if (leader) mbar_arrive_expect_tx(&sm.full[s], 2 * (P_A_TILE + P_B_TILE) + extra_tx);
-                tma_load_2d_pair(sm.a[s], &tmA, &sm.full[s], kt * BK, (int32_t)a_row0);
-                tma_load_2d_pair(sm.b[s], &tmB, &sm.full[s], kt * BK, (int32_t)(bt_row0 + 128 * rank));
+        }
+        uint32_t it = 0;
+        bool alive = true;
+        for (int i = 0; i < my_tiles && alive; ++i) {
+            const TileMap tm = map_tile(pair + i * npairs, 2 * BM, sm.off, grouped, groups, M, n_tiles, lane, err);
+            const int32_t a_row0 = tm.rb + tm.mt * 2 * BM + 128 * (int32_t)rank;
+            const int32_t b_row0 = (int32_t)((int64_t)tm.g * N + (int64_t)tm.nt * BN + 128 * rank);
+            if (lane == 0) {
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = (int)(it % P_STAGES);
+                    const uint32_t ph = (it / P_STAGES) & 1u;
+                    if (!wait_or_timeout(&sm.empty[s], ph ^ 1u, err, timeout_ns)) { alive = false; break; }
+                    if (leader) mbar_arrive_expect_tx(&sm.full[s], 2 * (P_A_TILE + P_B_TILE) + extra_tx);
+                    tma_load_2d_pair(sm.a[s], &tmA, &sm.full[s], kt * BK, a_row0);
+                    tma_load_2d_pair(sm.b[s], &tmB, &sm.full[s], kt * BK, b_row0);
+                }
             }
+            alive = __shfl_sync(0xFFFFFFFFu, alive, 0);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- scale-chunk TMA producer
-        if (elect_one()) {
+        if (lane == 0) {
             tma_prefetch_desc(&tmSA);
             tma_prefetch_desc(&tmSB);
-            for (int c = 0; c < NC; ++c) {
-                const int b = c & 1;
-                const uint32_t ph = (uint32_t)(c >> 1) & 1u;
-                if (!wait_or_timeout(&sm.sf_empty[b], ph ^ 1u, err, timeout_ns)) break;
-                mbar_arrive_expect_tx(&sm.sff[b], P_SFC_BYTES);
-                tma_load_2d(sm.sfc[b], &tmSA, &sm.sff[b], c * 4 * P_SF_CH, (int32_t)a_row0);
-                tma_load_2d(sm.sfc[b] + P_SFC_A, &tmSB, &sm.sff[b], c * 4 * P_SF_CH, (int32_t)bt_row0);
+        }
+        uint32_t cc = 0;
+        bool alive = true;
+        for (int i = 0; i < my_tiles && alive; ++i) {
+            const TileMap tm = map_tile(pair + i * npairs, 2 * BM, sm.off, grouped, groups, M, n_tiles, lane, err);
+            const int32_t a_row0 = tm.rb + tm.mt * 2 * BM + 128 * (int32_t)rank;
+            const int32_t bt_row0 = (int32_t)((int64_t)tm.g * N + (int64_t)tm.nt * BN);
+            if (lane == 0) {
+                for (int c = 0; c < NC; ++c, ++cc) {
+                    const int b = (int)(cc & 1u);
+                    const uint32_t ph = (cc >> 1) & 1u;
+                    if (!wait_or_timeout(&sm.sf_empty[b], ph ^ 1u, err, timeout_ns)) { alive = false; break; }
+                    mbar_arrive_expect_tx(&sm.sff[b], P_SFC_BYTES);
+                    tma_load_2d(sm.sfc[b], &tmSA, &sm.sff[b], c * 4 * P_SF_CH, a_row0);
+                    tma_load_2d(sm.sfc[b] + P_SFC_A, &tmSB, &sm.sff[b], c * 4 * P_SF_CH, bt_row0);
+                }
             }
+            alive = __shfl_sync(0xFFFFFFFFu, alive, 0);
         }
     } else if (warp == 2) {
         // ---------------------------------------------------------- MMA issuer (leader)
         if (leader && elect_one()) {
+            uint32_t it = 0, cc = 0;
             bool ok = true;
-            for (int kt = 0; kt < KT; ++kt) {
-                const int s = kt % P_STAGES;
-                const uint32_t ph = (uint32_t)(kt / P_STAGES) & 1u;
-                const int c = kt / P_SF_CH, t = kt - c * P_SF_CH, b = c & 1;
-                if (!wait_or_timeout(&sm.full[s], ph, err, timeout_ns) ||
-                    (t == 0 && !wait_or_timeout(&sm.sfr[b], (uint32_t)(c >> 1) & 1u, err, timeout_ns))) {
-                    ok = false;
-                    break;
-                }
+            for (int i = 0; i < my_tiles && ok; ++i) {
+                // the accumulator is free once both CTAs' epilogue warps have read the previous tile
+                if (!wait_or_timeout(&sm.tmem_empty, ((uint32_t)i & 1u) ^ 1u, err, timeout_ns)) break;
                 tc_fence_after();
-                const uint32_t sf_col = tmem + P_SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
-                const uint8_t* at = sm.sfc[b] + t * P_TILE_ATOMS;
-                tmem_cp_32x128b_warpx4_pair(sf_col + 0, smem_desc(smem_u32(at), 0, 128, kLayoutNone));
-                tmem_cp_32x128b_warpx4_pair(sf_col + 4, smem_desc(smem_u32(at + SFA_BYTES), 0, 128, kLayoutNone));
-                tmem_cp_32x128b_warpx4_pair(sf_col + 8, smem_desc(smem_u32(at + SFA_BYTES + 512), 0, 128, kLayoutNone));
-                const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = (int)(it % P_STAGES);
+                    const uint32_t ph = (it / P_STAGES) & 1u;
+                    const int t = kt % P_SF_CH;
+                    const uint32_t ch = cc + (uint32_t)(kt / P_SF_CH);
+                    const int b = (int)(ch & 1u);
+                    if (!wait_or_timeout(&sm.full[s], ph, err, timeout_ns) ||
+                        (t == 0 && !wait_or_timeout(&sm.sfr[b], (ch >> 1) & 1u, err, timeout_ns))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sf_col = tmem + P_SF_COL0 + SF_COLS_PER_STAGE * (uint32_t)s;
+                    const uint8_t* at = sm.sfc[b] + t * P_TILE_ATOMS;
+                    tmem_cp_32x128b_warpx4_pair(sf_col + 0, smem_desc(smem_u32(at), 0, 128, kLayoutNone));
+                    tmem_cp_32x128b_warpx4_pair(sf_col + 4, smem_desc(smem_u32(at + SFA_BYTES), 0, 128, kLayoutNone));
+                    tmem_cp_32x128b_warpx4_pair(sf_col + 8,
+                                                smem_desc(smem_u32(at + SFA_BYTES + 512), 0, 128, kLayoutNone));
+                    const uint32_t a_base = smem_u32(sm.a[s]), b_base = smem_u32(sm.b[s]);
 #pragma unroll
-                for (int k = 0; k < BK / 32; ++k) {
-                    const uint32_t idesc = idesc_mxf8f6f4(2 * BM, BN, (uint32_t)k, (uint32_t)k);
-                    mma_mxf8f6f4_pair(tmem, desc_kmajor_sw128(a_base + 32 * k), desc_kmajor_sw128(b_base + 32 * k),
-                                      idesc, (sf_col + 0) | ((uint32_t)k << 30), (sf_col + 4) | ((uint32_t)k << 30),
-                                      (kt > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < BK / 32; ++k) {
+                        const uint32_t idesc = idesc_mxf8f6f4(2 * BM, BN, (uint32_t)k, (uint32_t)k);
+                        mma_mxf8f6f4_pair(tmem, desc_kmajor_sw128(a_base + 32 * k), desc_kmajor_sw128(b_base + 32 * k),
+                                          idesc, (sf_col + 0) | ((uint32_t)k << 30), (sf_col + 4) | ((uint32_t)k << 30),
+                                          (kt > 0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair_multicast(&sm.empty[s], 0x3);
+                    if (t == P_SF_CH - 1 || kt == KT - 1) mma_commit_pair_multicast(&sm.sf_empty[b], 0x3);
                 }
-                mma_commit_pair_multicast(&sm.empty[s], 0x3);
-                if (t == P_SF_CH - 1 || kt == KT - 1) mma_commit_pair_multicast(&sm.sf_empty[b], 0x3);
+                if (ok) mma_commit_pair_multicast(&sm.tmem_full, 0x3);
+                cc += (uint32_t)NC;
             }
-            if (ok) mma_commit_pair_multicast(&sm.tmem_full, 0x3);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < P_EPI_WARP0) {
         // ---------------------------------------------------------- scale loaders
         // Lane l reads, for K tiles 2i and 2i + 1 of the chunk (i = warp - 4),
         // the 8 scale bytes of A rows l + 32 q (q < 4) and B rows l + 32 q
@@ -553,9 +600,10 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         // writes its two K tiles' atoms: word q of lane l = row l + 32 q.
         const int i2 = 2 * (warp - 4);
         const uint32_t leader_sfr0 = map_to_rank(smem_u32(&sm.sfr[0]), 0);
-        for (int c = 0; c < NC; ++c) {
-            const int b = c & 1;
-            const uint32_t ph = (uint32_t)(c >> 1) & 1u;
+        const uint32_t chunks = (uint32_t)my_tiles * (uint32_t)NC;
+        for (uint32_t cc = 0; cc < chunks; ++cc) {
+            const int b = (int)(cc & 1u);
+            const uint32_t ph = (cc >> 1) & 1u;
             const bool landed = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.sff[b], ph, err, timeout_ns));
             uint2 ra[4], rb[8];
             const uint8_t* dense = sm.sfc[b];
@@ -582,78 +630,61 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_sfr0 + 8u * (uint32_t)b);
         }
-    }
-
-    // -------------------------------------------------------------- epilogue
-    // All eight warps once the last MMA has completed (the operand ring is
-    // then free): warp w reads TMEM lanes 32 (w & 3) .. + 31 (this CTA's
-    // accumulator rows) and columns 128 (w >> 2) .. + 127, stages the 32 x 128
-    // block in 128-byte-swizzled boxes, then writes it with TMA stores (the
-    // unit clips rows past M and columns past N) when all 32 rows belong to
-    // the group, else row by row, skipping rows outside the group.
-    __syncwarp();
-    {
-        const int q = warp & 3, half = warp >> 2;
-        const int64_t row0 = a_row0 + 32 * q, col0 = n0 + 128 * half;
-        const bool ok = __all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.tmem_full, 0, err, timeout_ns));
-        if (ok && row0 < a_rows_end && col0 < N) {
+    } else if (warp >= P_EPI_WARP0) {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3, half = (warp - P_EPI_WARP0) >> 2;
+        const uint32_t leader_empty = map_to_rank(smem_u32(&sm.tmem_empty), 0);
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half);
+        for (int i = 0; i < my_tiles; ++i) {
+            const TileMap tm = map_tile(pair + i * npairs, 2 * BM, sm.off, grouped, groups, M, n_tiles, lane, err);
+            const int64_t row = (int64_t)tm.rb + (int64_t)tm.mt * 2 * BM + 128 * (int64_t)rank + 32 * q + lane;
+            const int64_t col0 = (int64_t)tm.nt * BN + 128 * half;
+            const bool row_ok = row < (int64_t)tm.re;
+            if (!__all_sync(0xFFFFFFFFu, wait_or_timeout(&sm.tmem_full, (uint32_t)i & 1u, err, timeout_ns))) break;
             tc_fence_after();
-            uint8_t* stage = &sm.a[0][0] + warp * P_EPI_WARP_BYTES;
-            uint32_t r[4][32];
+            if (!c_f32) {
+                uint32_t h[64];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * half + 32 * c), r[c]);
-            tmem_ld_wait();
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(taddr + (uint32_t)(16 * c), r);
+                    tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (c_f32) {     // columns 32c .. 32c + 31 = box c
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4*>(stage + c * 4096 + box_off(lane, j)) =
-                            make_uint4(r[c][4 * j], r[c][4 * j + 1], r[c][4 * j + 2], r[c][4 * j + 3]);
-                } else {         // columns 32c .. 32c + 31 = box c / 2, chunks 4 (c % 2) .. + 3
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t h[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            h[e] = f32x2_to_bf16x2(__uint_as_float(r[c][8 * j + 2 * e]),
-                                                   __uint_as_float(r[c][8 * j + 2 * e + 1]));
-                        *reinterpret_cast<uint4*>(stage + (c / 2) * 4096 + box_off(lane, 4 * (c % 2) + j)) =
-                            make_uint4(h[0], h[1], h[2], h[3]);
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        h[8 * c + e] = f32x2_to_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
                 }
-            }
-            const int boxes = c_f32 ? 4 : 2, box_cols = c_f32 ? 32 : 64;
-            if (row0 + 32 <= a_rows_end) {
-                fence_proxy_async_smem();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    for (int x = 0; x < boxes; ++x)
-                        if (col0 + x * box_cols < N)
-                            tma_store_2d(&tmC, stage + x * 4096, (int32_t)(col0 + x * box_cols), (int32_t)row0);
-                    bulk_commit_group();
-                    bulk_wait_group_read0();     // the staging must stay valid until read
+                if (lane == 0) mbar_arrive_cluster(leader_empty);
+                if (row_ok) {
+                    uint8_t* dst = reinterpret_cast<uint8_t*>(C) + (row * N + col0) * 2;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (col0 + 8 * j < N) st_v4(dst + 16 * j, make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]));
                 }
             } else {
-                __syncwarp();
-                // a row is 16 (bf16) or 32 (fp32) 16-byte chunks: lanes take
-                // chunk lane % chunks of row rr + lane / chunks
-                const int chunks = c_f32 ? 32 : 16, rows_per = 32 / chunks, esz = c_f32 ? 4 : 2;
-                const int ch = lane % chunks, box = ch / 8, j = ch % 8;
-                for (int rr = lane / chunks; rr < 32; rr += rows_per) {
-                    const int64_t row = row0 + rr;
-                    const int64_t col = col0 + (int64_t)ch * (16 / esz);
-                    if (row < a_rows_end && col < N)
-                        st_v4(reinterpret_cast<uint8_t*>(C) + (row * N + col) * esz,
-                              *reinterpret_cast<const uint4*>(stage + box * 4096 + box_off(rr, j)));
+                uint8_t* dst = reinterpret_cast<uint8_t*>(C) + (row * N + col0) * 4;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + (uint32_t)(32 * c), r);
+                    tmem_ld_wait();
+                    if (row_ok) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            if (col0 + 32 * c + 4 * j < N)
+                                st_v4(dst + 128 * c + 16 * j, make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
+                    }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(leader_empty);
             }
-            __syncwarp();
         }
     }
 
     // both CTAs done: no MMA, copy, TMEM read or remote arrival outstanding
+    __syncwarp();
     tc_fence_before();
     cluster_sync();
     if (warp == 2) {
@@ -688,7 +719,7 @@ bool use_pair(int64_t M, int64_t K) { return K % 512 == 0 && M > BM; }
 
 cudaError_t launch(const void* aq, const void* as, const void* bq, const void* bs, const int32_t* offsets,
                    int groups, int64_t M, int64_t N, int64_t K, void* c, int c_f32, uint32_t* err,
-                   int64_t tiles, int64_t pair_tiles, cudaStream_t st) {
+                   int64_t tiles, int64_t pair_tiles, int sms, cudaStream_t st) {
     const bool pair = use_pair(M, K);
     CUtensorMap ta, tb;
     cudaError_t e = make_tmap_u8_2d(&ta, aq, (uint64_t)M, (uint64_t)K, (uint64_t)K, BM, BK);
@@ -703,25 +734,21 @@ cudaError_t launch(const void* aq, const void* as, const void* bq, const void* b
                           (const uint8_t*)as, (const uint8_t*)bs, offsets, groups, M, N, K, c, c_f32, err,
                           wait_timeout_ns(), debug_extra_tx());
     }
-    CUtensorMap tsa, tsb, tc;
+    CUtensorMap tsa, tsb;
     e = make_tmap_2d(&tsa, as, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)M, (uint64_t)(K / 32), (uint64_t)(K / 32),
                      128, 4 * P_SF_CH, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess) return e;
     e = make_tmap_2d(&tsb, bs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(groups * N), (uint64_t)(K / 32),
                      (uint64_t)(K / 32), 256, 4 * P_SF_CH, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess) return e;
-    if (c_f32)
-        e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)M, (uint64_t)N, (uint64_t)N * 4, 32, 32,
-                         CU_TENSOR_MAP_SWIZZLE_128B);
-    else
-        e = make_tmap_2d(&tc, c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)M, (uint64_t)N, (uint64_t)N * 2, 32, 64,
-                         CU_TENSOR_MAP_SWIZZLE_128B);
-    if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gemm_mxfp8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pair_smem_bytes());
     if (e != cudaSuccess) return e;
     if (pair_tiles < 1) return cudaSuccess;
-    return launch_pdl(gemm_mxfp8_pair_kernel, dim3((unsigned)(2 * pair_tiles)), dim3(NUM_THREADS), pair_smem_bytes(),
-                      st, ta, tb, tsa, tsb, tc, offsets, groups, M, N, K, c, c_f32, err, wait_timeout_ns(),
+    // persistent: at most one pair per two SMs; the kernel counts the real
+    // tiles (grouped: from the device-side offsets) and walks them
+    const int64_t pairs = min64(pair_tiles, (int64_t)(sms > 1 ? sms / 2 : 1));
+    return launch_pdl(gemm_mxfp8_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(P_THREADS), pair_smem_bytes(),
+                      st, ta, tb, tsa, tsb, offsets, groups, M, N, K, c, c_f32, err, wait_timeout_ns(),
                       debug_extra_tx());
 }
 
@@ -729,22 +756,20 @@ cudaError_t launch(const void* aq, const void* as, const void* bq, const void* b
 
 cudaError_t launch_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs, int64_t m,
                               int64_t n, int64_t k, void* c, int c_f32, uint32_t* err, int sms, cudaStream_t st) {
-    (void)sms;
     const int64_t n_tiles = (n + BN - 1) / BN;
     return launch(aq, as, bq, bs, nullptr, 1, m, n, k, c, c_f32, err, ((m + BM - 1) / BM) * n_tiles,
-                  ((m + 2 * BM - 1) / (2 * BM)) * n_tiles, st);
+                  ((m + 2 * BM - 1) / (2 * BM)) * n_tiles, sms, st);
 }
 
 cudaError_t launch_grouped_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs,
                                       const int32_t* offsets, int groups, int64_t total_m, int64_t n, int64_t k,
                                       void* c, int c_f32, uint32_t* err, int sms, cudaStream_t st) {
-    (void)sms;
     // Upper bounds on the tile counts without reading the device-side
     // offsets: every group adds at most one partial row tile.
     const int64_t n_tiles = (n + BN - 1) / BN;
     return launch(aq, as, bq, bs, offsets, groups, total_m, n, k, c, c_f32, err,
                   ((total_m + BM - 1) / BM + groups) * n_tiles, ((total_m + 2 * BM - 1) / (2 * BM) + groups) * n_tiles,
-                  st);
+                  sms, st);
 }
 
 }  // namespace fpq
