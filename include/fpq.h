@@ -417,6 +417,35 @@ FPQ_API fpq_status fpq_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t
                                           const int64_t* dst_capacity, void* stream);
 
 /*
+ * fpq_moe_regroup -- the receiving side of the exchange in the PACK mode
+ * ["DeepSeek-V3 Blog 5: Low-Precision Training", Reducing Communication
+ * Overhead in MoE with FP8].  A PACK send buffer holds a rank's rows expert-
+ * major, so the rows bound for rank p (experts [p L, (p + 1) L)) are one
+ * contiguous run, and one all-to-all with per-rank row counts delivers them.
+ * The receiver then holds its rows source-major: all of source 0's rows for
+ * its experts (expert-major, slot order), then source 1's, ...  This call
+ * moves them into the receive layout above (expert-major; within an expert,
+ * source 0, 1, ...): segment (local expert l, source s) of
+ * counts_all[s][rank L + l] rows.
+ *
+ *   recv_codes, recv_scales  DEVICE uint8 [rows, hidden] E4M3 codes and
+ *               [rows, hidden / 32] E8M0 scales, source-major (input)
+ *   counts_all  DEVICE int32 [world, E] (as for fpq_moe_dispatch_layout)
+ *   rows        rows of the input and of the output buffers:
+ *               sum over s and l of counts_all[s][rank L + l]
+ *   codes, scales  DEVICE, same shapes (output; must not overlap the input)
+ *
+ * Requires world >= 1 dividing E, 1 <= E <= 1024, 0 <= rank < world, hidden
+ * a positive multiple of 32, 0 <= rows < 2^31, 16-byte aligned code
+ * buffers.  A negative count, or a segment past `rows`, is malformed device
+ * input: FPQ_ERR_DEVICE_BAD_INPUT in the device error word, that segment not
+ * copied.  Errors: FPQ_ERR_INVALID_ARG, FPQ_ERR_ALIGNMENT, FPQ_ERR_CUDA.
+ */
+FPQ_API fpq_status fpq_moe_regroup(const void* recv_codes, const void* recv_scales, const int32_t* counts_all,
+                                   int32_t world, int32_t num_experts, int32_t rank, int64_t hidden, int64_t rows,
+                                   void* codes, void* scales, void* stream);
+
+/*
  * fpq_grouped_scaled_gemm -- per-expert product over a token-permuted
  * activation matrix (MoE routed experts) [FP "Quick start": routed MoE
  * expert projections; DS "Как FP8 связан с MoE-архитектурой DeepSeek V3"]:

@@ -28,6 +28,7 @@ __all__ = [
     "fpq_get_device_error", "fpq_gemm_bf16", "fpq_gemm_bf16_layout", "fpq_transpose_bf16",
     "fpq_gemm_bf16_splitk_workspace_bytes", "fpq_gemm_bf16_splitk", "fpq_qat_backward_workspace_bytes",
     "fpq_moe_route_workspace_bytes", "fpq_moe_route", "fpq_moe_dispatch_layout", "fpq_moe_dispatch_mxfp8",
+    "fpq_moe_regroup",
     "fpq_quantize_block_strided", "fpq_dequantize_strided",
     "MOE_DIRECT", "MOE_PACK",
     "fpq_qat_backward",
@@ -93,6 +94,7 @@ def _load() -> ctypes.CDLL:
         "fpq_moe_route": (I32, [P, I64, I32, I32, P, P, SZ, P]),
         "fpq_moe_dispatch_layout": (I32, [P, I32, I32, I32, I32, P, P, P]),
         "fpq_moe_dispatch_mxfp8": (I32, [P, I64, I64, P, I32, I32, P, SZ, P, I32, P, P, P, P]),
+        "fpq_moe_regroup": (I32, [P, P, P, I32, I32, I32, I64, I64, P, P, P]),
         "fpq_qat_backward": (I32, [P, P, P, P, P, I64, I64, I64, I32, F, P, P, P, P, P, SZ, P]),
         "fpq_quantize_nvfp4_noalloc": (I32, [P, I64, I64, I64, P, P, P, P]),
     }
@@ -236,6 +238,15 @@ def fpq_moe_dispatch_mxfp8(x, tokens, hidden, topk_ids, topk, num_experts, works
                                          _ptr(workspace) if workspace is not None else None, wsb, _ptr(dst_row0),
                                          n_dest, _ptr(dst_codes), _ptr(dst_scales), _ptr(dst_capacity),
                                          _stream(stream)), "fpq_moe_dispatch_mxfp8")
+
+
+def fpq_moe_regroup(recv_codes, recv_scales, counts_all, world, num_experts, rank, hidden, rows, codes, scales,
+                    stream=None):
+    """Source-major received rows -> the expert-grouped receive layout."""
+    if rows == 0:
+        return
+    _check(load().fpq_moe_regroup(_ptr(recv_codes), _ptr(recv_scales), _ptr(counts_all), world, num_experts, rank,
+                                  hidden, rows, _ptr(codes), _ptr(scales), _stream(stream)), "fpq_moe_regroup")
 
 
 def fpq_transpose_bf16(x, out, rows, cols, stream=None):

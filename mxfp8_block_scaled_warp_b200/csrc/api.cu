@@ -245,7 +245,7 @@ fpq_status fpq_lora_merge_fakequant(const void* w, const void* lora_a, const voi
     const DeviceState* d = device_state(&st);
     if (!d) return st;
     return from_cuda(fpq::launch_lora_merge_fakequant(w, lora_a, lora_b, n, k, r, alpha_over_r, wq, ws, w_fq,
-                                                      (cudaStream_t)stream), "lora merge launch");
+                                                      d->sms, (cudaStream_t)stream), "lora merge launch");
 }
 
 fpq_status fpq_scaled_gemm(fpq_format fmt_a, const void* aq, const void* as, fpq_format fmt_b,
@@ -404,6 +404,26 @@ fpq_status fpq_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hidden,
                                                     dst_row0, n_dest, dst_codes, dst_scales, dst_capacity, d->err,
                                                     (cudaStream_t)stream),
                      "moe dispatch launch");
+}
+
+fpq_status fpq_moe_regroup(const void* recv_codes, const void* recv_scales, const int32_t* counts_all,
+                           int32_t world, int32_t num_experts, int32_t rank, int64_t hidden, int64_t rows,
+                           void* codes, void* scales, void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (world < 1 || num_experts < 1 || num_experts > 1024 || num_experts % world || rank < 0 || rank >= world ||
+        hidden < 32 || hidden % 32 || hidden > (1 << 24) || rows < 0 || rows >= (1ll << 31)) {
+        set_detail("need world >= 1 dividing num_experts in [1, 1024], 0 <= rank < world, hidden a positive "
+                   "multiple of 32, 0 <= rows < 2^31");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if (rows == 0) return FPQ_OK;
+    if ((st = check_ptrs({recv_codes, recv_scales, counts_all, codes, scales})) != FPQ_OK) return st;
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    return from_cuda(fpq::launch_moe_regroup(recv_codes, recv_scales, counts_all, world, num_experts, rank, hidden,
+                                             rows, codes, scales, d->err, d->sms, (cudaStream_t)stream),
+                     "moe regroup launch");
 }
 
 size_t fpq_gemm_bf16_splitk_workspace_bytes(int64_t m, int64_t n, int64_t k) {

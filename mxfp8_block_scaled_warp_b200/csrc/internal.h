@@ -30,7 +30,7 @@ cudaError_t launch_dequantize(int fmt, const void* q, const void* scales, const 
 
 cudaError_t launch_lora_merge_fakequant(const void* w, const void* a, const void* b, int64_t n,
                                         int64_t k, int r, float alpha_over_r, void* wq, float* ws,
-                                        void* w_fq, cudaStream_t st);
+                                        void* w_fq, int sms, cudaStream_t st);
 
 // Dense block-scaled GEMMs: C[m,n] = sum_k A[m,k] B[n,k].
 cudaError_t launch_gemm_mxfp8(const void* aq, const void* as, const void* bq, const void* bs,
@@ -72,6 +72,9 @@ cudaError_t launch_moe_route(const int32_t* ids, int64_t tokens, int topk, int e
                              void* workspace, uint32_t* err, cudaStream_t st);
 cudaError_t launch_moe_layout(const int32_t* counts_all, int world, int experts, int rank, int pack,
                               int64_t* dst_row0, int32_t* recv_offsets, cudaStream_t st);
+cudaError_t launch_moe_regroup(const void* src_q, const void* src_s, const int32_t* counts_all, int world,
+                               int experts, int rank, int64_t hidden, int64_t rows, void* dst_q, void* dst_s,
+                               uint32_t* err, int sms, cudaStream_t st);
 cudaError_t launch_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hidden, const int32_t* ids, int topk,
                                       int experts, const void* workspace, const int64_t* dst_row0, int n_dest,
                                       void* const* dst_codes, void* const* dst_scales, const int64_t* dst_capacity,

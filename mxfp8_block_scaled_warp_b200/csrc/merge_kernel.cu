@@ -173,7 +173,8 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
 
 cudaError_t launch_lora_merge_fakequant(const void* w, const void* a, const void* b, int64_t n,
                                         int64_t k, int r, float alpha_over_r, void* wq, float* ws,
-                                        void* w_fq, cudaStream_t st) {
+                                        void* w_fq, int sms, cudaStream_t st) {
+    (void)sms;
     if (r < 1 || r > kMaxRank) return cudaErrorInvalidValue;
     const size_t smem = sizeof(float) * 2 * 128 * (size_t)r;
     if (smem > 48 * 1024) {

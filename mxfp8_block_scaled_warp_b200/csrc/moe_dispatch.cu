@@ -229,6 +229,81 @@ moe_dispatch_mxfp8_kernel(const uint4* __restrict__ x, int64_t tokens, int64_t h
     }
 }
 
+// Regroup (the receiving side of a rank-to-rank exchange): rows that
+// arrived source-major -- all of source 0's rows for this rank's experts,
+// expert-major in slot order, then source 1's, ... -- into the receive
+// layout (expert-major; within an expert, source 0, 1, ...).  Segment
+// (l, s) of C[s][rank L + l] rows moves from
+//   src = sum_{s' < s, l'} C[s'][rank L + l'] + sum_{l' < l} C[s][rank L + l']
+// to
+//   dst = sum_{l' < l, s'} C[s'][rank L + l'] + sum_{s' < s} C[s'][rank L + l].
+// One column of CTAs per segment (blockIdx.y = l world + s), warp 0 works out
+// the segment's rows and starts; then each warp copies one row at a time
+// (codes, then its E8M0 scales) with 16-byte vectors.  Negative counts or a
+// segment outside `rows` are reported and not copied.
+__global__ void __launch_bounds__(32 * kWarps)
+moe_regroup_kernel(const uint8_t* __restrict__ src_q, const uint8_t* __restrict__ src_s,
+                   const int32_t* __restrict__ counts_all, int world, int experts, int rank, int64_t hidden,
+                   int64_t rows, uint8_t* __restrict__ dst_q, uint8_t* __restrict__ dst_s, uint32_t* err) {
+    __shared__ int64_t seg[3];      // rows, src start, dst start (-1 rows: malformed)
+    const int L = experts / world;
+    const int l = (int)blockIdx.y / world, s = (int)blockIdx.y - l * world;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int32_t* c = counts_all;
+    const int e0 = rank * L;
+    if (warp == 0) {
+        int64_t src = 0, dst = 0;
+        bool bad = false;
+        for (int i = lane; i < s * L; i += 32) {           // sources before s, all local experts
+            const int32_t v = c[(int64_t)(i / L) * experts + e0 + i % L];
+            bad |= v < 0;
+            src += v;
+        }
+        for (int i = lane; i < l; i += 32) src += c[(int64_t)s * experts + e0 + i];
+        for (int i = lane; i < l * world; i += 32) {       // local experts before l, all sources
+            const int32_t v = c[(int64_t)(i % world) * experts + e0 + i / world];
+            bad |= v < 0;
+            dst += v;
+        }
+        for (int i = lane; i < s; i += 32) dst += c[(int64_t)i * experts + e0 + l];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            src += __shfl_xor_sync(0xFFFFFFFFu, src, o);
+            dst += __shfl_xor_sync(0xFFFFFFFFu, dst, o);
+        }
+        bad = __any_sync(0xFFFFFFFFu, bad);
+        if (lane == 0) {
+            const int64_t n = c[(int64_t)s * experts + e0 + l];
+            if (bad || n < 0 || src + n > rows || dst + n > rows) {
+                if (blockIdx.x == 0) raise_device_error(err, FPQ_ERR_DEVICE_BAD_INPUT);
+                seg[0] = -1;
+            } else {
+                seg[0] = n;
+            }
+            seg[1] = src;
+            seg[2] = dst;
+        }
+    }
+    __syncthreads();
+    const int64_t n = seg[0], src = seg[1], dst = seg[2];
+    if (n <= 0) return;
+    const int64_t sbytes = hidden / 32;
+    const bool svec = (sbytes % 16) == 0;
+    for (int64_t r = (int64_t)blockIdx.x * kWarps + warp; r < n; r += (int64_t)gridDim.x * kWarps) {
+        const uint4* qs = reinterpret_cast<const uint4*>(src_q + (src + r) * hidden);
+        uint4* qd = reinterpret_cast<uint4*>(dst_q + (dst + r) * hidden);
+        for (int64_t v = lane; v < hidden / 16; v += 32) st_v4(qd + v, ld_stream(qs + v));
+        const uint8_t* ss = src_s + (src + r) * sbytes;
+        uint8_t* sd = dst_s + (dst + r) * sbytes;
+        if (svec) {
+            for (int64_t v = lane; v < sbytes / 16; v += 32)
+                *reinterpret_cast<uint4*>(sd + 16 * v) = *reinterpret_cast<const uint4*>(ss + 16 * v);
+        } else {
+            for (int64_t v = lane; v < sbytes; v += 32) sd[v] = ss[v];
+        }
+    }
+}
+
 }  // namespace
 
 int64_t moe_tokens_per_chunk(int64_t tokens) { return max64(1, (tokens + 4735) / 4736); }
@@ -275,6 +350,17 @@ cudaError_t launch_moe_dispatch_mxfp8(const void* x, int64_t tokens, int64_t hid
     return launch_pdl(moe_dispatch_mxfp8_kernel, dim3((unsigned)((chunks + kWarps - 1) / kWarps)), dim3(32 * kWarps),
                       smem, st, (const uint4*)x, tokens, hidden, ids, topk, experts, base, tpc, chunks, dst_row0,
                       experts / n_dest, (uint8_t* const*)dst_codes, (uint8_t* const*)dst_scales, dst_capacity, err);
+}
+
+cudaError_t launch_moe_regroup(const void* src_q, const void* src_s, const int32_t* counts_all, int world,
+                               int experts, int rank, int64_t hidden, int64_t rows, void* dst_q, void* dst_s,
+                               uint32_t* err, int sms, cudaStream_t st) {
+    // about four CTAs per SM over all segments (experts / world * world = experts of them)
+    const int gx = (int)max64(1, min64(65535, (int64_t)4 * (sms > 0 ? sms : 1) / experts));
+    moe_regroup_kernel<<<dim3((unsigned)gx, (unsigned)experts), 32 * kWarps, 0, st>>>(
+        (const uint8_t*)src_q, (const uint8_t*)src_s, counts_all, world, experts, rank, hidden, rows,
+        (uint8_t*)dst_q, (uint8_t*)dst_s, err);
+    return cudaGetLastError();
 }
 
 }  // namespace fpq

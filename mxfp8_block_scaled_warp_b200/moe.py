@@ -11,11 +11,13 @@ from one source, its (token, choice) pairs in token order, then choice order.
 
 One rank (or no process group): the fused kernel writes the rows straight
 into the grouped buffer.  Several ranks: the per-expert counts are
-all-gathered, the kernel writes an expert-major send buffer, and one
-point-to-point transfer per (expert, peer) segment (NCCL over NVLink; no TMA
-of any kind touches a peer's memory) lands each segment at its row in the
-receiver's buffer.  Every step of the computation runs in the library's
-kernels; this module allocates buffers and moves segments.
+all-gathered, the kernel writes an expert-major send buffer (the rows bound
+for rank p, experts [p L, (p + 1) L), are one contiguous run), one
+all-to-all per tensor (codes, scales) with per-rank row counts moves every
+run to its rank (NCCL over NVLink; no TMA of any kind touches a peer's
+memory), and a kernel regroups the rows that arrived source-major into the
+expert-then-source order.  Every step of the computation runs in the
+library's kernels; this module allocates buffers and issues the collectives.
 """
 from __future__ import annotations
 
@@ -24,10 +26,10 @@ from typing import NamedTuple
 import torch
 import torch.distributed as dist
 
-from . import (MOE_DIRECT, MOE_PACK, fpq_moe_dispatch_layout, fpq_moe_dispatch_mxfp8, fpq_moe_route,
-               fpq_moe_route_workspace_bytes)
+from . import (MOE_DIRECT, MOE_PACK, fpq_moe_dispatch_layout, fpq_moe_dispatch_mxfp8, fpq_moe_regroup,
+               fpq_moe_route, fpq_moe_route_workspace_bytes)
 
-__all__ = ["Dispatched", "route", "dispatch", "segment_plan", "exchange_rows"]
+__all__ = ["Dispatched", "route", "dispatch", "split_sizes", "exchange_rows"]
 
 
 class Dispatched(NamedTuple):
@@ -49,14 +51,30 @@ def route(topk_ids: torch.Tensor, num_experts: int, stream=None):
     return counts, ws
 
 
+_PTR_TABLES: dict = {}        # device pointer tables of destination buffer sets, by address
+
+
+def _ptr_tables(buffers, dev):
+    """Device arrays of the buffers' code and scale addresses and row
+    capacities, built once per buffer set (a fresh set of addresses makes a
+    new entry; a few recent sets are kept)."""
+    key = (dev.index, tuple((c.data_ptr(), s.data_ptr(), c.shape[0]) for c, s in buffers))
+    t = _PTR_TABLES.get(key)
+    if t is None:
+        if len(_PTR_TABLES) >= 16:
+            _PTR_TABLES.pop(next(iter(_PTR_TABLES)))
+        t = (torch.tensor([c.data_ptr() for c, _ in buffers], dtype=torch.int64, device=dev),
+             torch.tensor([s.data_ptr() for _, s in buffers], dtype=torch.int64, device=dev),
+             torch.tensor([c.shape[0] for c, _ in buffers], dtype=torch.int64, device=dev))
+        _PTR_TABLES[key] = t
+    return t
+
+
 def _dispatch_into(x, topk_ids, num_experts, ws, dst_row0, buffers, stream=None):
     """Quantize + write every pair's row into `buffers` [(codes, scales)],
     expert e to buffers[e // (E / len(buffers))]."""
     tokens, topk = topk_ids.shape
-    dev = x.device
-    codes_p = torch.tensor([c.data_ptr() for c, _ in buffers], dtype=torch.int64, device=dev)
-    scales_p = torch.tensor([s.data_ptr() for _, s in buffers], dtype=torch.int64, device=dev)
-    cap = torch.tensor([c.shape[0] for c, _ in buffers], dtype=torch.int64, device=dev)
+    codes_p, scales_p, cap = _ptr_tables(buffers, x.device)
     fpq_moe_dispatch_mxfp8(x, tokens, x.shape[1], topk_ids, topk, num_experts, ws, dst_row0, len(buffers),
                            codes_p, scales_p, cap, stream)
 
@@ -92,65 +110,45 @@ def dispatch(x: torch.Tensor, topk_ids: torch.Tensor, num_experts: int, group=No
     rows = tokens * topk_ids.shape[1]
     send_q, send_s = torch.empty((rows, hidden), **u8), torch.empty((rows, hidden // 32), **u8)
     _dispatch_into(x, topk_ids, num_experts, ws, dst_row0, [(send_q, send_s)], stream)
-    counts_host = counts_all.cpu()           # segment sizes for the transfers (waits for the counts)
-    codes, scales = exchange_rows(send_q, send_s, counts_host, rank, world, num_experts, group)
+    counts_host = counts_all.cpu()           # row counts of the all-to-all (waits for the counts)
+    codes, scales = exchange_rows(send_q, send_s, counts_host, rank, world, num_experts, group,
+                                  counts_dev=counts_all, stream=stream)
     return Dispatched(codes, scales, offsets, counts_all)
 
 
-def segment_plan(counts_all, rank: int, world: int, num_experts: int):
-    """Host-side row arithmetic of the exchange, from the all-gathered counts
-    (int [world, E]): the send segments of this rank ([(peer, expert, first
-    row in the expert-major send buffer, rows)]), the receive segments
-    ([(source, expert, first row in this rank's grouped buffer, rows)]) and
-    this rank's receive row count."""
+def split_sizes(counts_all, rank: int, world: int, num_experts: int):
+    """Host-side row counts of the all-to-all, from the all-gathered counts
+    (int [world, E]): rows this rank sends to each rank (its experts' runs
+    of the expert-major send buffer) and rows it receives from each rank."""
     c = [[int(v) for v in row] for row in counts_all.tolist()] if hasattr(counts_all, "tolist") else counts_all
     L = num_experts // world
-    sends, row = [], 0
-    for e in range(num_experts):
-        if c[rank][e]:
-            sends.append((e // L, e, row, c[rank][e]))
-        row += c[rank][e]
-    recvs, row = [], 0
-    for e in range(rank * L, (rank + 1) * L):
-        for s in range(world):
-            if c[s][e]:
-                recvs.append((s, e, row, c[s][e]))
-            row += c[s][e]
-    return sends, recvs, row
+    send = [sum(c[rank][p * L:(p + 1) * L]) for p in range(world)]
+    recv = [sum(c[s][rank * L:(rank + 1) * L]) for s in range(world)]
+    return send, recv
 
 
-def exchange_rows(send_codes, send_scales, counts_all, rank: int, world: int, num_experts: int, group=None):
-    """Move every (expert, source) segment of the expert-major send buffers to
-    the expert's rank, at its row in that rank's grouped buffer.  Segments
-    for this rank are copied locally; the others go as one send and one
-    receive per segment and tensor, matched by (source, expert) order on both
-    sides.  Works on any backend with point-to-point support (NCCL on GPUs,
-    gloo on CPU tensors)."""
-    sends, recvs, rows = segment_plan(counts_all, rank, world, num_experts)
+def exchange_rows(send_codes, send_scales, counts_all, rank: int, world: int, num_experts: int, group=None,
+                  counts_dev=None, regroup=None, stream=None):
+    """Move this rank's expert-major send rows to the experts' ranks: one
+    all-to-all per tensor (each rank's run of rows to that rank), then the
+    regroup of the rows received source-major into this rank's grouped
+    buffer (expert-major; within an expert, source 0, 1, ...).
+    `counts_all` (host, int [world, E]) gives the row counts; `counts_dev`
+    is the same table on the device, read by the regroup kernel.  `regroup`
+    replaces the device regroup step (same arguments as fpq_moe_regroup;
+    used by CPU tests of the collective plumbing).  Works on any backend
+    with all-to-all support (NCCL on GPUs, gloo on CPU tensors)."""
+    send, recv = split_sizes(counts_all, rank, world, num_experts)
     hidden = send_codes.shape[1]
-    codes = torch.empty((rows, hidden), dtype=torch.uint8, device=send_codes.device)
-    scales = torch.empty((rows, send_scales.shape[1]), dtype=torch.uint8, device=send_codes.device)
-    ops = []
-    local = {}
-    for peer, e, r0, n in sends:
-        if peer == rank:
-            local[e] = (r0, n)
-            continue
-        ops.append(dist.P2POp(dist.isend, send_codes[r0:r0 + n], dist.get_global_rank(group, peer)
-                              if group is not None else peer, group))
-        ops.append(dist.P2POp(dist.isend, send_scales[r0:r0 + n], dist.get_global_rank(group, peer)
-                              if group is not None else peer, group))
-    for src, e, r0, n in recvs:
-        if src == rank:
-            s0, _ = local[e]
-            codes[r0:r0 + n].copy_(send_codes[s0:s0 + n])
-            scales[r0:r0 + n].copy_(send_scales[s0:s0 + n])
-            continue
-        ops.append(dist.P2POp(dist.irecv, codes[r0:r0 + n], dist.get_global_rank(group, src)
-                              if group is not None else src, group))
-        ops.append(dist.P2POp(dist.irecv, scales[r0:r0 + n], dist.get_global_rank(group, src)
-                              if group is not None else src, group))
-    if ops:
-        for w in dist.batch_isend_irecv(ops):
-            w.wait()
+    rows = sum(recv)
+    dev = send_codes.device
+    recv_q = torch.empty((rows, hidden), dtype=torch.uint8, device=dev)
+    recv_s = torch.empty((rows, send_scales.shape[1]), dtype=torch.uint8, device=dev)
+    sent = sum(send)
+    dist.all_to_all_single(recv_q, send_codes[:sent], recv, send, group=group)
+    dist.all_to_all_single(recv_s, send_scales[:sent], recv, send, group=group)
+    codes = torch.empty_like(recv_q)
+    scales = torch.empty_like(recv_s)
+    (regroup or fpq_moe_regroup)(recv_q, recv_s, counts_dev, world, num_experts, rank, hidden, rows, codes, scales,
+                                 stream)
     return codes, scales

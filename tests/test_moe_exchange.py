@@ -1,10 +1,11 @@
 """Multi-rank plumbing of the MoE FP8 dispatch on CPU (gloo, world sizes 2
-and 3): the counts all-gather, the segment arithmetic and the point-to-point
+and 3): the counts all-gather, the all-to-all row counts and the all-to-all
 exchange of ``mxfp8_block_scaled_warp_b200.moe``, with each rank's
-expert-major send buffer built by the oracle (the CUDA kernels that build it
-on a GPU are checked against the same oracle in the GPU tests).  The
+expert-major send buffer built by the oracle and the device regroup step
+stood in for by its definition (``regroup_standin``; the CUDA kernels that
+do both on a GPU are checked against the oracle in the GPU tests).  The
 received buffers must equal the oracle's dispatch over all ranks, byte for
-byte, and the segment plan must give the oracle's group offsets."""
+byte."""
 import os
 import socket
 import sys
@@ -35,6 +36,27 @@ def _inputs(world):
     return xs, ids
 
 
+def regroup_standin(recv_q, recv_s, counts_dev, world, experts, rank, hidden, rows, codes, scales, stream=None):
+    """fpq_moe_regroup by its definition: rows that arrived source-major
+    (source 0's rows for this rank's experts, expert-major, then source 1's,
+    ...) into expert-major order, sources in order within an expert."""
+    c = np.asarray(counts_dev, np.int64)
+    L = experts // world
+    start, a = {}, 0
+    for s in range(world):
+        for l in range(L):
+            start[(l, s)] = a
+            a += int(c[s][rank * L + l])
+    d = 0
+    for l in range(L):
+        for s in range(world):
+            n = int(c[s][rank * L + l])
+            codes[d:d + n] = recv_q[start[(l, s)]:start[(l, s)] + n]
+            scales[d:d + n] = recv_s[start[(l, s)]:start[(l, s)] + n]
+            d += n
+    assert d == rows
+
+
 def _worker(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
@@ -51,9 +73,8 @@ def _worker(rank, world, port, q):
         counts_all = torch.stack(parts)
         send_q, send_s, _ = oracle.moe_dispatch([xs[rank]], [ids[rank]], EXPERTS)[0]   # expert-major pack
         codes, scales = moe.exchange_rows(torch.from_numpy(send_q), torch.from_numpy(send_s), counts_all, rank,
-                                          world, EXPERTS, None)
-        _, recvs, rows = moe.segment_plan(counts_all, rank, world, EXPERTS)
-        q.put((rank, codes.numpy(), scales.numpy(), rows, recvs))
+                                          world, EXPERTS, None, counts_dev=counts_all, regroup=regroup_standin)
+        q.put((rank, codes.numpy(), scales.numpy()))
     finally:
         dist.destroy_process_group()
 
@@ -68,8 +89,8 @@ def test_exchange_matches_oracle_dispatch(world):
         p.start()
     got = {}
     for _ in range(world):
-        rank, codes, scales, rows, recvs = q.get(timeout=180)
-        got[rank] = (codes, scales, rows, recvs)
+        rank, codes, scales = q.get(timeout=180)
+        got[rank] = (codes, scales)
     for p in procs:
         p.join(60)
         assert p.exitcode == 0
@@ -77,33 +98,18 @@ def test_exchange_matches_oracle_dispatch(world):
     import oracle
     xs, ids = _inputs(world)
     want = oracle.moe_dispatch(xs, ids, EXPERTS)
-    L = EXPERTS // world
     for r in range(world):
-        codes, scales, rows, recvs = got[r]
+        codes, scales = got[r]
         wq, ws, woff = want[r]
-        assert rows == woff[-1]
+        assert codes.shape[0] == woff[-1]
         assert np.array_equal(codes, wq) and np.array_equal(scales, ws)
-        # the first receive segment of each local expert starts at its group offset
-        for l in range(L):
-            segs = [seg for seg in recvs if seg[1] == r * L + l]
-            if segs:
-                assert segs[0][2] == woff[l]
-
-
-def test_segment_plan_single_rank():
-    sys.path.insert(0, ROOT)
-    from mxfp8_block_scaled_warp_b200 import moe
-    counts_all = torch.tensor([[2, 0, 3]], dtype=torch.int32)
-    sends, recvs, rows = moe.segment_plan(counts_all, 0, 1, 3)
-    assert sends == [(0, 0, 0, 2), (0, 2, 2, 3)]
-    assert recvs == [(0, 0, 0, 2), (0, 2, 2, 3)]
-    assert rows == 5
 
 
 def _dispatch_worker(rank, world, port, q):
-    """moe.dispatch on gloo ranks with its three device steps (route, layout,
-    the quantize + pack kernel) stood in for by the oracle's definitions; the
-    counts all-gather, the segment plan and the transfers run as written."""
+    """moe.dispatch on gloo ranks with its four device steps (route, layout,
+    the quantize + pack kernel, the regroup) stood in for by their
+    definitions; the counts all-gather, the row counts and the all-to-all
+    transfers run as written."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -130,6 +136,7 @@ def _dispatch_worker(rank, world, port, q):
         buffers[0][1].copy_(torch.from_numpy(s))
 
     moe.route, moe.fpq_moe_dispatch_layout, moe._dispatch_into = fake_route, fake_layout, fake_pack
+    moe.fpq_moe_regroup = regroup_standin
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         xs, ids = _inputs(world)

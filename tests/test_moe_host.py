@@ -23,7 +23,10 @@ def test_dispatch_rejects_bad_inputs_before_device_work():
 
 
 @pytest.mark.parametrize("world,experts", [(1, 5), (2, 8), (4, 8), (4, 16)])
-def test_segment_plan_matches_oracle_layout(world, experts):
+def test_split_sizes_match_oracle_layout(world, experts):
+    """The all-to-all's row counts: what rank r sends to rank p is the run of
+    p's experts in r's expert-major pack, and what r receives from all
+    sources adds up to the oracle's grouped buffer."""
     rng = np.random.default_rng(world * 100 + experts)
     k, hidden = 2, 32
     xs, ids = [], []
@@ -35,29 +38,19 @@ def test_segment_plan_matches_oracle_layout(world, experts):
     counts_all = np.stack([oracle.moe_route_plan(i, experts)[0] for i in ids])
     want = oracle.moe_dispatch(xs, ids, experts)
     L = experts // world
+    sends = {}
     for r in range(world):
-        sends, recvs, rows = moe.segment_plan(torch.from_numpy(counts_all), r, world, experts)
-        assert rows == want[r][2][-1]
-        # receive segments tile [0, rows) in (local expert, source) order
-        pos = 0
-        for src, e, r0, n in recvs:
-            assert r0 == pos and n == counts_all[src][e] and e // L == r
-            pos += n
-        assert pos == rows
-        # the first segment of each local expert starts at its group offset
-        for l in range(L):
-            segs = [seg for seg in recvs if seg[1] == r * L + l]
-            if segs:
-                assert segs[0][2] == want[r][2][l]
-        # send segments tile this rank's expert-major pack
-        pos = 0
-        for peer, e, r0, n in sends:
-            assert r0 == sum(counts_all[r][:e]) and n == counts_all[r][e] and peer == e // L
-        assert sum(n for *_, n in sends) == counts_all[r].sum()
+        send, recv = moe.split_sizes(torch.from_numpy(counts_all), r, world, experts)
+        sends[r] = send
+        assert sum(recv) == want[r][2][-1]
+        assert sum(send) == counts_all[r].sum()
+        for p in range(world):
+            assert send[p] == counts_all[r][p * L:(p + 1) * L].sum()
+    for r in range(world):                                        # the two sides of every transfer agree
+        _, recv = moe.split_sizes(torch.from_numpy(counts_all), r, world, experts)
+        assert recv == [sends[s][r] for s in range(world)]
 
 
-def test_segment_plan_accepts_nested_lists():
-    sends, recvs, rows = moe.segment_plan([[1, 0, 2, 3], [0, 4, 0, 1]], 1, 2, 4)
-    assert rows == 2 + 0 + 3 + 1                                  # experts 2 and 3, both sources
-    assert sends == [(0, 1, 0, 4), (1, 3, 4, 1)]
-    assert recvs == [(0, 2, 0, 2), (0, 3, 2, 3), (1, 3, 5, 1)]
+def test_split_sizes_accept_nested_lists():
+    send, recv = moe.split_sizes([[1, 0, 2, 3], [0, 4, 0, 1]], 1, 2, 4)
+    assert send == [4, 1] and recv == [5, 1]

@@ -197,3 +197,52 @@ def test_rejects_bad_args(fpq):
         p = torch.zeros(1, dtype=torch.int64, device="cuda")
         fpq.fpq_moe_dispatch_mxfp8(x, 4, 48, t, 2, 8, ws, torch.zeros(8, dtype=torch.int64, device="cuda"), 1, p, p,
                                    p)
+
+
+@pytest.mark.parametrize("world,experts,k,hidden", [(2, 8, 2, 256), (3, 12, 3, 96), (8, 64, 8, 7168),
+                                                    (4, 16, 4, 2048)])
+def test_pack_exchange_regroup(fpq, orc, world, experts, k, hidden):
+    """The several-rank path end to end on one GPU: every source's PACK send
+    buffer (the kernels), the all-to-all stood in for by moving each
+    source's run of rows for rank r into r's receive buffer in source order,
+    then fpq_moe_regroup: each rank's grouped buffer equals the oracle's
+    dispatch over all ranks byte for byte.  Some sources hold no tokens."""
+    L = experts // world
+    tokens = [0 if s == 1 else 20 + 13 * s for s in range(world)]
+    xs = [_x(t, hidden, 900 + s) for s, t in enumerate(tokens)]
+    ids = [_ids(t, experts, k, 910 + s) for s, t in enumerate(tokens)]
+    srcs = [Source(fpq, xs[s], ids[s], experts) for s in range(world)]
+    counts_all = torch.stack([s.counts for s in srcs]).contiguous()
+    c = counts_all.cpu().numpy().astype(np.int64)
+    packs = []
+    for s in range(world):
+        buf = _buffers(max(1, tokens[s] * k), hidden)
+        srcs[s].dispatch(counts_all, world, s, fpq.MOE_PACK, [buf])
+        packs.append(buf)
+    want = orc.moe_dispatch([workloads.as_u16(x) for x in xs], [i.numpy() for i in ids], experts)
+    for r in range(world):
+        runs_q, runs_s = [], []
+        for s in range(world):
+            a = int(c[s][:r * L].sum())
+            n = int(c[s][r * L:(r + 1) * L].sum())
+            runs_q.append(packs[s][0][a:a + n])
+            runs_s.append(packs[s][1][a:a + n])
+        recv_q, recv_s = torch.cat(runs_q).contiguous(), torch.cat(runs_s).contiguous()
+        rows = recv_q.shape[0]
+        assert rows == want[r][2][-1]
+        out = _buffers(max(1, rows), hidden)
+        fpq.fpq_moe_regroup(recv_q, recv_s, counts_all, world, experts, r, hidden, rows, out[0], out[1])
+        assert np.array_equal(out[0][:rows].cpu().numpy(), want[r][0])
+        assert np.array_equal(out[1][:rows].cpu().numpy(), want[r][1])
+    assert fpq.fpq_get_device_error() == 0
+
+
+def test_regroup_malformed_counts_reported(fpq):
+    """Counts that place a segment past the buffer: FPQ_ERR_DEVICE_BAD_INPUT,
+    and the segment is not copied."""
+    counts = torch.tensor([[3, 2], [4, 50]], dtype=torch.int32, device="cuda")      # world 2, E 2, rank 1: 52 rows
+    recv_q, recv_s = _buffers(10, 64)
+    out_q, out_s = _buffers(10, 64)
+    fpq.fpq_moe_regroup(recv_q, recv_s, counts, 2, 2, 1, 64, 10, out_q, out_s)
+    assert fpq.fpq_get_device_error() == BAD_INPUT
+    assert (out_q[2:] == 0xEE).all()                 # rows of the oversize segment untouched
