@@ -488,9 +488,10 @@ class QatBackward(Step):
     """The backward of the QAT linear layer (straight-through estimator) at
     the QAT workload's shape: x 8192x7168, W 2048x7168, LoRA r = 16, alpha/r
     = 2; dx, dW_eff, dA, dB in bf16 on the bf16 tensor-core GEMM, each
-    operand read in its stored layout, dA and dB split over the contraction.
-    The same launches as fpq_qat_backward, issued through the C ABI one by
-    one so that each product is timed (dA and dB with their reductions)."""
+    operand read in its stored layout; dA and dB from one pass over dW (each
+    dW tile feeds both products) plus an ordered reduction of the partial
+    sums.  The same launches as fpq_qat_backward, issued through the C ABI
+    one by one so that each product is timed."""
     name = "qat_backward"
     dominant = "gemm_bf16_dx"
     CONFIG = {"workload": "qat_backward: dy 8192x2048 N(0,1); x_fq = 1x128 fake-quant of x 8192x7168 "
@@ -521,14 +522,13 @@ class QatBackward(Step):
         wsb = fpq.fpq_qat_backward_workspace_bytes(m, n, k, r)
         self.ws = torch.empty(((wsb + 15) // 16 * 16,), dtype=torch.uint8, device=dev) if wsb else None
         u8 = dict(dtype=torch.uint8, device=dev)
-        self.ws_a = torch.empty((fpq.fpq_gemm_bf16_splitk_workspace_bytes(r, k, n),), **u8)
-        self.ws_b = torch.empty((fpq.fpq_gemm_bf16_splitk_workspace_bytes(n, r, k),), **u8)
+        self.ws_g = torch.empty((fpq.fpq_qat_lora_grads_workspace_bytes(n, k, r),), **u8)
         self.dx_host = torch.empty((m, k), dtype=torch.bfloat16).pin_memory()
         self.da_host = torch.empty((r, k), dtype=torch.bfloat16).pin_memory()
         self.db_host = torch.empty((n, r), dtype=torch.bfloat16).pin_memory()
         self.flops = 2.0 * (2 * m * n * k + 2 * r * n * k)
         self.quant_bytes = 0.0          # no quantize kernel in this step
-        self.launches = 6                # dA and dB: split-K GEMM + slice reduction each
+        self.launches = 4                # dA and dB: one fused pass over dW + the partial-sum reduction
         self.config = dict(self.CONFIG)
 
     def kernels(self):
@@ -536,8 +536,8 @@ class QatBackward(Step):
         return [
             ("gemm_bf16_dx", lambda: f.fpq_gemm_bf16_layout(self.dy, 0, self.w_fq, 1, m, k, n, 1.0, self.dx)),
             ("gemm_bf16_dw", lambda: f.fpq_gemm_bf16_layout(self.dy, 1, self.x_fq, 1, n, k, m, 1.0, self.dw)),
-            ("gemm_bf16_da", lambda: f.fpq_gemm_bf16_splitk(self.b, 1, self.dw, 1, r, k, n, aor, self.da, self.ws_a)),
-            ("gemm_bf16_db", lambda: f.fpq_gemm_bf16_splitk(self.dw, 0, self.a, 0, n, r, k, aor, self.db, self.ws_b)),
+            ("lora_grads", lambda: f.fpq_qat_lora_grads(self.dw, self.a, self.b, n, k, r, aor, self.da, self.db,
+                                                        self.ws_g)),
         ]
 
     def whole_step(self, side_stream):
@@ -549,7 +549,8 @@ class QatBackward(Step):
     def kernel_work(self):
         m, n, k, r = self.m, self.n, self.k, self.r
         return {"gemm_bf16_dx": ("TFLOP/s", 2.0 * m * n * k), "gemm_bf16_dw": ("TFLOP/s", 2.0 * m * n * k),
-                "gemm_bf16_da": ("TFLOP/s", 2.0 * r * n * k), "gemm_bf16_db": ("TFLOP/s", 2.0 * r * n * k)}
+                # HBM-bound: dW, A, B read once, dA and dB written once
+                "lora_grads": ("GB/s", 2.0 * (n * k + r * k + n * r) + 2.0 * (r * k + n * r))}
 
     def e2e_step(self, stream, side_stream):
         """dy from pinned host memory, the public fpq_qat_backward call, dx,
@@ -807,7 +808,7 @@ def _source_hash(kernel: str) -> str | None:
            "gemm_mxfp8": "gemm_mxfp8.cu", "quant_fp8_1x128": "quant_kernels.cu",
            "quant_mxfp8": "quant_kernels.cu", "lora_merge_fq": "merge_kernel.cu",
            "gemm_nvfp4": "gemm_nvfp4.cu", "gemm_bf16_dx": "gemm_bf16.cu",
-           "moe_dispatch_mxfp8": "moe_dispatch.cu"}.get(kernel)
+           "moe_dispatch_mxfp8": "moe_dispatch.cu", "lora_grads": "lora_grads.cu"}.get(kernel)
     if not src:
         return None
     with open(os.path.join(ROOT, "mxfp8_block_scaled_warp_b200", "csrc", src), "rb") as f:

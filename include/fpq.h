@@ -326,9 +326,10 @@ FPQ_API fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, i
  *   da      bf16 [r, k];  db bf16 [n, r]
  *   workspace   fpq_qat_backward_workspace_bytes(m, n, k, r) bytes, 16-byte
  *               aligned, caller-owned, not read before written: fp32 partial
- *               sums of da and db, whose few output tiles split their
- *               contraction across the SMs (at most 16 slices each, added in
- *               slice order by a second kernel, so results are repeatable)
+ *               sums of da and db (for r <= 64 those of fpq_qat_lora_grads,
+ *               sized for the current device's SM count; for larger r the
+ *               split-K slices of two bf16 GEMMs, at most 16 each), added in
+ *               a fixed order by a second kernel, so results are repeatable
  *
  * The products are ordered on `stream` like any other work: dx, which no
  * other product needs, runs on a library-owned second stream forked from
@@ -340,6 +341,31 @@ FPQ_API fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, i
  * FPQ_ERR_ALIGNMENT, FPQ_ERR_WORKSPACE, FPQ_ERR_CUDA; device-side wait
  * timeouts go to the device error word.
  */
+/*
+ * fpq_qat_lora_grads -- the two LoRA gradients of the QAT backward in one
+ * pass over the weight gradient [same source, same numerics as in
+ * fpq_qat_backward]:  da = (alpha/r) B^T dw,  db = (alpha/r) dw A^T, fp32
+ * accumulation, bf16 out.  Each 128 x 128 tile of dw is read once and feeds
+ * both tensor-core products (one CTA per 128-row strip of dw and range of K
+ * tiles); the fp32 partial sums go to the workspace and a second kernel adds
+ * them in a fixed order (repeatable results).
+ *
+ *   dw      bf16 [n, k];  lora_a bf16 [r, k];  lora_b bf16 [n, r]
+ *   da      bf16 [r, k];  db bf16 [n, r]
+ *   workspace   fpq_qat_lora_grads_workspace_bytes(n, k, r) bytes (the
+ *               current device's SM count enters the size), 16-byte aligned,
+ *               caller-owned, not read before written
+ *
+ * Requires n, k positive multiples of 8, r a multiple of 8 in [8, 64], every
+ * pointer 16-byte aligned.  Errors: FPQ_ERR_INVALID_ARG, FPQ_ERR_ALIGNMENT,
+ * FPQ_ERR_WORKSPACE, FPQ_ERR_CUDA; device-side wait timeouts go to the device
+ * error word.
+ */
+FPQ_API size_t fpq_qat_lora_grads_workspace_bytes(int64_t n, int64_t k, int32_t r);
+FPQ_API fpq_status fpq_qat_lora_grads(const void* dw, const void* lora_a, const void* lora_b, int64_t n, int64_t k,
+                                      int32_t r, float alpha_over_r, void* da, void* db, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
 FPQ_API size_t fpq_qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);
 FPQ_API fpq_status fpq_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
                                     const void* lora_b, int64_t m, int64_t n, int64_t k, int32_t r,

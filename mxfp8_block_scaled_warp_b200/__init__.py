@@ -31,7 +31,7 @@ __all__ = [
     "fpq_moe_regroup",
     "fpq_quantize_block_strided", "fpq_dequantize_strided",
     "MOE_DIRECT", "MOE_PACK",
-    "fpq_qat_backward",
+    "fpq_qat_backward", "fpq_qat_lora_grads", "fpq_qat_lora_grads_workspace_bytes",
     "fpq_quantize_nvfp4_noalloc", "NOALLOC_NVFP4_MAX_BATCH",
     "quantize", "dequantize", "lora_merge_fakequant", "scaled_gemm", "scaled_gemm_nvfp4", "grouped_scaled_gemm",
     "scale_shape", "code_shape", "gemm_bf16", "qat_backward",
@@ -88,6 +88,8 @@ def _load() -> ctypes.CDLL:
         "fpq_gemm_bf16_splitk_workspace_bytes": (SZ, [I64, I64, I64]),
         "fpq_gemm_bf16_splitk": (I32, [P, I32, P, I32, I64, I64, I64, F, P, P, SZ, P]),
         "fpq_qat_backward_workspace_bytes": (SZ, [I64, I64, I64, I32]),
+        "fpq_qat_lora_grads_workspace_bytes": (SZ, [I64, I64, I32]),
+        "fpq_qat_lora_grads": (I32, [P, P, P, I64, I64, I32, F, P, P, P, SZ, P]),
         "fpq_moe_route_workspace_bytes": (SZ, [I64, I32]),
         "fpq_quantize_block_strided": (I32, [I32, P, I64, I64, I64, I64, I64, P, I64, I64, P, P, P, SZ, P]),
         "fpq_dequantize_strided": (I32, [I32, P, I64, I64, P, P, I64, I64, I64, P, I64, I64, P]),
@@ -251,6 +253,17 @@ def fpq_moe_regroup(recv_codes, recv_scales, counts_all, world, num_experts, ran
 
 def fpq_transpose_bf16(x, out, rows, cols, stream=None):
     _check(load().fpq_transpose_bf16(_ptr(x), _ptr(out), rows, cols, _stream(stream)), "fpq_transpose_bf16")
+
+
+def fpq_qat_lora_grads_workspace_bytes(n: int, k: int, r: int) -> int:
+    return load().fpq_qat_lora_grads_workspace_bytes(n, k, r)
+
+
+def fpq_qat_lora_grads(dw, lora_a, lora_b, n, k, r, alpha_over_r, da, db, workspace, stream=None):
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().fpq_qat_lora_grads(_ptr(dw), _ptr(lora_a), _ptr(lora_b), n, k, r, alpha_over_r, _ptr(da), _ptr(db),
+                                     _ptr(workspace) if workspace is not None else None, wsb, _stream(stream)),
+           "fpq_qat_lora_grads")
 
 
 def fpq_qat_backward_workspace_bytes(m: int, n: int, k: int, r: int) -> int:

@@ -468,6 +468,33 @@ fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, int64_t c
     return from_cuda(fpq::launch_transpose_bf16(in, out, rows, cols, (cudaStream_t)stream), "transpose launch");
 }
 
+size_t fpq_qat_lora_grads_workspace_bytes(int64_t n, int64_t k, int32_t r) {
+    if (n < 8 || k < 8 || r < 8 || r % 8 || !fpq::lora_grads_fused(r)) return 0;
+    return fpq::lora_grads_workspace_bytes(n, k, r, fpq::current_sms());
+}
+
+fpq_status fpq_qat_lora_grads(const void* dw, const void* lora_a, const void* lora_b, int64_t n, int64_t k, int32_t r,
+                              float alpha_over_r, void* da, void* db, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    t_detail[0] = 0;
+    fpq_status st;
+    if (n < 8 || n % 8 || k < 8 || k % 8 || r < 8 || r % 8 || r > 64 || n > (1 << 30) || k > (1 << 30)) {
+        set_detail("need n, k positive multiples of 8 and r a multiple of 8 in [8, 64]");
+        return FPQ_ERR_INVALID_ARG;
+    }
+    if ((st = check_ptrs({dw, lora_a, lora_b, da, db})) != FPQ_OK) return st;
+    const DeviceState* d = device_state(&st);
+    if (!d) return st;
+    const size_t need = fpq::lora_grads_workspace_bytes(n, k, r, d->sms);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) {
+        set_detail("need a 16-byte aligned workspace of fpq_qat_lora_grads_workspace_bytes() bytes");
+        return FPQ_ERR_WORKSPACE;
+    }
+    return from_cuda(fpq::launch_lora_grads(dw, lora_a, lora_b, n, k, r, alpha_over_r, da, db, workspace, d->err,
+                                            d->sms, (cudaStream_t)stream),
+                     "lora gradients launch");
+}
+
 size_t fpq_qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) {
     if (m < 1 || n < 1 || k < 1 || r < 1) return 0;
     return fpq::qat_backward_workspace_bytes(m, n, k, r);

@@ -133,6 +133,80 @@ __device__ __forceinline__ uint32_t e4m3x2_of_quotients(float x0, float x1, cons
     return lo;
 }
 
+// Packed pairs of fp32 values in one 64-bit register (element 0 in the low
+// half) for the paired fp32 instructions of sm_100: each lane of
+// fma.rn.f32x2 / mul.rn.f32x2 is one IEEE round-to-nearest fma / multiply,
+// exactly as the scalar instruction.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float lo_of(uint64_t p) { return __uint_as_float((uint32_t)p); }
+__device__ __forceinline__ float hi_of(uint64_t p) { return __uint_as_float((uint32_t)(p >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// The two fp32 values of a bf16x2 word (exact), as a pair.
+__device__ __forceinline__ uint64_t bf16x2_pair(uint32_t w) { return pack2(bf16_lo(w), bf16_hi(w)); }
+
+// Eight E2M1 codes (bits 4i .. 4i + 3 = element i) of four pairs of fp32
+// values, round to nearest even, saturating to +-6.
+__device__ __forceinline__ uint32_t e2m1x8_of_pairs(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(lo_of(p0)), "f"(hi_of(p0)), "f"(lo_of(p1)), "f"(hi_of(p1)), "f"(lo_of(p2)), "f"(hi_of(p2)),
+          "f"(lo_of(p3)), "f"(hi_of(p3)));
+    return r;
+}
+
+// Four E4M3 codes (byte i = element i) of two pairs of fp32 values, round
+// to nearest even, finite values saturating to +-448.
+__device__ __forceinline__ uint32_t e4m3x4_of_pairs(uint64_t p0, uint64_t p1) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 h0, h1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
+        "mov.b32 %0, {h0, h1};\n\t}"
+        : "=r"(r) : "f"(lo_of(p0)), "f"(hi_of(p0)), "f"(lo_of(p1)), "f"(hi_of(p1)));
+    return r;
+}
+
+// E4M3 codes of fp32(x / s) for the eight bf16 values of four words (byte i
+// of out = element i), from the products with both ends of the quotient
+// bracket (lo2 / hi2: the ends as packed pairs), formed two at a time.
+// Returns false when any element's two ends give different codes (a
+// quotient close to a rounding boundary); `out` is then unusable and the
+// caller encodes these elements from correctly rounded divisions.
+__device__ __forceinline__ bool e4m3x8_bracketed(const uint32_t (&w)[4], uint64_t lo2, uint64_t hi2, uint2& out) {
+    const uint64_t x0 = bf16x2_pair(w[0]), x1 = bf16x2_pair(w[1]), x2 = bf16x2_pair(w[2]), x3 = bf16x2_pair(w[3]);
+    out.x = e4m3x4_of_pairs(mul2(x0, lo2), mul2(x1, lo2));
+    out.y = e4m3x4_of_pairs(mul2(x2, lo2), mul2(x3, lo2));
+    const uint32_t u0 = e4m3x4_of_pairs(mul2(x0, hi2), mul2(x1, hi2));
+    const uint32_t u1 = e4m3x4_of_pairs(mul2(x2, hi2), mul2(x3, hi2));
+    return ((out.x ^ u0) | (out.y ^ u1)) == 0u;
+}
+
+// E4M3 codes of fp32(x / s) for the eight bf16 values of four words, from
+// correctly rounded divisions.
+__device__ __forceinline__ uint2 e4m3x8_divided(const uint32_t (&w)[4], float s) {
+    uint64_t q[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) q[j] = pack2(__fdiv_rn(bf16_lo(w[j]), s), __fdiv_rn(bf16_hi(w[j]), s));
+    return make_uint2(e4m3x4_of_pairs(q[0], q[1]), e4m3x4_of_pairs(q[2], q[3]));
+}
+
 // E2M1 codes of fp32(x0/s) (bits 0-3) and fp32(x1/s) (bits 4-7).
 __device__ __forceinline__ uint32_t e2m1x2_of_quotients(float x0, float x1, const QuotientBracket& b) {
     uint32_t lo = f32x2_to_e2m1x2(__fmul_rn(x0, b.lo), __fmul_rn(x1, b.lo));
@@ -221,6 +295,11 @@ __device__ __forceinline__ uint4 ld_stream_hint(const void* p, uint64_t pol) {
 }
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+// 16-byte store of output that is not read again soon (cache-streaming: the
+// line is evicted first, so it does not displace operands other CTAs reuse).
+__device__ __forceinline__ void st_v4_stream(void* p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 __device__ __forceinline__ void st_v2(void* p, uint2 v) {
     asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(p), "r"(v.x), "r"(v.y) : "memory");

@@ -390,7 +390,9 @@ int smem_bytes() { return (int)sizeof(Smem) + 1024; }
 // arrive on the leader's tmem_empty, and only then convert and store to C,
 // while the code and scale producers, which run ahead by the ring's depth,
 // and the MMAs of the next tile proceed.  Each thread stores one row segment
-// (rows outside the group and columns past N skipped).
+// (rows outside the group and columns past N skipped) with cache-streaming
+// stores, so that C does not push out of L2 the operand tiles that the tiles
+// in flight share.
 //
 // Warp roles in both CTAs: warp 0 code-tile TMA producer; warp 1 scale-chunk
 // TMA producer; warp 2 TMEM allocator (leader: MMA issuer); warps 4-7 scale
@@ -660,7 +662,8 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                     uint8_t* dst = reinterpret_cast<uint8_t*>(C) + (row * N + col0) * 2;
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (col0 + 8 * j < N) st_v4(dst + 16 * j, make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]));
+                        if (col0 + 8 * j < N)
+                            st_v4_stream(dst + 16 * j, make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]));
                 }
             } else {
                 uint8_t* dst = reinterpret_cast<uint8_t*>(C) + (row * N + col0) * 4;
@@ -673,7 +676,8 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
                             if (col0 + 32 * c + 4 * j < N)
-                                st_v4(dst + 128 * c + 16 * j, make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
+                                st_v4_stream(dst + 128 * c + 16 * j,
+                                             make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
                     }
                 }
                 tc_fence_before();

@@ -86,6 +86,15 @@ cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t 
 // QAT backward (straight-through estimator); workspace of
 // qat_backward_workspace_bytes bytes.
 size_t qat_backward_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t r);
+// The LoRA gradients dA = alpha B^T dW, dB = alpha dW A^T in one pass over
+// dW (r <= 64); the workspace holds their fp32 partial sums.
+bool lora_grads_fused(int64_t r);
+size_t lora_grads_workspace_bytes(int64_t n, int64_t k, int64_t r, int sms);
+cudaError_t launch_lora_grads(const void* dw, const void* lora_a, const void* lora_b, int64_t n, int64_t k, int r,
+                              float alpha_over_r, void* da, void* db, void* workspace, uint32_t* err, int sms,
+                              cudaStream_t st);
+// SM count of the current device (0 if there is none)
+int current_sms();
 cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
                                 const void* lora_b, int64_t m, int64_t n, int64_t k, int64_t r, float alpha_over_r,
                                 void* dx, void* dw, void* da, void* db, void* ws, uint32_t* err, int sms,

@@ -100,13 +100,22 @@ cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t 
     return launch_pdl(transpose_bf16_kernel, grid, dim3(256), 0, st, (const uint16_t*)in, (uint16_t*)out, R, C);
 }
 
-// The skinny products dA [r, k] and dB [n, r] have few output tiles (r is
-// at most 256), so they split their contraction over the SMs and add fp32
-// partial sums in a second kernel; the workspace holds those partials (at
-// most kMaxSplits slices of each).  Every operand is read in the layout it
-// is stored in (the GEMM takes K-major or MN-major operands).
+// The skinny products dA [r, k] and dB [n, r]: for r <= 64 one kernel reads
+// each tile of dW once and issues both products from it (lora_grads.cu),
+// its workspace holding the fp32 partial sums; for larger r each is a
+// split-K bf16 GEMM (partials of at most kMaxSplits slices each).  Every
+// operand is read in the layout it is stored in (the GEMM takes K-major or
+// MN-major operands).
 size_t qat_backward_workspace_bytes(int64_t, int64_t n, int64_t k, int64_t r) {
+    if (lora_grads_fused(r)) return lora_grads_workspace_bytes(n, k, r, current_sms());
     return round_up((size_t)kMaxSplits * (size_t)(r * k) * 4) + round_up((size_t)kMaxSplits * (size_t)(n * r) * 4);
+}
+
+int current_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms;
 }
 
 cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_fq, const void* lora_a,
@@ -129,14 +138,20 @@ cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_
     e = launch_gemm_bf16(dy, true, x_fq, true, n, k, m, 1.0f, dw, err, st);
     // dX [m, k] = dY Wfq: contraction over n; dY [m, n] K-major, Wfq [n, k] MN-major
     if (e == cudaSuccess) e = launch_gemm_bf16(dy, false, w_fq, true, m, k, n, 1.0f, dx, err, f->side);
-    // dA [r, k] = (alpha / r) B^T dW: contraction over n; B [n, r] and dW [n, k] MN-major
-    if (e == cudaSuccess)
-        e = launch_gemm_bf16_splitk(lora_b, true, dw, true, r, k, n, alpha_over_r, da, part_a,
-                                    bf16_split_count(r, k, n, sms), err, st);
-    // dB [n, r] = (alpha / r) dW A^T: contraction over k; dW [n, k] and A [r, k] K-major
-    if (e == cudaSuccess)
-        e = launch_gemm_bf16_splitk(dw, false, lora_a, false, n, r, k, alpha_over_r, db, part_b,
-                                    bf16_split_count(n, r, k, sms), err, st);
+    if (lora_grads_fused(r)) {
+        // dA and dB from one pass over dW (each tile read once, both products issued from it)
+        if (e == cudaSuccess)
+            e = launch_lora_grads(dw, lora_a, lora_b, n, k, (int)r, alpha_over_r, da, db, ws, err, sms, st);
+    } else {
+        // dA [r, k] = (alpha / r) B^T dW: contraction over n; B [n, r] and dW [n, k] MN-major
+        if (e == cudaSuccess)
+            e = launch_gemm_bf16_splitk(lora_b, true, dw, true, r, k, n, alpha_over_r, da, part_a,
+                                        bf16_split_count(r, k, n, sms), err, st);
+        // dB [n, r] = (alpha / r) dW A^T: contraction over k; dW [n, k] and A [r, k] K-major
+        if (e == cudaSuccess)
+            e = launch_gemm_bf16_splitk(dw, false, lora_a, false, n, r, k, alpha_over_r, db, part_b,
+                                        bf16_split_count(n, r, k, sms), err, st);
+    }
     // the join is made on every path, so a capture is never left forked
     cudaError_t j = cudaEventRecord(f->join, f->side);
     if (j == cudaSuccess) j = cudaStreamWaitEvent(st, f->join, 0);

@@ -304,18 +304,33 @@ __device__ __forceinline__ void nvfp4_encode_unit(const Unit& v, float g, bool g
     const float S = code < 127u ? __fmul_rn(s_dec[code], g) : __fmul_rn(e4m3_to_f32(code), g);
     uint32_t packed[2] = {0u, 0u};
     if (S != 0.0f) {
+        bool exact = true;
         if (g_ok && reciprocal_ok(S) && code < 127u) {
             // fp32(inv(code) * fp32(1/g)) is within 2^-22 of 1/S, close
-            // enough for the bracket (bracket_from_reciprocal)
+            // enough for the bracket (bracket_from_reciprocal); the unit's
+            // 16 products with each bracket end are formed in pairs, and the
+            // unit falls back to divisions only if any code differs
             const QuotientBracket br = bracket_from_reciprocal(S, __fmul_rn(s_inv[code], rg));
+            const uint64_t lo2 = pack2(br.lo, br.lo), hi2 = pack2(br.hi, br.hi);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                packed[j >> 2] |= e2m1x2_of_quotients(bf16_lo(v.w[j]), bf16_hi(v.w[j]), br) << (8 * (j & 3));
+            for (int h = 0; h < 2; ++h) {
+                const uint64_t x0 = bf16x2_pair(v.w[4 * h]), x1 = bf16x2_pair(v.w[4 * h + 1]),
+                               x2 = bf16x2_pair(v.w[4 * h + 2]), x3 = bf16x2_pair(v.w[4 * h + 3]);
+                packed[h] = e2m1x8_of_pairs(mul2(x0, lo2), mul2(x1, lo2), mul2(x2, lo2), mul2(x3, lo2));
+                const uint32_t up = e2m1x8_of_pairs(mul2(x0, hi2), mul2(x1, hi2), mul2(x2, hi2), mul2(x3, hi2));
+                exact = exact && packed[h] == up;
+            }
         } else {
+            exact = false;
+        }
+        if (!exact) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t byte = f32x2_to_e2m1x2(__fdiv_rn(bf16_lo(v.w[j]), S), __fdiv_rn(bf16_hi(v.w[j]), S));
-                packed[j >> 2] |= byte << (8 * (j & 3));
+            for (int h = 0; h < 2; ++h) {
+                uint64_t q[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    q[j] = pack2(__fdiv_rn(bf16_lo(v.w[4 * h + j]), S), __fdiv_rn(bf16_hi(v.w[4 * h + j]), S));
+                packed[h] = e2m1x8_of_pairs(q[0], q[1], q[2], q[3]);
             }
         }
     }

@@ -195,3 +195,73 @@ def test_gemm_bf16_splitk_rejects_small_workspace(fpq):
         fpq.fpq_gemm_bf16_splitk(t, 0, t, 0, 64, 64, 64, 1.0, t, ws)
     with pytest.raises(fpq.FpqError):
         fpq.fpq_gemm_bf16_splitk(t, 0, t, 0, 64, 64, 64, 1.0, t, None)
+
+
+def _lora_grads(fpq, dw, a, b, n, k, r, aor):
+    da = torch.empty((r, k), dtype=torch.bfloat16, device="cuda")
+    db = torch.empty((n, r), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((fpq.fpq_qat_lora_grads_workspace_bytes(n, k, r),), dtype=torch.uint8, device="cuda")
+    fpq.fpq_qat_lora_grads(dw, a, b, n, k, r, aor, da, db, ws)
+    return da, db
+
+
+@pytest.mark.parametrize("n,k,r", [(8, 8, 8), (272, 136, 16), (136, 1000, 8), (2048, 7168, 16), (520, 264, 64),
+                                   (7168, 2048, 32), (200, 8200, 24), (128, 128, 40)])
+def test_qat_lora_grads(fpq, orc, n, k, r):
+    """dA = (alpha/r) B^T dW and dB = (alpha/r) dW A^T from one pass over
+    dW: ragged strips of 128 rows, ragged K tiles, every r the fused kernel
+    takes (multiples of 8 up to 64)."""
+    dw, a, b = rand((n, k), 980 + n, std=0.05), rand((r, k), 981 + r, std=0.01), rand((n, r), 982 + k, std=0.01)
+    da, db = _lora_grads(fpq, dev(dw), dev(a), dev(b), n, k, r, 2.0)
+    assert fpq.fpq_get_device_error() == 0
+    check(da, orc.gemm_bf16_full(np.ascontiguousarray(b.T), np.ascontiguousarray(dw.T), 2.0), orc, "da")
+    check(db, orc.gemm_bf16_full(dw, a, 2.0), orc, "db")
+
+
+def test_qat_lora_grads_integer_exact(fpq, orc):
+    """Entries in {-1, 0, 1}: every partial sum over dW's rows (dA, up to
+    2048 terms split by 128-row strips) and over its columns (dB, 4096 terms
+    split by K ranges) is an exact integer in fp32, so the outputs must be
+    the round-to-nearest-even bf16 of alpha times the exact sums; a strip or
+    K range lost or added twice changes them."""
+    rng = np.random.default_rng(33)
+    n, k, r = 2048, 4096, 16
+    idw, ia, ib = rng.integers(-1, 2, (n, k)), rng.integers(-1, 2, (r, k)), rng.integers(-1, 2, (n, r))
+    bf = lambda v: workloads.as_u16(torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16))
+    da, db = _lora_grads(fpq, dev(bf(idw)), dev(bf(ia)), dev(bf(ib)), n, k, r, 0.25)
+    assert np.array_equal(workloads.as_u16(da), orc.bf16_round(0.25 * (ib.T @ idw).astype(np.float64)))
+    assert np.array_equal(workloads.as_u16(db), orc.bf16_round(0.25 * (idw @ ia.T).astype(np.float64)))
+
+
+def test_qat_lora_grads_repeatable(fpq):
+    n, k, r = 2048, 7168, 16
+    dw, a, b = dev(rand((n, k), 990, std=0.05)), dev(rand((r, k), 991)), dev(rand((n, r), 992))
+    da1, db1 = _lora_grads(fpq, dw, a, b, n, k, r, 2.0)
+    da2, db2 = _lora_grads(fpq, dw, a, b, n, k, r, 2.0)
+    assert torch.equal(da1.view(torch.int16), da2.view(torch.int16))
+    assert torch.equal(db1.view(torch.int16), db2.view(torch.int16))
+
+
+def test_qat_lora_grads_rejects_bad_args(fpq):
+    t = torch.zeros(128, 128, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((fpq.fpq_qat_lora_grads_workspace_bytes(128, 128, 64),), dtype=torch.uint8, device="cuda")
+    for r in (12, 72, 0):                   # not a multiple of 8, or outside [8, 64]
+        with pytest.raises(fpq.FpqError):
+            fpq.fpq_qat_lora_grads(t, t, t, 128, 128, r, 1.0, t, t, ws)
+    with pytest.raises(fpq.FpqError):       # k not a multiple of 8
+        fpq.fpq_qat_lora_grads(t, t, t, 128, 124, 8, 1.0, t, t, ws)
+    small = ws[:fpq.fpq_qat_lora_grads_workspace_bytes(128, 128, 8) - 16]
+    with pytest.raises(fpq.FpqError):
+        fpq.fpq_qat_lora_grads(t, t, t, 128, 128, 8, 1.0, t, t, small)
+
+
+@pytest.mark.parametrize("r", [64, 72])
+def test_qat_backward_rank_paths(fpq, orc, r):
+    """r = 64 takes the fused dA/dB pass, r = 72 the two split-K GEMMs."""
+    m, n, k = 256, 272, 520
+    dy, x_fq, w_fq, a, b = _qat_inputs(m, n, k, r, 1000 + r)
+    dx, dw, da, db = fpq.qat_backward(dev(dy), dev(x_fq), dev(w_fq), dev(a), dev(b), 2.0)
+    rdx, rdw, rda, rdb = orc.qat_backward(dy, x_fq, w_fq, a, b, 2.0)
+    for got, ref, what in ((dx, rdx, "dx"), (dw, rdw, "dw"), (da, rda, "da"), (db, rdb, "db")):
+        check(got, ref, orc, what)
+    assert fpq.fpq_get_device_error() == 0

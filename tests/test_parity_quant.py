@@ -261,8 +261,11 @@ def test_moe_prequant_full_size_batch(fpq, orc):
 
 # ------------------------------------------------------------------ LoRA merge + fake-quant
 
-@pytest.mark.parametrize("n,k,r", [(256, 384, 16), (200, 256, 1), (130, 512, 64), (1, 128, 3), (133, 256, 3), (200, 384, 5)])
+@pytest.mark.parametrize("n,k,r", [(256, 384, 16), (200, 256, 1), (130, 512, 64), (1, 128, 3), (133, 256, 3), (200, 384, 5),
+                                   (384, 256, 8), (136, 384, 24), (256, 128, 32), (129, 256, 40)])
 def test_lora_merge_fakequant_small(fpq, orc, n, k, r):
+    """Every padded rank the kernel instantiates (8, 16, 32, 64) and ranks
+    below them (zero-padded), ragged last block rows."""
     w = rand((n, k), 40, std=0.02)
     a = rand((r, k), 41, std=0.01)
     b = rand((n, r), 42, std=0.01)
