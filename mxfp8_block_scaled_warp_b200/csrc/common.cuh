@@ -265,6 +265,14 @@ __device__ __forceinline__ bool reciprocal_ok(float s) { return s >= 1.17549435e
 // pair of 15-bit magnitudes (integer order = magnitude order for finite
 // values; NaN patterns order above infinity, so a NaN propagates).
 __device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7FFF7FFFu; }
+// Per half: a value whose magnitude is the larger of the two magnitudes
+// (sign bits to be masked off by the caller), NaN if either is NaN.  One
+// bf16x2 max-of-magnitudes instruction instead of a mask and an integer max.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 __device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) { return __vmaxu2(a, b); }
 __device__ __forceinline__ uint32_t hmax2(uint32_t a) { return max(a & 0xFFFFu, a >> 16); }
 

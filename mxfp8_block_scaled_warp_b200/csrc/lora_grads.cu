@@ -35,7 +35,6 @@ namespace {
 using namespace sm100;
 
 constexpr int TK = 128;                       // K tile (columns of dW) and strip height (rows of dW)
-constexpr int STAGES = 4;
 constexpr int DW_TILE = TK * TK * 2;          // 32 KB: two boxes of 64 columns x 128 rows
 constexpr int DW_BOX = DW_TILE / 2;
 constexpr int MAX_RP = 64;                    // padded rank handled here
@@ -43,12 +42,19 @@ constexpr int NUM_THREADS = 256;
 constexpr int EPI_WARP0 = 4;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
+// Ring depth: as many 32 KB tiles of dW (plus A's tile) in flight as shared
+// memory holds, so that a CTA's K range (about six tiles when the strips x
+// K ranges fill the SMs) is requested from HBM almost at once.
+__host__ __device__ constexpr int ring_stages(int rp) { return rp <= 16 ? 6 : rp <= 32 ? 5 : 4; }
+
+template <int RP>
 struct __align__(1024) Smem {
-    uint8_t dw[STAGES][DW_TILE];
-    uint8_t a[STAGES][2 * MAX_RP * 128];      // A's K tile: two boxes of 64 columns x RP rows
-    uint8_t bt[2 * MAX_RP * 128];             // B^T of the strip: two boxes of 64 rows-of-dW x RP rows
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    static constexpr int ST = ring_stages(RP);
+    uint8_t dw[ST][DW_TILE];
+    uint8_t a[ST][2 * RP * 128];              // A's K tile: two boxes of 64 columns x RP rows
+    uint8_t bt[2 * RP * 128];                 // B^T of the strip: two boxes of 64 rows-of-dW x RP rows
+    uint64_t full[ST];
+    uint64_t empty[ST];
     uint64_t da_full[2];
     uint64_t da_empty[2];
     uint64_t db_full;
@@ -115,7 +121,8 @@ lora_grads_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                   const uint16_t* __restrict__ lora_b, int64_t n, int64_t k, int r, int splits, int kts,
                   float* __restrict__ part_a, float* __restrict__ part_b, uint32_t* err) {
     extern __shared__ uint8_t smem_raw[];
-    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<RP>& sm = *reinterpret_cast<Smem<RP>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int STAGES = Smem<RP>::ST;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int strip = (int)blockIdx.x / splits, split = (int)blockIdx.x - strip * splits;
     const int64_t n0 = (int64_t)strip * TK;
@@ -260,6 +267,7 @@ lora_grads_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
         }
     }
 
+    __syncwarp();     // the role warps' other lanes wait here for the elected lane, without polling
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -268,33 +276,61 @@ lora_grads_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     }
 }
 
+// sum_s p[s * stride + 0..3] for s = 0 .. S-1, added in s order; the
+// partial vectors are loaded eight at a time so their L2 round trips overlap
+__device__ __forceinline__ float4 ordered_sum4(const float* p, int64_t stride, int S) {
+    float4 acc = __ldcg(reinterpret_cast<const float4*>(p));
+    for (int s0 = 1; s0 < S; s0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (s0 + u < S) v[u] = __ldcg(reinterpret_cast<const float4*>(p + (int64_t)(s0 + u) * stride));
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (s0 + u < S) {
+                acc.x = __fadd_rn(acc.x, v[u].x);
+                acc.y = __fadd_rn(acc.y, v[u].y);
+                acc.z = __fadd_rn(acc.z, v[u].z);
+                acc.w = __fadd_rn(acc.w, v[u].w);
+            }
+    }
+    return acc;
+}
+
 // dA[j][c] = bf16(alpha * sum_s part_a[s][c][j]) and dB[row][j] =
-// bf16(alpha * sum_s part_b[s][row][j]), s ascending; one output per thread.
+// bf16(alpha * sum_s part_b[s][row][j]), s ascending; one thread per four
+// consecutive ranks of one column of dA or one row of dB (r is a multiple
+// of 8, rows of the partials are rp floats, rp a multiple of 16).
 __global__ void __launch_bounds__(256)
 lora_grads_reduce_kernel(const float* __restrict__ part_a, const float* __restrict__ part_b, int strips,
                          int splits, int64_t n, int64_t k, int r, int rp, float alpha, uint16_t* __restrict__ da,
                          uint16_t* __restrict__ db) {
     pdl_trigger();
     pdl_wait();
-    const int64_t na = k * r, total = na + n * r;
+    const int rq = r / 4;
+    const int64_t na = k * rq, total = na + n * rq;
     for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < total; i += (int64_t)gridDim.x * 256) {
         if (i < na) {
-            const int64_t c = i / r;
-            const int j = (int)(i - c * r);
-            float acc = __ldcg(part_a + c * rp + j);
-            for (int s = 1; s < strips; ++s) acc = __fadd_rn(acc, __ldcg(part_a + ((int64_t)s * k + c) * rp + j));
-            da[(int64_t)j * k + c] = (uint16_t)f32_to_bf16(__fmul_rn(acc, alpha));
+            const int64_t c = i / rq;
+            const int j = 4 * (int)(i - c * rq);
+            const float4 a = ordered_sum4(part_a + c * rp + j, k * rp, strips);
+            da[(int64_t)j * k + c] = (uint16_t)f32_to_bf16(__fmul_rn(a.x, alpha));
+            da[(int64_t)(j + 1) * k + c] = (uint16_t)f32_to_bf16(__fmul_rn(a.y, alpha));
+            da[(int64_t)(j + 2) * k + c] = (uint16_t)f32_to_bf16(__fmul_rn(a.z, alpha));
+            da[(int64_t)(j + 3) * k + c] = (uint16_t)f32_to_bf16(__fmul_rn(a.w, alpha));
         } else {
-            const int64_t e = i - na, row = e / r;
-            const int j = (int)(e - row * r);
-            float acc = __ldcg(part_b + row * rp + j);
-            for (int s = 1; s < splits; ++s) acc = __fadd_rn(acc, __ldcg(part_b + ((int64_t)s * n + row) * rp + j));
-            db[row * r + j] = (uint16_t)f32_to_bf16(__fmul_rn(acc, alpha));
+            const int64_t e = i - na, row = e / rq;
+            const int j = 4 * (int)(e - row * rq);
+            const float4 b = ordered_sum4(part_b + row * rp + j, n * rp, splits);
+            *reinterpret_cast<uint2*>(db + row * r + j) =
+                make_uint2(f32x2_to_bf16x2(__fmul_rn(b.x, alpha), __fmul_rn(b.y, alpha)),
+                           f32x2_to_bf16x2(__fmul_rn(b.z, alpha), __fmul_rn(b.w, alpha)));
         }
     }
 }
 
-int smem_bytes() { return (int)sizeof(Smem) + 1024; }
+template <int RP>
+int smem_bytes() { return (int)sizeof(Smem<RP>) + 1024; }
 
 inline int pad16(int r) { return (r + 15) / 16 * 16; }
 
@@ -320,7 +356,8 @@ cudaError_t launch_rp(const void* dw, const void* a, const void* b, int64_t n, i
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(lora_grads_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes());
+        e = cudaFuncSetAttribute(lora_grads_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem_bytes<RP>());
         if (e != cudaSuccess) return e;
         configured[dev] = 1;
     }
@@ -335,10 +372,10 @@ cudaError_t launch_rp(const void* dw, const void* a, const void* b, int64_t n, i
     float* part_a = static_cast<float*>(ws);
     float* part_b = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                              ((size_t)p.strips * (size_t)k * RP * 4 + 255) / 256 * 256);
-    e = launch_pdl(lora_grads_kernel<RP>, dim3((unsigned)(p.strips * p.splits)), dim3(NUM_THREADS), smem_bytes(), st,
-                   tw, ta, (const uint16_t*)b, n, k, r, p.splits, p.kts, part_a, part_b, err);
+    e = launch_pdl(lora_grads_kernel<RP>, dim3((unsigned)(p.strips * p.splits)), dim3(NUM_THREADS),
+                   smem_bytes<RP>(), st, tw, ta, (const uint16_t*)b, n, k, r, p.splits, p.kts, part_a, part_b, err);
     if (e != cudaSuccess) return e;
-    const int64_t total = (n + k) * r;
+    const int64_t total = (n + k) * (r / 4);
     const int grid = (int)min64((total + 255) / 256, (int64_t)(sms > 0 ? sms : 1) * 8);
     return launch_pdl(lora_grads_reduce_kernel, dim3((unsigned)grid), dim3(256), 0, st, (const float*)part_a,
                       (const float*)part_b, p.strips, p.splits, n, k, r, RP, alpha, (uint16_t*)da, (uint16_t*)db);

@@ -16,11 +16,14 @@ __device__ __forceinline__ Unit load_unit(const uint4* x, int64_t u) {
     return Unit{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
 }
 
+// Largest magnitude pattern of the unit's 16 values (15 bits; a NaN
+// anywhere gives a NaN pattern, which every caller treats as NaN whatever
+// its payload).
 __device__ __forceinline__ uint32_t unit_absmax(const Unit& v) {
-    uint32_t m = abs2(v.w[0]);
+    uint32_t m = absmax_bf16x2(v.w[0], v.w[1]);
 #pragma unroll
-    for (int i = 1; i < 8; ++i) m = max2(m, abs2(v.w[i]));
-    return hmax2(m);
+    for (int i = 2; i < 8; ++i) m = absmax_bf16x2(m, v.w[i]);
+    return hmax2(abs2(m));
 }
 
 // Reduce a magnitude pattern over `width` adjacent lanes (power of two).
