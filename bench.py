@@ -27,6 +27,7 @@ sample of the workload per step.
 from __future__ import annotations
 
 import argparse
+import glob
 import hashlib
 import json
 import os
@@ -741,6 +742,8 @@ class Dequant(Step):
         self.quant_bytes = self.mx_bytes + self.nv_bytes + self.a_bytes + self.b_bytes
         self.launches = 8
         self.config = dict(self.CONFIG)
+        if experts != 64:
+            self.config["workload"] = self.CONFIG["workload"].replace("64 experts", f"{experts} experts")
 
     @property
     def work(self) -> float:
@@ -808,11 +811,20 @@ def _source_hash(kernel: str) -> str | None:
            "gemm_mxfp8": "gemm_mxfp8.cu", "quant_fp8_1x128": "quant_kernels.cu",
            "quant_mxfp8": "quant_kernels.cu", "lora_merge_fq": "merge_kernel.cu",
            "gemm_nvfp4": "gemm_nvfp4.cu", "gemm_bf16_dx": "gemm_bf16.cu",
-           "moe_dispatch_mxfp8": "moe_dispatch.cu", "lora_grads": "lora_grads.cu"}.get(kernel)
+           "moe_dispatch_mxfp8": "moe_dispatch.cu", "lora_grads": "lora_grads.cu",
+           "quant_nvfp4": "quant_kernels.cu", "quant_fp8_128x128": "quant_kernels.cu",
+           "dequant_mxfp8": "quant_kernels.cu"}.get(kernel)
     if not src:
         return None
-    with open(os.path.join(ROOT, "mxfp8_block_scaled_warp_b200", "csrc", src), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    # the kernel's source file and every header of the library (a change in
+    # a shared device helper changes the kernel too)
+    csrc = os.path.join(ROOT, "mxfp8_block_scaled_warp_b200", "csrc")
+    h = hashlib.sha256()
+    for path in [os.path.join(csrc, src)] + sorted(glob.glob(os.path.join(csrc, "*.cuh")) +
+                                                   glob.glob(os.path.join(csrc, "*.h"))):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def _traffic(kernel: str, workload: str):
@@ -1152,8 +1164,8 @@ def main():
     dev = torch.device("cuda", local)
     pg = init_replicas(world, "nccl", dev)
 
-    if args.experts and args.workload != "moe_prequant":
-        raise SystemExit("--experts applies to --workload moe_prequant only")
+    if args.experts and args.workload not in ("moe_prequant", "dequant"):
+        raise SystemExit("--experts applies to --workload moe_prequant and dequant only")
     step = STEPS[args.workload](fpq, dev, **({"experts": args.experts} if args.experts else {}))
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
