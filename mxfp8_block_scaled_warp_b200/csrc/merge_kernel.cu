@@ -14,7 +14,8 @@ namespace fpq {
 namespace {
 
 constexpr int kMaxRank = 64;
-constexpr int MT = 256;                         // 16 row groups x 16 column groups of threads
+constexpr int RPT = 4;                          // rows of a block per thread
+constexpr int MT = 16 * (128 / RPT);            // 128 / RPT row groups x 16 column groups of threads
 constexpr int kWBytes = 128 * 128 * 2;          // the block of W in shared memory
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -25,8 +26,8 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// One CTA per 128x128 block of W; thread (ty, tx) owns rows 8 ty .. 8 ty + 7
-// and columns 8 tx .. 8 tx + 7 of the block.  The rank is padded to R (8,
+// One CTA per 128x128 block of W; thread (ty, tx) owns rows RPT ty .. RPT ty
+// + RPT - 1 and columns 8 tx .. 8 tx + 7 of the block.  The rank is padded to R (8,
 // 16, 32 or 64) with zero rows of A and columns of B: the padded terms add
 // +0 to a running sum that is never -0 (it starts at +0, and a round-to-
 // nearest sum is -0 only when both addends are), so they change nothing.
@@ -36,8 +37,8 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // ([R][128] pairs), and A's columns of the block as fp32 ([R][128], each
 // row stored as two 64-column halves so that a thread's 4-column loads of
 // one half are contiguous across the 16 column groups).  Per rank step j
-// a thread loads 8 pairs of B and 8 values of A (6 shared loads) and
-// issues 32 paired fmas (64 fmas), j ascending from zero as the
+// a thread loads RPT pairs of B and 8 values of A (RPT / 2 + 2 shared
+// loads) and issues 4 RPT paired fmas, j ascending from zero as the
 // definition states.
 template <int R>
 __global__ void __launch_bounds__(MT, 2)
@@ -54,10 +55,10 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     const int rmax = (int)min64(128, n - row0);
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
 
-    // W: this thread's 8 rows x 16 bytes, into shared memory behind the delta
+    // W: this thread's RPT rows x 16 bytes, into shared memory behind the delta
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rr = 8 * ty + i;
+    for (int i = 0; i < RPT; ++i) {
+        const int rr = RPT * ty + i;
         if (rr < rmax) cp_async16(sW + rr * 128 + 8 * tx, w + (row0 + rr) * k + col0 + 8 * tx);
     }
     // A: R rows of the block's 128 columns, 16-byte loads (zero rows past r)
@@ -73,14 +74,16 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
             *reinterpret_cast<float4*>(dst + 64) = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
         }
     }
-    // B: thread (row = tid % 128, half = tid / 128) takes ranks half * R/2 ..;
-    // consecutive threads write consecutive pairs of one rank row
+    // B: thread (row = tid % 128, part = tid / 128) takes ranks part * R/P
+    // .. (P = MT / 128 parts); consecutive threads write consecutive pairs of
+    // one rank row
     {
-        const int row = tid & 127, j0 = (tid >> 7) * (R / 2);
+        constexpr int P = MT / 128;
+        const int row = tid & 127, j0 = (tid >> 7) * (R / P);
         const bool row_ok = row < rmax;
         const uint16_t* brow = b + (row0 + row) * r;
 #pragma unroll
-        for (int jj = 0; jj < R / 2; ++jj) {
+        for (int jj = 0; jj < R / P; ++jj) {
             const int j = j0 + jj;
             const float f = (row_ok && j < r) ? __uint_as_float((uint32_t)brow[j] << 16) : 0.0f;
             sB2[j * 128 + row] = pack2(f, f);
@@ -88,21 +91,26 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     }
     __syncthreads();
 
-    uint64_t acc[8][4];
+    uint64_t acc[RPT][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < RPT; ++i)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[i][e] = 0;
 #pragma unroll 16
     for (int j = 0; j < R; ++j) {
-        const ulonglong2* bp = reinterpret_cast<const ulonglong2*>(sB2 + j * 128 + 8 * ty);
-        const ulonglong2 b0 = bp[0], b1 = bp[1], b2 = bp[2], b3 = bp[3];
+        const ulonglong2* bp = reinterpret_cast<const ulonglong2*>(sB2 + j * 128 + RPT * ty);
+        uint64_t bb[RPT];
+#pragma unroll
+        for (int h = 0; h < RPT / 2; ++h) {
+            const ulonglong2 bv = bp[h];
+            bb[2 * h] = bv.x;
+            bb[2 * h + 1] = bv.y;
+        }
         const ulonglong2 a0 = *reinterpret_cast<const ulonglong2*>(sA + j * 128 + 4 * tx);
         const ulonglong2 a1 = *reinterpret_cast<const ulonglong2*>(sA + j * 128 + 64 + 4 * tx);
-        const uint64_t bb[8] = {b0.x, b0.y, b1.x, b1.y, b2.x, b2.y, b3.x, b3.y};
         const uint64_t aa[4] = {a0.x, a0.y, a1.x, a1.y};
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < RPT; ++i)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][e] = fma2(bb[i], aa[e], acc[i][e]);
     }
@@ -110,18 +118,18 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     // merge, round to bf16, block amax
     cp_async_wait_all();     // this thread's own copies of W
     const uint64_t al2 = pack2(alpha_over_r, alpha_over_r);
-    uint32_t v[8][4];
+    uint32_t v[RPT][4];
     uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(sW + (8 * ty + i) * 128 + 8 * tx);
+    for (int i = 0; i < RPT; ++i) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(sW + (RPT * ty + i) * 128 + 8 * tx);
         const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const uint64_t x = fma2(al2, acc[i][e], pack2(bf16_lo(ww[e]), bf16_hi(ww[e])));
             v[i][e] = f32x2_to_bf16x2(lo_of(x), hi_of(x));
         }
-        if (8 * ty + i < rmax)
+        if (RPT * ty + i < rmax)
 #pragma unroll
             for (int e = 0; e < 4; ++e) m = max2(m, abs2(v[i][e]));
     }
@@ -145,8 +153,8 @@ lora_merge_fq_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict_
     // differ anywhere (a quotient near a rounding boundary), the row's 8
     // elements are encoded from correctly rounded divisions
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rr = 8 * ty + i;
+    for (int i = 0; i < RPT; ++i) {
+        const int rr = RPT * ty + i;
         if (rr < rmax) {
             uint2 cw;
             if (!fast || !e4m3x8_bracketed(v[i], lo2, hi2, cw)) cw = e4m3x8_divided(v[i], sc);

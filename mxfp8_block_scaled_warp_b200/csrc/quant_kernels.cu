@@ -447,39 +447,62 @@ __device__ __forceinline__ void store_bf16x16(uint4* out, int64_t u, const float
     st_v4(out + 2 * u + 1, make_uint4(h[4], h[5], h[6], h[7]));
 }
 
+// Units in flight per thread in the dequantizers: all of an iteration's
+// code (and scale) loads are issued before any unit is decoded.
+constexpr int kDqUnroll = 4;
+
 // fmt: 0 = 1x128 (fp32 scale per 8 units), 2 = MXFP8 (E8M0 per 2 units),
 // 1 = 128x128 (fp32 scale per 128x128 block).
+template <int kFmt>
+__device__ __forceinline__ float fp8_unit_scale(const void* __restrict__ scales, int64_t u, int64_t rows,
+                                                int64_t cols) {
+    if (kFmt == 2) {
+        const uint32_t code = ((const uint8_t*)scales)[u >> 1];
+        return code == 0xFFu ? __uint_as_float(0x7FC00000u)
+             : code == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(code << 23);
+    } else if (kFmt == 0) {
+        return ((const float*)scales)[u >> 3];
+    } else {
+        const int64_t units_per_row = cols / 16;
+        const int64_t row = u / units_per_row, colu = u - row * units_per_row;
+        const int64_t b = row / rows, r = row - b * rows;
+        const int64_t nbr = (rows + 127) / 128, nbc = cols / 128;
+        return ((const float*)scales)[(b * nbr + r / 128) * nbc + colu / 8];
+    }
+}
+
 template <int kFmt, bool S>
 __global__ void __launch_bounds__(kThreads, 3)
 dequant_fp8_kernel(const uint4* __restrict__ q, const void* __restrict__ scales, uint4* __restrict__ out,
                    int64_t units, int64_t rows, int64_t cols, UnitStrides m) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    const int64_t units_per_row = cols / 16;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
-        uint4 c = ld_stream(q + in_unit<S>(m, u));
-        float sc;
-        if (kFmt == 2) {
-            uint32_t code = ((const uint8_t*)scales)[u >> 1];
-            sc = code == 0xFFu ? __uint_as_float(0x7FC00000u)
-               : code == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(code << 23);
-        } else if (kFmt == 0) {
-            sc = ((const float*)scales)[u >> 3];
-        } else {
-            int64_t row = u / units_per_row, colu = u - row * units_per_row;
-            int64_t b = row / rows, r = row - b * rows;
-            int64_t nbr = (rows + 127) / 128, nbc = cols / 128;
-            sc = ((const float*)scales)[(b * nbr + r / 128) * nbc + colu / 8];
-        }
-        uint32_t w[4] = {c.x, c.y, c.z, c.w};
-        float f[16];
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kDqUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kDqUnroll + threadIdx.x; base < units; base += stride) {
+        uint4 c[kDqUnroll];
+        float sc[kDqUnroll];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float2 lo = e4m3x2_to_f32x2(w[j] & 0xFFFFu), hi = e4m3x2_to_f32x2(w[j] >> 16);
-            f[4 * j + 0] = lo.x * sc; f[4 * j + 1] = lo.y * sc;
-            f[4 * j + 2] = hi.x * sc; f[4 * j + 3] = hi.y * sc;
+        for (int i = 0; i < kDqUnroll; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) {
+                c[i] = ld_stream(q + in_unit<S>(m, u));
+                sc[i] = fp8_unit_scale<kFmt>(scales, u, rows, cols);
+            }
         }
-        store_bf16x16(out, out_unit<S>(m, u), f);
+#pragma unroll
+        for (int i = 0; i < kDqUnroll; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) {
+                const uint32_t w[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+                float f[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 lo = e4m3x2_to_f32x2(w[j] & 0xFFFFu), hi = e4m3x2_to_f32x2(w[j] >> 16);
+                    f[4 * j + 0] = lo.x * sc[i]; f[4 * j + 1] = lo.y * sc[i];
+                    f[4 * j + 2] = hi.x * sc[i]; f[4 * j + 3] = hi.y * sc[i];
+                }
+                store_bf16x16(out, out_unit<S>(m, u), f);
+            }
+        }
     }
 }
 
@@ -488,19 +511,33 @@ __global__ void __launch_bounds__(kThreads, 3)
 dequant_nvfp4_kernel(const uint2* __restrict__ q, const uint8_t* __restrict__ s, const float* __restrict__ g,
                      uint4* __restrict__ out, int64_t units, int64_t units_per_matrix, UnitStrides m) {
     pdl_trigger();   // dependents may launch now; they wait for this grid to finish
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units; u += stride) {
-        uint2 c = q[in_unit<S>(m, u)];
-        const float Sc = e4m3_to_f32(s[u]) * g[u / units_per_matrix];
-        uint32_t w[2] = {c.x, c.y};
-        float f[16];
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kDqUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kDqUnroll + threadIdx.x; base < units; base += stride) {
+        uint2 c[kDqUnroll];
+        float Sc[kDqUnroll];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float2 e = e2m1x2_to_f32x2((w[j >> 2] >> (8 * (j & 3))) & 0xFFu);
-            f[2 * j] = e.x * Sc;
-            f[2 * j + 1] = e.y * Sc;
+        for (int i = 0; i < kDqUnroll; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) {
+                c[i] = q[in_unit<S>(m, u)];
+                Sc[i] = e4m3_to_f32(s[u]) * g[u / units_per_matrix];
+            }
         }
-        store_bf16x16(out, out_unit<S>(m, u), f);
+#pragma unroll
+        for (int i = 0; i < kDqUnroll; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) {
+                const uint32_t w[2] = {c[i].x, c[i].y};
+                float f[16];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float2 e = e2m1x2_to_f32x2((w[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+                    f[2 * j] = e.x * Sc[i];
+                    f[2 * j + 1] = e.y * Sc[i];
+                }
+                store_bf16x16(out, out_unit<S>(m, u), f);
+            }
+        }
     }
 }
 
@@ -593,7 +630,7 @@ cudaError_t launch_dequantize(int fmt, const void* q, const void* scales, const 
                               int64_t batch, int64_t rows, int64_t cols, void* out, int sms, cudaStream_t st,
                               const OperandStrides* strides) {
     const int64_t units = batch * rows * cols / 16;
-    const int grid = grid_for(units, kThreads, sms);
+    const int grid = grid_for(units, kThreads * kDqUnroll, sms);
     bool sd = false;
     const UnitStrides m = unit_strides(strides, rows, cols, sd);
 #define FPQ_DEQ(F)                                                                                                \
