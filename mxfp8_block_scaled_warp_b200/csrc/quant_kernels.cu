@@ -437,6 +437,103 @@ quant_nvfp4_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint
     }
 }
 
+// One or two matrices: the persistent ordering buys no L2 reuse between
+// matrices, and an item's units walked one after another leave little in
+// flight, so the two passes are two launches instead: a streaming amax
+// kernel (kUnroll units in flight per thread, CTA reduction, one atomicMax
+// per matrix and CTA) and a grid-stride encode kernel whose launch follows
+// the amax kernel's completion in stream order (the input's second read
+// is mostly served by L2 at these sizes).  Workspace as above (only the
+// amax words are used).
+constexpr int NV_SMALL_BATCH = 2;
+
+template <bool S>
+__global__ void __launch_bounds__(kThreads, 3)
+nvfp4_amax_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint32_t* __restrict__ ws,
+                  UnitStrides m) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
+    __shared__ uint32_t s_wmax[NV_SMALL_BATCH][kThreads / 32];
+    const int64_t units = batch * upm;
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kUnroll;
+    uint32_t am0 = 0, am1 = 0;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kUnroll + threadIdx.x; base < units; base += stride) {
+        Unit v[kUnroll];
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) v[i] = load_unit(x, in_unit<S>(m, u));
+        }
+#pragma unroll
+        for (int i = 0; i < kUnroll; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) {
+                const uint32_t a = unit_absmax(v[i]);
+                if (u < upm) am0 = max(am0, a);
+                else am1 = max(am1, a);
+            }
+        }
+    }
+    am0 = group_max<32>(am0);
+    am1 = group_max<32>(am1);
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        s_wmax[0][warp] = am0;
+        s_wmax[1][warp] = am1;
+    }
+    __syncthreads();
+    if (threadIdx.x < batch) {
+        uint32_t mm = 0;
+#pragma unroll
+        for (int k = 0; k < kThreads / 32; ++k) mm = max(mm, s_wmax[threadIdx.x][k]);
+        if (mm) atomicMax(ws + 4 + threadIdx.x, mm);
+    }
+}
+
+template <bool S>
+__global__ void __launch_bounds__(kThreads, 4)
+nvfp4_encode_kernel(const uint4* __restrict__ x, int64_t batch, int64_t upm, uint2* __restrict__ q,
+                    uint8_t* __restrict__ s, float* __restrict__ g_out, const uint32_t* __restrict__ ws,
+                    UnitStrides m) {
+    pdl_trigger();   // dependents may launch now; they wait for this grid to finish
+    __shared__ ScaleTables tab6;                 // fp32(amax_b / 6) by mantissa
+    __shared__ float s_dec[128];                 // dec(c) for E4M3 codes c = 0..126
+    __shared__ float s_inv[128];                 // fp32(1 / dec(c)) for c = 1..126
+    init_scale_tables(tab6, 6.0f);
+    if (threadIdx.x < 128) {
+        const uint32_t c = threadIdx.x;
+        const float d = c == 127 ? 0.0f : e4m3_to_f32(c);
+        s_dec[c] = d;
+        s_inv[c] = (c == 0 || c == 127) ? 0.0f : __frcp_rn(d);
+    }
+    const float g0 = nvfp4_tensor_scale(__ldcg(ws + 4));
+    const float g1 = batch > 1 ? nvfp4_tensor_scale(__ldcg(ws + 5)) : 1.0f;
+    if (blockIdx.x == 0 && threadIdx.x < batch) g_out[threadIdx.x] = threadIdx.x == 0 ? g0 : g1;
+    __syncthreads();
+    const bool ok0 = reciprocal_ok(g0), ok1 = reciprocal_ok(g1);
+    const QuotientBracket gb0 = quotient_bracket(ok0 ? g0 : 1.0f), gb1 = quotient_bracket(ok1 ? g1 : 1.0f);
+    const float rg0 = __frcp_rn(ok0 ? g0 : 1.0f), rg1 = __frcp_rn(ok1 ? g1 : 1.0f);
+    const int64_t units = batch * upm;
+    constexpr int kIn = 2;                       // units in flight per thread
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kIn;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads * kIn + threadIdx.x; base < units; base += stride) {
+        Unit v[kIn];
+#pragma unroll
+        for (int i = 0; i < kIn; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) v[i] = load_unit(x, in_unit<S>(m, u));
+        }
+#pragma unroll
+        for (int i = 0; i < kIn; ++i) {
+            const int64_t u = base + (int64_t)i * kThreads;
+            if (u < units) {
+                const bool first = u < upm;
+                nvfp4_encode_unit(v[i], first ? g0 : g1, first ? ok0 : ok1, first ? gb0 : gb1, first ? rg0 : rg1,
+                                  tab6, s_dec, s_inv, q + out_unit<S>(m, u), s + u);
+            }
+        }
+    }
+}
+
 // ----------------------------------------------------------------- dequantize
 
 __device__ __forceinline__ void store_bf16x16(uint4* out, int64_t u, const float (&f)[16]) {
@@ -605,6 +702,20 @@ cudaError_t launch_quantize(int fmt, const void* x, int64_t batch, int64_t rows,
         uint32_t* ws = (uint32_t*)workspace;
         cudaError_t e = cudaMemsetAsync(ws, 0, nvfp4_workspace_words(batch) * sizeof(uint32_t), st);
         if (e != cudaSuccess) return e;
+        if (batch <= NV_SMALL_BATCH) {
+            const int ga = grid_for(units, kThreads * kUnroll, sms);
+            const int ge = (int)max64(1, min64((units + 2 * kThreads - 1) / (2 * kThreads), (int64_t)sms * 4));
+            if (sd) {
+                nvfp4_amax_kernel<true><<<ga, kThreads, 0, st>>>((const uint4*)x, batch, upm, ws, m);
+                nvfp4_encode_kernel<true><<<ge, kThreads, 0, st>>>((const uint4*)x, batch, upm, (uint2*)q,
+                                                                   (uint8_t*)scales, tensor_scale, ws, m);
+            } else {
+                nvfp4_amax_kernel<false><<<ga, kThreads, 0, st>>>((const uint4*)x, batch, upm, ws, m);
+                nvfp4_encode_kernel<false><<<ge, kThreads, 0, st>>>((const uint4*)x, batch, upm, (uint2*)q,
+                                                                    (uint8_t*)scales, tensor_scale, ws, m);
+            }
+            break;
+        }
         const int64_t slots = (int64_t)sms * NV_MIN_BLOCKS;
         int upt = NV_UNITS_PER_THREAD;
         while (upt > 1 && batch * ((upm + (int64_t)kThreads * upt - 1) / ((int64_t)kThreads * upt)) < 2 * slots) upt /= 2;
