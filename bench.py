@@ -193,23 +193,25 @@ class Step:
 
     def whole_step(self, side_stream):
         """One step as the timed graph and the end-to-end loop run it: the
-        kernels named in `side` forked onto `side_stream` (they overlap the
-        others' ramp-up and tail), the rest in order on the current stream."""
+        kernels named in `side` on `side_stream`, forked from the current
+        stream before the step's first kernel (so they run beside the kernels
+        listed before `join_before`, not after them), the rest in order on
+        the current stream, which waits for the side stream before
+        `join_before`."""
         cur = torch.cuda.current_stream()
-        forked = False
+        joined = not self.side
+        if self.side:
+            side_stream.wait_stream(cur)              # the step's inputs are ready on both streams
         for name, fn in self.kernels():
             if name in self.side:
-                if not forked:
-                    side_stream.wait_stream(cur)
-                    forked = True
                 with torch.cuda.stream(side_stream):
                     fn()
                 continue
-            if forked and name == self.join_before:
+            if not joined and name == self.join_before:
                 cur.wait_stream(side_stream)
-                forked = False
+                joined = True
             fn()
-        if forked:
+        if not joined:
             cur.wait_stream(side_stream)
 
 
@@ -578,6 +580,9 @@ class Nvfp4Gemm(Step):
               "m": 4096, "n": 2048, "k": 7168, "l2": "flushed before every step (256 MiB write)"}
     dtype = "e2m1xe2m1->f32 (bf16 in/out)"
     tensor_ratio = 4.0         # dense fp4 / bf16, nominal 9 / 2.25
+    side = ("quant_nvfp4_b",)          # B's quantizer runs beside A's
+    join_before = "gemm_nvfp4"
+    E2E_IN, E2E_OUT = ("a", "b"), ("c",)
 
     def __init__(self, fpq, dev, m=4096, n=2048, k=7168):
         self.f = fpq
@@ -620,8 +625,7 @@ class Nvfp4Gemm(Step):
     def e2e_step(self, stream, side_stream):
         self.a.copy_(self.a_host, non_blocking=True)
         self.b.copy_(self.b_host, non_blocking=True)
-        for _, fn in self.kernels():
-            fn()
+        self.whole_step(side_stream)
         self.c_host.copy_(self.c, non_blocking=True)
         return self.a_host.numel() * 2 + self.b_host.numel() * 2, self.c.numel() * 2
 

@@ -51,7 +51,50 @@ def test_reference_line(capsys):
 def test_launch_note_names_forked_kernels():
     note = bench.launch_note(object.__new__(bench.DsFp8Gemm))
     assert "quant_fp8_128x128 on a second stream" in note
-    assert "second stream" not in bench.launch_note(object.__new__(bench.Nvfp4Gemm))
+    assert "quant_nvfp4_b on a second stream" in bench.launch_note(object.__new__(bench.Nvfp4Gemm))
+    assert "second stream" not in bench.launch_note(object.__new__(bench.MoeGrouped))
+
+
+def test_whole_step_forks_side_kernels_before_the_first_kernel(monkeypatch):
+    """The side kernels must not wait for the kernels listed before them:
+    the side stream is forked from the current stream before the step's
+    first kernel, and joined back just before `join_before`."""
+    log = []
+
+    class FakeStream:
+        def __init__(self, name):
+            self.name = name
+
+        def wait_stream(self, other):
+            log.append(f"{self.name} waits {other.name}")
+
+    main, side = FakeStream("main"), FakeStream("side")
+    current = [main]
+
+    class Ctx:
+        def __init__(self, s):
+            self.s = s
+
+        def __enter__(self):
+            self.prev = current[0]
+            current[0] = self.s
+
+        def __exit__(self, *a):
+            current[0] = self.prev
+
+    monkeypatch.setattr(bench.torch.cuda, "current_stream", lambda: current[0])
+    monkeypatch.setattr(bench.torch.cuda, "stream", lambda s: Ctx(s))
+
+    class Step(bench.Step):
+        side = ("b",)
+        join_before = "g"
+
+        def kernels(self):
+            run = lambda n: (lambda: log.append(f"{n} on {current[0].name}"))
+            return [("a", run("a")), ("b", run("b")), ("g", run("g")), ("h", run("h"))]
+
+    Step().whole_step(side)
+    assert log == ["side waits main", "a on main", "b on side", "main waits side", "g on main", "h on main"]
 
 
 def test_traffic_only_for_unchanged_source(tmp_path, monkeypatch):
