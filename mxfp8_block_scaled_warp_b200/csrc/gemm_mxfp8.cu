@@ -647,13 +647,17 @@ gemm_mxfp8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             if (!c_f32) {
                 uint32_t h[64];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t r[16];
+                for (int c = 0; c < 8; c += 2) {
+                    // two loads in flight per wait: four TMEM round trips instead of eight
+                    uint32_t r[16], r2[16];
                     tmem_ld_32x32b_x16(taddr + (uint32_t)(16 * c), r);
+                    tmem_ld_32x32b_x16(taddr + (uint32_t)(16 * c + 16), r2);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
+                    for (int e = 0; e < 8; ++e) {
                         h[8 * c + e] = f32x2_to_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+                        h[8 * c + 8 + e] = f32x2_to_bf16x2(__uint_as_float(r2[2 * e]), __uint_as_float(r2[2 * e + 1]));
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
