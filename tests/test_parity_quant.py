@@ -230,6 +230,21 @@ def test_nvfp4_quant_and_dequant(fpq, orc, case):
     assert_same(host(out), orc.dequant_nvfp4(oq, os_, og), "dequantized bf16")
 
 
+@pytest.mark.parametrize("second", ["scaled", "zero"])
+def test_nvfp4_two_matrices(fpq, orc, second):
+    """Two matrices take the two-launch path (amax pass, then encode); the
+    second matrix has its own tensor scale (4x the first's spread, or an
+    all-zero matrix whose tensor scale is 1)."""
+    a = rand((96, 512), 35, std=0.02, outliers=0.01)
+    b = rand((96, 512), 36, std=0.08) if second == "scaled" else np.zeros((96, 512), np.uint16)
+    x = np.stack([a, b])
+    q, s, g = fpq.quantize(dev(x), fpq.NVFP4)
+    oq, os_, og = orc.quant_nvfp4(x)
+    assert_same(host(g), f32_bits(og), "tensor scales")
+    assert_same(host(s), os_, "E4M3 block scales")
+    assert_same(host(q), oq, "packed E2M1 codes")
+
+
 def test_nvfp4_batched_per_matrix_scale(fpq, orc):
     x = np.stack([rand((64, 128), 30 + i, std=0.02 * (i + 1)) for i in range(5)])
     q, s, g = fpq.quantize(dev(x), fpq.NVFP4)
