@@ -329,7 +329,9 @@ FPQ_API fpq_status fpq_transpose_bf16(const void* in, void* out, int64_t rows, i
  *               sums of da and db (for r <= 64 those of fpq_qat_lora_grads,
  *               sized for the current device's SM count; for larger r the
  *               split-K slices of two bf16 GEMMs, at most 16 each), added in
- *               a fixed order by a second kernel, so results are repeatable
+ *               a fixed order by a second kernel, so results are repeatable;
+ *               then the tile counters of the dX and dW products (zeroed by
+ *               the call), from which their persistent CTAs claim tiles
  *
  * The products are ordered on `stream` like any other work: dx, which no
  * other product needs, runs on a library-owned second stream forked from

@@ -48,8 +48,11 @@ cudaError_t launch_gemm_nvfp4(const void* aq, const void* as, const float* ag, c
 
 // C = alpha P Q^T, C [m, n] bf16.  P is [m, k] (K-major) or, with p_mn,
 // stored as [k, m] (MN-major); likewise Q [n, k] or, with q_mn, [k, n].
+// tile_counter: a zeroed device int from which the persistent CTAs claim
+// tiles (for products that share the GPU with another); nullptr: CTA c
+// takes tiles c, c + grid, ...
 cudaError_t launch_gemm_bf16(const void* p, bool p_mn, const void* q, bool q_mn, int64_t m, int64_t n, int64_t k,
-                             float alpha, void* c, uint32_t* err, cudaStream_t st);
+                             float alpha, void* c, uint32_t* err, cudaStream_t st, int* tile_counter = nullptr);
 
 // Split-K variant for products with few output tiles: fp32 partial sums of
 // `splits` K slices in `partial` ([splits, m, n] fp32), then a reduce kernel

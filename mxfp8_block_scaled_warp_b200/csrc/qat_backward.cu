@@ -106,9 +106,17 @@ cudaError_t launch_transpose_bf16(const void* in, void* out, int64_t R, int64_t 
 // split-K bf16 GEMM (partials of at most kMaxSplits slices each).  Every
 // operand is read in the layout it is stored in (the GEMM takes K-major or
 // MN-major operands).
-size_t qat_backward_workspace_bytes(int64_t, int64_t n, int64_t k, int64_t r) {
-    if (lora_grads_fused(r)) return lora_grads_workspace_bytes(n, k, r, current_sms());
+// The workspace ends with the two tile counters of the dX and dW products
+// (kCounterBytes, zeroed by the call), which share the GPU.
+constexpr size_t kCounterBytes = 256;
+
+size_t grads_workspace_bytes(int64_t n, int64_t k, int64_t r) {
+    if (lora_grads_fused(r)) return round_up(lora_grads_workspace_bytes(n, k, r, current_sms()));
     return round_up((size_t)kMaxSplits * (size_t)(r * k) * 4) + round_up((size_t)kMaxSplits * (size_t)(n * r) * 4);
+}
+
+size_t qat_backward_workspace_bytes(int64_t, int64_t n, int64_t k, int64_t r) {
+    return grads_workspace_bytes(n, k, r) + kCounterBytes;
 }
 
 int current_sms() {
@@ -132,12 +140,19 @@ cudaError_t launch_qat_backward(const void* dy, const void* x_fq, const void* w_
     Fork* f = nullptr;
     cudaError_t e = fork_state(&f);
     if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + grads_workspace_bytes(n, k, r), 0, 2 * sizeof(int), st)) !=
+        cudaSuccess)
+        return e;
     if ((e = cudaEventRecord(f->fork, st)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(f->side, f->fork, 0)) != cudaSuccess) return e;
+    // Both products claim their tiles from counters (zeroed here, on st
+    // before the fork is taken), so that dX's CTAs, which start on the SMs
+    // dW's finish, take only the tiles that are left.
+    int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + grads_workspace_bytes(n, k, r));
     // dW [n, k] = dY^T Xfq: contraction over m; dY [m, n] and Xfq [m, k] MN-major
-    e = launch_gemm_bf16(dy, true, x_fq, true, n, k, m, 1.0f, dw, err, st);
+    e = launch_gemm_bf16(dy, true, x_fq, true, n, k, m, 1.0f, dw, err, st, counters);
     // dX [m, k] = dY Wfq: contraction over n; dY [m, n] K-major, Wfq [n, k] MN-major
-    if (e == cudaSuccess) e = launch_gemm_bf16(dy, false, w_fq, true, m, k, n, 1.0f, dx, err, f->side);
+    if (e == cudaSuccess) e = launch_gemm_bf16(dy, false, w_fq, true, m, k, n, 1.0f, dx, err, f->side, counters + 1);
     if (lora_grads_fused(r)) {
         // dA and dB from one pass over dW (each tile read once, both products issued from it)
         if (e == cudaSuccess)
