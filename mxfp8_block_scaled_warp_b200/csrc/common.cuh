@@ -50,17 +50,6 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
     return r;
 }
 
-// two fp32 -> two E2M1 codes in one byte, round to nearest even, saturating
-// to +-6; `lo` lands in bits 0..3.
-__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-        "cvt.u32.u8 %0, t;\n\t}"
-        : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
 // E4M3 code (low byte of `c`) -> fp32, exact (through the f16x2 converter).
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
     uint32_t h2;
@@ -205,14 +194,6 @@ __device__ __forceinline__ uint2 e4m3x8_divided(const uint32_t (&w)[4], float s)
 #pragma unroll
     for (int j = 0; j < 4; ++j) q[j] = pack2(__fdiv_rn(bf16_lo(w[j]), s), __fdiv_rn(bf16_hi(w[j]), s));
     return make_uint2(e4m3x4_of_pairs(q[0], q[1]), e4m3x4_of_pairs(q[2], q[3]));
-}
-
-// E2M1 codes of fp32(x0/s) (bits 0-3) and fp32(x1/s) (bits 4-7).
-__device__ __forceinline__ uint32_t e2m1x2_of_quotients(float x0, float x1, const QuotientBracket& b) {
-    uint32_t lo = f32x2_to_e2m1x2(__fmul_rn(x0, b.lo), __fmul_rn(x1, b.lo));
-    const uint32_t hi = f32x2_to_e2m1x2(__fmul_rn(x0, b.hi), __fmul_rn(x1, b.hi));
-    if (lo != hi) lo = f32x2_to_e2m1x2(__fdiv_rn(x0, b.s), __fdiv_rn(x1, b.s));
-    return lo;
 }
 
 // ----------------------------------------------------------------- per-block scale tables
